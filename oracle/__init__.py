@@ -1,0 +1,255 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention forward.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference leg may import this package.  It shares no code
+with the CUDA library and never imports it.
+
+Contents
+--------
+``attention``                 the plain definition, in C (``attn_oracle.c``), fp64, one
+                              query row at a time.  Sources: "FlashAttention"
+                              (fp-ai-systems) section "The problem: the n x n score
+                              matrix"; "Flash Attention -- Module 12.3" section
+                              "Definition"; "FlashAttention 1-2-3" section "The Math
+                              Behind the Online Softmax Trick" (two-pass stable softmax).
+``online_softmax_attention``  the method's own algorithm restated in numpy fp64: keys in
+                              blocks, running max m and running sum l per row, the
+                              partial output rescaled by exp(m_old - m_new), one division
+                              by l at the end ("FlashAttention 1-2-3" sections
+                              "FlashAttention-1" and "The Math Behind the Online Softmax
+                              Trick"; "FlashAttention" section "Online softmax: the
+                              enabling trick").  An optional threshold tau keeps a stale
+                              max until the new one exceeds it by more than tau (log2
+                              units); the result is the same in exact arithmetic.
+``lse_combine``               merges partial results over disjoint key sets by their
+                              log-sum-exp, the reduction step of split-KV decoding
+                              ("FlashAttention 1-2-3" section "Beyond FlashAttention":
+                              partial softmax per KV chunk, then a reduction).
+``score_matrix_bytes``,       byte counts the pages print ("FlashAttention" section "The
+``standard_attention_traffic`` problem"; "FlashAttention 1-2-3" section "The Memory Wall").
+
+Parity status: every function above is pinned by ``tests/test_oracle.py`` (closed forms,
+invariants, brute force, a library routine, and the pages' printed byte counts).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libattn_oracle.so")
+_lib = None
+
+F64, F16, BF16 = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compiles attn_oracle.c with gcc (no fast-math) into libattn_oracle.so."""
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-Wall", "-fPIC", "-shared", "-pthread", _SRC,
+             "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = load_library(build())
+    return _lib
+
+
+def default_threads() -> int:
+    """Host threads the C oracle uses by default (the CPUs this process may run on)."""
+    return int(_load().attn_oracle_default_threads())
+
+
+def _as_bits(x):
+    """Returns (contiguous numpy array, dtype code) without changing any value."""
+    try:
+        import torch
+    except ImportError:  # pragma: no cover
+        torch = None
+    if torch is not None and isinstance(x, torch.Tensor):
+        x = x.detach().cpu().contiguous()
+        if x.dtype == torch.float16:
+            return x.view(torch.int16).numpy(), F16
+        if x.dtype == torch.bfloat16:
+            return x.view(torch.int16).numpy(), BF16
+        return x.to(torch.float64).numpy(), F64
+    a = np.ascontiguousarray(x)
+    if a.dtype == np.float16:
+        return a.view(np.int16), F16
+    return np.ascontiguousarray(a, dtype=np.float64), F64
+
+
+def load_library(path: str):
+    """Opens an oracle shared library built from attn_oracle.c (or a copy of it)."""
+    lib = ctypes.CDLL(path)
+    lib.attn_oracle_fwd.restype = ctypes.c_int
+    lib.attn_oracle_fwd.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+    ]
+    lib.attn_oracle_default_threads.restype = ctypes.c_int
+    return lib
+
+
+def attention(q, k, v, scale: float, causal: bool, rows: Optional[Sequence[int]] = None,
+              nthreads: int = 0, lib=None):
+    """O and LSE of softmax(scale * Q K^T [+ causal mask]) V in fp64.
+
+    q: [B,H,Nq,d], k/v: [B,H,Nkv,d] (torch fp16/bf16/any float tensor, or numpy), all
+    three of one dtype.  Causal masking is aligned bottom-right (query i sees keys
+    j <= i + Nkv - Nq).  rows: optional global row ids (b*H*Nq + h*Nq + i); the result
+    then has one row per id.  Returns (o, lse) as numpy float64: o [B,H,Nq,d] and
+    lse [B,H,Nq], or o [len(rows), d] and lse [len(rows)].  ``lib`` selects another
+    build of attn_oracle.c (the mutation tests use it); default: this package's.
+    """
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    assert tuple(k.shape) == (B, H, Nkv, d) and tuple(v.shape) == (B, H, Nkv, d)
+    qa, dt = _as_bits(q)
+    ka, dk = _as_bits(k)
+    va, dv = _as_bits(v)
+    assert dt == dk == dv, "q, k and v must share one dtype"
+    if rows is None:
+        nrows = B * H * Nq
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        nrows = int(rows_arr.size)
+    o = np.zeros((max(nrows, 1), d), dtype=np.float64)
+    lse = np.zeros((max(nrows, 1),), dtype=np.float64)
+    if nrows == 0:
+        return o[:0], lse[:0]
+    rc = (lib or _load()).attn_oracle_fwd(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, dt,
+        o.ctypes.data, lse.ctypes.data, B, H, Nq, Nkv, d, float(scale), int(bool(causal)),
+        None if rows_arr is None else rows_arr.ctypes.data, nrows, int(nthreads),
+    )
+    if rc != 0:
+        raise RuntimeError(f"attn_oracle_fwd failed with {rc}")
+    if rows is None:
+        return o.reshape(B, H, Nq, d), lse.reshape(B, H, Nq)
+    return o, lse
+
+
+def _f64(x):
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().cpu().to(torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, dtype=np.float64)
+
+
+def online_softmax_attention(q, k, v, scale: float, causal: bool, block_sizes=(128,),
+                             tau: float = 0.0):
+    """The tiled online-softmax forward, restated in numpy fp64.
+
+    Keys are visited in consecutive blocks whose sizes cycle through ``block_sizes``.
+    Per query row the state is (m, l, O~): running max (in log2 units), running sum of
+    2^(x - m) and the unnormalised output.  For each block with scores x (already
+    multiplied by log2(e) * scale, masked entries -inf):
+
+        m_new = max(m, max(x))
+        if m_new - m > tau:   O~ *= 2^(m - m_new);  l *= 2^(m - m_new);  m = m_new
+        p = 2^(x - m);  l += sum(p);  O~ += p @ V_block
+
+    and at the end O = O~ / l and LSE = (m + log2 l) * ln 2.  tau = 0 is the eager update
+    the pages describe; tau > 0 keeps the stale max (lazy rescale), exact in exact
+    arithmetic because O~ and l always share the same m.  Rows that see no key give O=0,
+    LSE=-inf.  Returns numpy (o [B,H,Nq,d], lse [B,H,Nq]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    log2e = 1.0 / np.log(2.0)
+    o = np.zeros((B, H, Nq, d))
+    lse = np.full((B, H, Nq), -np.inf)
+    rows = np.arange(Nq)[:, None]
+    for b in range(B):
+        for h in range(H):
+            m = np.full(Nq, -np.inf)
+            l = np.zeros(Nq)
+            acc = np.zeros((Nq, d))
+            start, bi = 0, 0
+            while start < Nkv:
+                bs = int(block_sizes[bi % len(block_sizes)])
+                bi += 1
+                cols = np.arange(start, min(start + bs, Nkv))[None, :]
+                x = (q[b, h] @ k[b, h, cols[0]].T) * (scale * log2e)
+                if causal:
+                    x = np.where(cols <= rows + (Nkv - Nq), x, -np.inf)
+                m_new = np.maximum(m, x.max(axis=1))
+                with np.errstate(invalid="ignore"):
+                    jump = m_new - m
+                    move = (jump > tau) | (np.isneginf(m) & np.isfinite(m_new))
+                    alpha = np.where(move, np.exp2(np.where(move, m - m_new, 0.0)), 1.0)
+                acc *= alpha[:, None]
+                l *= alpha
+                m = np.where(move, m_new, m)
+                m_safe = np.where(np.isneginf(m), 0.0, m)
+                p = np.exp2(x - m_safe[:, None])
+                l += p.sum(axis=1)
+                acc += p @ v[b, h, cols[0]]
+                start += bs
+            seen = l > 0
+            o[b, h] = np.where(seen[:, None], acc / np.where(seen, l, 1.0)[:, None], 0.0)
+            with np.errstate(divide="ignore"):
+                lse[b, h] = np.where(seen, (m + np.log2(np.where(seen, l, 1.0))) * np.log(2.0),
+                                     -np.inf)
+    return o, lse
+
+
+def lse_combine(o_parts, lse_parts):
+    """Merges S partial results over disjoint key sets into the full result.
+
+    o_parts: [S, ..., d], each normalised over its own keys; lse_parts: [S, ...] with
+    -inf for a part that saw no key.  With M = max_s lse_s and
+    L = M + ln sum_s exp(lse_s - M):  O = sum_s exp(lse_s - L) * O_s,  LSE = L.
+    All parts empty gives O = 0, LSE = -inf.
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    M = lse_parts.max(axis=0)
+    M_safe = np.where(np.isneginf(M), 0.0, M)
+    w = np.exp(lse_parts - M_safe)
+    tot = w.sum(axis=0)
+    with np.errstate(divide="ignore"):
+        L = np.where(tot > 0, M_safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    L_safe = np.where(np.isneginf(L), 0.0, L)
+    wn = np.where(np.isneginf(lse_parts), 0.0, np.exp(lse_parts - L_safe))
+    o = (wn[..., None] * o_parts).sum(axis=0)
+    return o, L
+
+
+def score_matrix_bytes(n: int, elem_bytes: int) -> int:
+    """Bytes of one head's n x n score matrix ("FlashAttention", section "The problem")."""
+    return n * n * elem_bytes
+
+
+def standard_attention_traffic(n: int, d: int, elem_bytes: int) -> dict:
+    """Per-head HBM bytes of materialising attention, term by term, as the
+    "FlashAttention 1-2-3" page estimates it in section "The Memory Wall": read Q, K, V;
+    write and read S; write and read P; write O."""
+    qkv = 3 * n * d * elem_bytes
+    s = 2 * n * n * elem_bytes
+    p = 2 * n * n * elem_bytes
+    o = n * d * elem_bytes
+    return {"qkv_read": qkv, "s_write_read": s, "p_write_read": p, "o_write": o,
+            "total": qkv + s + p + o}

@@ -1,0 +1,275 @@
+"""Pins for the fp64 CPU oracle, against facts the pages and the mathematics fix.
+
+None of these compares the oracle with itself: each check is a closed form, an
+invariant, brute force written independently (numpy exp/sum with an explicit mask), a
+library routine (torch CPU fp64 SDPA), or a byte count printed on the pages.
+"""
+import csv
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_59_b200.inputs import make_qkv, randn
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def _visible_mask(Nq, Nkv, causal):
+    """Boolean [Nq, Nkv]: query i sees key j (bottom-right alignment when causal)."""
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nkv)[None, :]
+    return (j <= i + (Nkv - Nq)) if causal else np.ones((Nq, Nkv), dtype=bool)
+
+
+def _brute(q, k, v, scale, causal):
+    """exp(S) / sum exp(S) with no max subtraction; fine for |S| well below 700."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    mask = _visible_mask(Nq, Nkv, causal)
+    o = np.zeros((B, H, Nq, d))
+    lse = np.full((B, H, Nq), -np.inf)
+    for b in range(B):
+        for h in range(H):
+            s = scale * np.einsum("ic,jc->ij", q[b, h], k[b, h])
+            e = np.where(mask, np.exp(s), 0.0)
+            z = e.sum(axis=1)
+            seen = z > 0
+            o[b, h] = np.where(seen[:, None], e / np.where(seen, z, 1)[:, None], 0) @ v[b, h]
+            lse[b, h] = np.where(seen, np.log(np.where(seen, z, 1)), -np.inf)
+    return o, lse
+
+
+SHAPES = [
+    # B, H, Nq, Nkv, d
+    (1, 1, 1, 1, 8),
+    (1, 2, 5, 5, 16),
+    (2, 3, 17, 17, 32),
+    (1, 2, 9, 23, 16),   # Nq < Nkv
+    (1, 2, 23, 9, 16),   # Nq > Nkv: causal rows 0..13 see nothing
+    (1, 1, 130, 130, 64),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_bruteforce_tiny(oracle_mod, shape, causal, dtype):
+    B, H, Nq, Nkv, d = shape
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, dtype, 11 + d)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = oracle_mod.attention(q, k, v, scale, causal)
+    ob, lb = _brute(q, k, v, scale, causal)
+    np.testing.assert_allclose(o, ob, rtol=0, atol=1e-12)
+    assert np.array_equal(np.isneginf(lse), np.isneginf(lb))
+    fin = np.isfinite(lb)
+    np.testing.assert_allclose(lse[fin], lb[fin], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_matches_torch_sdpa_fp64(oracle_mod, causal):
+    """Library special case: torch's CPU fp64 math SDPA (square causal = its is_causal)."""
+    B, H, N, d = 2, 3, 40, 32
+    q, k, v = make_qkv(B, H, N, N, d, torch.bfloat16, 99)
+    scale = 0.3
+    o, _ = oracle_mod.attention(q, k, v, scale, causal)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double(), k.double(), v.double(), is_causal=causal, scale=scale
+    ).numpy()
+    np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+
+
+def test_matches_torch_sdpa_bottom_right_mask(oracle_mod):
+    B, H, Nq, Nkv, d = 1, 2, 12, 31, 16
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, torch.float16, 5)
+    mask = torch.from_numpy(_visible_mask(Nq, Nkv, True))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double(), k.double(), v.double(), attn_mask=mask, scale=0.25
+    ).numpy()
+    o, _ = oracle_mod.attention(q, k, v, 0.25, True)
+    np.testing.assert_allclose(o, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_normalised(oracle_mod, causal):
+    """Softmax rows sum to one: with V all ones every visible row of O is exactly 1."""
+    B, H, Nq, Nkv, d = 1, 2, 37, 37, 16
+    q, k, _ = make_qkv(B, H, Nq, Nkv, d, torch.float16, 3, q_std=3.0)
+    v = torch.ones(B, H, Nkv, d, dtype=torch.float16)
+    o, _ = oracle_mod.attention(q, k, v, 1.0, causal)
+    np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-12)
+
+
+def test_causal_row0_is_v0(oracle_mod):
+    """The causal mask leaves query 0 only key 0: O_0 = V_0 exactly, LSE_0 = s_00."""
+    B, H, N, d = 2, 2, 29, 32
+    q, k, v = make_qkv(B, H, N, N, d, torch.bfloat16, 21, q_std=4.0)
+    scale = 0.177
+    o, lse = oracle_mod.attention(q, k, v, scale, True)
+    assert np.array_equal(o[:, :, 0, :], _f64(v)[:, :, 0, :])
+    s00 = scale * np.einsum("bhc,bhc->bh", _f64(q)[:, :, 0], _f64(k)[:, :, 0])
+    np.testing.assert_allclose(lse[:, :, 0], s00, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_identical_keys_give_mean_of_visible_v(oracle_mod, causal):
+    B, H, Nq, Nkv, d = 1, 2, 19, 26, 16
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, torch.float16, 8)
+    k = k[:, :, :1, :].expand(B, H, Nkv, d).contiguous()
+    scale = 0.5
+    o, lse = oracle_mod.attention(q, k, v, scale, causal)
+    vis = _visible_mask(Nq, Nkv, causal)
+    vf, qf, kf = _f64(v), _f64(q), _f64(k)
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nq):
+                J = np.nonzero(vis[i])[0]
+                np.testing.assert_allclose(o[b, h, i], vf[b, h, J].mean(axis=0), atol=1e-12)
+                s = scale * qf[b, h, i] @ kf[b, h, 0]
+                assert lse[b, h, i] == pytest.approx(s + math.log(len(J)), abs=1e-12)
+
+
+def test_scale_zero_gives_mean(oracle_mod):
+    B, H, Nq, Nkv, d = 2, 1, 11, 11, 8
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, torch.bfloat16, 4)
+    o, lse = oracle_mod.attention(q, k, v, 0.0, True)
+    vf = _f64(v)
+    for i in range(Nq):
+        np.testing.assert_allclose(o[:, :, i], vf[:, :, : i + 1].mean(axis=2), atol=1e-12)
+        np.testing.assert_allclose(lse[:, :, i], math.log(i + 1), atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_shift_invariance(oracle_mod, causal):
+    """Adding u to every key adds scale*q_i.u to row i's scores: O is unchanged and LSE
+    moves by exactly that amount (the max subtraction must cancel it)."""
+    B, H, Nq, Nkv, d = 1, 2, 13, 21, 16
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, torch.float64, 6)
+    u = randn((d,), 77, torch.float64, std=3.0)
+    scale = 0.4
+    o, lse = oracle_mod.attention(q, k, v, scale, causal)
+    o2, lse2 = oracle_mod.attention(q, k + u, v, scale, causal)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-11)
+    shift = scale * np.einsum("bhic,c->bhi", _f64(q), _f64(u))
+    fin = np.isfinite(lse)
+    np.testing.assert_allclose((lse2 - lse)[fin], shift[fin], rtol=0, atol=1e-10)
+
+
+def test_large_scores_stay_finite(oracle_mod):
+    """Scores near 1e4 overflow a softmax without max subtraction; the oracle must not."""
+    B, H, N, d = 1, 1, 16, 8
+    q, k, v = make_qkv(B, H, N, N, d, torch.float64, 12)
+    o, lse = oracle_mod.attention(q * 100, k * 100, v, 1.0, False)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    qf, kf = _f64(q) * 100, _f64(k) * 100
+    s = qf[0, 0] @ kf[0, 0].T
+    # row-wise argmax dominates: O equals V at the argmax within float rounding
+    top = s.argmax(axis=1)
+    gap = np.sort(s, axis=1)[:, -1] - np.sort(s, axis=1)[:, -2]
+    sure = gap > 60
+    np.testing.assert_allclose(o[0, 0][sure], _f64(v)[0, 0][top[sure]], atol=1e-12)
+
+
+def test_fully_masked_rows(oracle_mod):
+    """Causal with Nq > Nkv: query i sees keys j <= i - (Nq - Nkv); rows before that see
+    nothing and give O = 0, LSE = -inf."""
+    q, k, v = make_qkv(1, 1, 10, 4, 8, torch.float16, 2)
+    o, lse = oracle_mod.attention(q, k, v, 1.0, True)
+    assert (o[0, 0, :6] == 0).all() and np.isneginf(lse[0, 0, :6]).all()
+    assert np.isfinite(lse[0, 0, 6:]).all()
+    np.testing.assert_array_equal(o[0, 0, 6], _f64(v)[0, 0, 0])
+
+
+def test_sixteen_bit_decoding_is_exact(oracle_mod):
+    """The C oracle decodes fp16/bf16 bit patterns itself; it must agree bit for bit
+    with the same values passed as fp64 (subnormals, extremes and signed zero too)."""
+    special = [0.0, -0.0, 6.0e-8, -6.0e-8, 1.0e-5, 65504.0, -65504.0, 0.333, 1024.5]
+    for dtype in (torch.float16, torch.bfloat16):
+        q, k, v = make_qkv(1, 2, 9, 9, 16, dtype, 31)
+        vals = torch.tensor(special, dtype=dtype)
+        v.view(-1)[: len(special)] = vals
+        k.view(-1)[-len(special):] = vals * 0.001
+        o16, l16 = oracle_mod.attention(q, k, v, 0.1, False)
+        o64, l64 = oracle_mod.attention(q.double(), k.double(), v.double(), 0.1, False)
+        assert np.array_equal(o16, o64) and np.array_equal(l16, l64)
+
+
+def test_rows_subset_and_threads(oracle_mod):
+    B, H, Nq, Nkv, d = 2, 2, 33, 40, 16
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, torch.bfloat16, 13)
+    o, lse = oracle_mod.attention(q, k, v, 0.2, True, nthreads=1)
+    o4, lse4 = oracle_mod.attention(q, k, v, 0.2, True, nthreads=4)
+    assert np.array_equal(o, o4) and np.array_equal(lse, lse4)
+    rows = [0, 5, 32, 33, 70, B * H * Nq - 1]
+    orow, lrow = oracle_mod.attention(q, k, v, 0.2, True, rows=rows)
+    of, lf = o.reshape(-1, d), lse.reshape(-1)
+    assert np.array_equal(orow, of[rows]) and np.array_equal(lrow, lf[rows])
+
+
+@pytest.mark.parametrize("tau", [0.0, 8.0])
+@pytest.mark.parametrize("causal", [False, True])
+def test_online_blockwise_equals_two_pass(oracle_mod, tau, causal):
+    """The tiled online softmax (the method) reaches the two-pass definition."""
+    rng = np.random.default_rng(int(tau) * 10 + causal)
+    for trial in range(4):
+        Nq, Nkv = int(rng.integers(1, 70)), int(rng.integers(1, 90))
+        if causal and trial == 0:
+            Nq, Nkv = 64, 64
+        q, k, v = make_qkv(1, 2, Nq, Nkv, 16, torch.float64, 100 + trial, q_std=3.0)
+        blocks = tuple(int(b) for b in rng.integers(1, 33, size=5))
+        o2, l2 = oracle_mod.attention(q, k, v, 0.7, causal)
+        o1, l1 = oracle_mod.online_softmax_attention(q, k, v, 0.7, causal, blocks, tau)
+        np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-12)
+        assert np.array_equal(np.isneginf(l1), np.isneginf(l2))
+        fin = np.isfinite(l2)
+        np.testing.assert_allclose(l1[fin], l2[fin], rtol=0, atol=1e-12)
+
+
+def test_split_combine_equals_unsplit(oracle_mod):
+    """Split-KV: partial results over any partition of the keys, merged by LSE, equal
+    the result over all keys (one part may be empty)."""
+    rng = np.random.default_rng(5)
+    B, H, Nq, Nkv, d = 2, 2, 1, 300, 32
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, torch.bfloat16, 55, q_std=2.0)
+    o_full, l_full = oracle_mod.attention(q, k, v, 0.3, False)
+    for S in (1, 2, 5, 16):
+        cuts = np.sort(rng.choice(np.arange(1, Nkv), size=S - 1, replace=False))
+        bounds = [0, *cuts.tolist(), Nkv]
+        parts_o, parts_l = [], []
+        for a, b in zip(bounds[:-1], bounds[1:]):
+            o_s, l_s = oracle_mod.attention(q, k[:, :, a:b], v[:, :, a:b], 0.3, False)
+            parts_o.append(o_s)
+            parts_l.append(l_s)
+        parts_o.append(np.zeros_like(parts_o[0]))
+        parts_l.append(np.full_like(parts_l[0], -np.inf))
+        o, l = oracle_mod.lse_combine(parts_o, parts_l)
+        np.testing.assert_allclose(o, o_full, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l, l_full, rtol=0, atol=1e-12)
+    o, l = oracle_mod.lse_combine([np.zeros((3, 4))] * 2, [np.full(3, -np.inf)] * 2)
+    assert (o == 0).all() and np.isneginf(l).all()
+
+
+def test_golden_byte_counts(oracle_mod):
+    with open(os.path.join(GOLDEN, "byte_counts.txt")) as f:
+        rows = [r for r in csv.reader((line for line in f if not line.startswith("#")),
+                                     delimiter="|")]
+    assert len(rows) == 7
+    for kind, n, d, eb, term, val, unit, _cite in rows:
+        n, d, eb, val = int(n), int(d), int(eb), int(val)
+        if kind == "score_matrix":
+            assert oracle_mod.score_matrix_bytes(n, eb) == val
+        else:
+            t = oracle_mod.standard_attention_traffic(n, d, eb)
+            if term == "total":
+                printed = [int(r[5]) for r in rows if r[0] == kind and r[4] != "total"]
+                assert sum(printed) == val
+                assert abs(t["total"] / 1e6 - val) < 2
+            else:
+                assert round(t[term] / 1e6) == val
