@@ -1,0 +1,427 @@
+"""Benchmark of the exact attention forward on B200: prefill TFLOP/s and decode HBM GB/s.
+
+One step = one pass of the hot path over one batch of synthetic input:
+  * the headline line times the long causal prefill (B=1, H=32, N=8192, d=128, bf16), one
+    fa_fwd call per step;
+  * the "decode" object times the split-KV decode (B=16, H=32, Nq=1, Nkv=32768, d=128,
+    bf16), one fa_fwd call (split kernel + combine kernel) per step.
+Inputs are resident in HBM and larger than L2 (126 MB) when the timed region starts.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (N > 1, one process per GPU via torch.distributed.run): every rank runs the
+same independent problem (heads are independent; no collective on the data path);
+timings are max over ranks, value = all ranks' FLOPs / that time (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_59_b200 import binding  # noqa: E402
+from exact_io_aware_59_b200.inputs import WORKLOADS, Workload, workload_qkv  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s at 1 B200 (% of dense bf16 peak); decode HBM GB/s"
+PREFILL = "long_prefill_causal"
+DECODE = "decode"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- accounting
+def causal_pairs(Nq: int, Nkv: int) -> int:
+    """Visible (query, key) pairs under the bottom-right causal mask."""
+    off = Nkv - Nq
+    total = 0
+    # sum_i min(Nkv, max(0, i + off + 1)) in closed form by segments
+    lo = max(0, -off)                       # first row that sees a key
+    hi = min(Nq, Nkv - off)                 # rows [lo, hi) see i + off + 1 keys
+    if hi > lo:
+        total += (hi - lo) * (off + 1) + (hi - 1 + lo) * (hi - lo) // 2
+    if Nq > max(hi, lo):
+        total += (Nq - max(hi, lo)) * Nkv
+    return total
+
+
+def attention_flops(w: Workload) -> int:
+    """4 * d per visible (query, key) pair: 2d for q.k and 2d for p*v; causal counts the
+    visible lower triangle only."""
+    pairs = causal_pairs(w.Nq, w.Nkv) if w.causal else w.Nq * w.Nkv
+    return 4 * w.d * w.B * w.H * pairs
+
+
+def algorithmic_bytes(w: Workload, o_bytes: int) -> int:
+    """Read Q, K, V once; write O and LSE once."""
+    BH = w.B * w.H
+    return BH * (w.Nq * w.d * 2 + 2 * w.Nkv * w.d * 2 + w.Nq * w.d * o_bytes + w.Nq * 4)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            ident = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", ident, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.reader.join(timeout=2)
+
+    def summary(self):
+        rows = []
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, flag in enumerate(r[3])
+                          if flag.lower() == "active"})
+        busy = [r for r in rows if r[2] > 300.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in busy),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(busy),
+                "power_w_max": max(r[2] for r in rows)}
+
+
+# ---------------------------------------------------------------- timing helpers
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(fn, steps: int, warmup: int, ws: int, stream) -> float:
+    """Milliseconds per step over `steps` calls, CUDA events on the launch stream."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    return max_over_ranks(start.elapsed_time(end) / steps, ws)
+
+
+def check(rc, where):
+    if rc != binding.FA_OK:
+        raise binding.FaError(rc, where)
+
+
+def make_call(w: Workload, q, k, v, o, lse, stream):
+    ic = binding.FA_BF16 if w.dtype == torch.bfloat16 else binding.FA_F16
+    oc = binding._dtype_code(o.dtype)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+            w.B, w.H, w.Nq, w.Nkv, w.d, float(w.softmax_scale), int(w.causal),
+            stream.cuda_stream, ic, oc)
+
+    def call():
+        check(binding.fa_fwd(*args), "fa_fwd")
+
+    return call
+
+
+def run_workload(w: Workload, steps, warmup, ws, stream, out_dtype):
+    q, k, v = workload_qkv(w, device="cuda")
+    o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=out_dtype, device="cuda")
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device="cuda")
+    call = make_call(w, q, k, v, o, lse, stream)
+    with torch.cuda.stream(stream):
+        ms = time_steps(call, steps, warmup, ws, stream)
+    return ms, (q, k, v, o, lse)
+
+
+def run_e2e(w: Workload, tensors, steps, warmup, ws, stream):
+    """The same call with pinned HOST inputs: per step, copy Q/K/V host->device, run,
+    copy O and LSE device->host; all inside the timed region."""
+    q, k, v, o, lse = tensors
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    call = make_call(w, q, k, v, o, lse, stream)
+
+    def step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        call()
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        ms = time_steps(step, steps, warmup, ws, stream)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    return ms, h2d, d2h
+
+
+_HOST_INPUTS = {}
+
+
+def cpu_baseline(w: Workload, budget_s: float, seed: int = 0):
+    """The fp64 oracle, as it stands, on a bounded row sample of the workload; returns
+    (TFLOP/s, threads, description, seconds).  Rows are drawn uniformly over heads and
+    positions, so the causal FLOPs per row average those of the whole workload."""
+    import numpy as np
+
+    import oracle
+
+    g = np.random.default_rng(seed)
+    if w.name not in _HOST_INPUTS:
+        _HOST_INPUTS[w.name] = workload_qkv(w, device="cpu")
+    q, k, v = _HOST_INPUTS[w.name]
+    threads = oracle.default_threads()
+    n_total = w.B * w.H * w.Nq
+
+    def row_flops(rows):
+        i = rows % w.Nq
+        vis = np.minimum(w.Nkv, np.maximum(0, i + (w.Nkv - w.Nq) + 1)) if w.causal else w.Nkv
+        return int(4 * w.d * np.sum(vis))
+
+    n = max(threads * 2, 16)
+    while True:
+        rows = np.sort(g.choice(n_total, size=min(n, n_total), replace=False))
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, w.softmax_scale, w.causal, rows=rows, nthreads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or len(rows) == n_total:
+            break
+        n = int(min(n_total, max(n * 2, n * budget_s / max(dt, 1e-3) * 1.1)))
+    tflops = row_flops(rows) / dt / 1e12
+    desc = (f"{len(rows)} of {n_total} query rows of {w.name}, drawn uniformly at random "
+            f"(seed {seed}); {dt:.1f} s of CPU work")
+    return tflops, threads, desc, dt
+
+
+# ---------------------------------------------------------------- arms
+def arm_reference(args, ws, rank):
+    """The oracle, as it stands, on the host cores: each step a bounded row sample."""
+    if rank != 0:
+        return
+    w = WORKLOADS[PREFILL]
+    # Bounded sample per step so that the whole run stays within a few minutes.
+    per_step = min(2.0, max(0.05, 90.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(w, per_step, seed=99)
+    vals = []
+    threads, desc, secs = 0, "", 0.0
+    for s in range(args.steps):
+        v, threads, desc, dt = cpu_baseline(w, per_step, seed=s)
+        vals.append(v)
+        secs += dt
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs * 1e3 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, "fp64 oracle"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w: Workload, o_dtype: str):
+    return {"workload": f"{w.name}: B={w.B} H={w.H} Nq={w.Nq} Nkv={w.Nkv} d={w.d} "
+                        f"{str(w.dtype).replace('torch.', '')} causal={w.causal}",
+            "B": w.B, "H": w.H, "Nq": w.Nq, "Nkv": w.Nkv, "d": w.d, "causal": w.causal,
+            "o_dtype": o_dtype, "parallelism": "independent problem per GPU",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
+def arm_ours(args, ws, rank, local):
+    torch.cuda.set_device(local)
+    stream = torch.cuda.Stream()
+    peaks, peak_src = load_peaks()
+    out_dtype = torch.bfloat16
+
+    # prefill (headline)
+    wp = WORKLOADS[PREFILL]
+    with ClockSampler(local) as clk:
+        ms_p, tensors = run_workload(wp, args.steps, args.warmup, ws, stream, out_dtype)
+    assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+    flops = attention_flops(wp)
+    tflops = flops / (ms_p * 1e-3) / 1e12
+    value = tflops * ws
+    peak_t = peaks["bf16_tflops"]
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "prefill_traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as f:
+            t = json.load(f)
+        if t.get("kernel_rev") == KERNEL_REV:
+            traffic = t.get("bytes_per_launch")
+
+    # decode
+    decode = None
+    if not args.skip_decode:
+        wd = WORKLOADS[DECODE]
+        dsteps = max(3, args.steps // 8)
+        with ClockSampler(local) as clk_d:
+            ms_d, dt_ = run_workload(wd, dsteps, args.warmup, ws, stream, out_dtype)
+        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+        del dt_
+        bytes_d = algorithmic_bytes(wd, 2)
+        gbs = bytes_d / (ms_d * 1e-3) / 1e9
+        decode = {
+            "workload": workload_config(wd, "bf16")["workload"], "value": gbs * ws,
+            "unit": "GB/s", "ms_per_step": ms_d, "steps": dsteps,
+            "gpu_launches": 2 * dsteps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": peak_src,
+                         "algorithmic_bytes_per_launch": bytes_d},
+            "clocks": clk_d.summary(),
+        }
+        torch.cuda.empty_cache()
+
+    # end to end through the C ABI with host buffers
+    e2e = None
+    if not args.skip_e2e:
+        esteps = max(3, min(args.steps, 20))
+        ms_e, h2d, d2h = run_e2e(wp, tensors, esteps, 2, ws, stream)
+        e2e = {"value": flops / (ms_e * 1e-3) / 1e12 * ws, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e,
+               "steps": esteps}
+    del tensors
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.skip_cpu:
+        v, threads, desc, _ = cpu_baseline(wp, args.cpu_seconds)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_p,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(wp, "bf16"),
+            "gpu_launches": args.steps,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_t,
+                         "unit": "TFLOP/s", "frac": tflops / peak_t, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst (kernel timed back to back)",
+                         "flops_per_launch": flops,
+                         "frac_of_sustained": tflops / peaks.get("bf16_tflops_sustained", peak_t)},
+            "clocks": clk.summary(),
+            "decode": decode,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+# Bumped whenever the prefill kernel changes, so stale ncu traffic is not reported.
+KERNEL_REV = "prefill-v1"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    ws, rank, local = dist_info()
+    if ws > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            arm_reference(args, ws, rank)
+        else:
+            arm_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

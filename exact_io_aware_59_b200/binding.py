@@ -1,0 +1,176 @@
+"""ctypes binding of libfa_b200.so (declared in include/fa.h).
+
+Argument marshalling only: every step of the attention runs in the library's CUDA
+kernels.  The raw functions keep the C names and argument order; ``attention`` is a
+convenience wrapper that takes torch CUDA tensors, allocates O and LSE and passes torch's
+current stream.  There is no fallback: if the library cannot be loaded, every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from typing import Optional
+
+from . import build as _build
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ARCH = 0, 1, 2, 3
+FA_ERR_CUDA, FA_ERR_NOMEM, FA_ERR_DEVICE_TIMEOUT = 4, 5, 6
+FA_F16, FA_BF16, FA_F32 = 0, 1, 2
+
+HEADER = os.path.join(_build.INCLUDE, "fa.h")
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = f"{where} failed: {status_string(code)} ({code})"
+        if code == FA_ERR_CUDA and _lib is not None:
+            msg += f", cudaError {int(_lib.fa_last_cuda_error())}"
+        super().__init__(msg)
+
+
+_VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_SIGNATURES = {
+    "fa_fwd": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I],
+    "fa_fwd_prefill": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I, _I],
+    "fa_fwd_decode": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
+    "fa_decode_workspace_bytes": [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
+    "fa_device_status": [ctypes.POINTER(_I), _I],
+    "fa_selftest_wait_timeout": [_VP],
+    "fa_release_workspace": [],
+    "fa_last_cuda_error": [],
+    "fa_status_string": [_I],
+    "fa_version": [],
+}
+
+
+def declared_functions() -> list:
+    """Names of the functions include/fa.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", text, flags=re.M)
+
+
+def library(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Loads libfa_b200.so (building it first when it is missing or stale)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB_PATH
+        if build_if_missing and not _build.up_to_date():
+            _build.build()
+        if not os.path.exists(path):
+            raise RuntimeError(f"libfa_b200.so is missing ({path}); build it with "
+                               "`python -m exact_io_aware_59_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, argtypes in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = argtypes
+            fn.restype = ctypes.c_char_p if name == "fa_status_string" else ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return library().fa_status_string(int(code)).decode()
+
+
+# ---------------------------------------------------------------- raw C calls
+def fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype, o_dtype) -> int:
+    return library().fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream,
+                            in_dtype, o_dtype)
+
+
+def fa_fwd_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype,
+                   o_dtype, num_ctas) -> int:
+    return library().fa_fwd_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream,
+                                    in_dtype, o_dtype, num_ctas)
+
+
+def fa_fwd_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype,
+                  num_splits) -> int:
+    return library().fa_fwd_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype,
+                                   o_dtype, num_splits)
+
+
+def fa_decode_workspace_bytes(B, H, Nkv, d, num_splits) -> int:
+    out = ctypes.c_size_t(0)
+    rc = library().fa_decode_workspace_bytes(B, H, Nkv, d, num_splits, ctypes.byref(out))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_decode_workspace_bytes")
+    return int(out.value)
+
+
+def fa_device_status(clear: bool = True) -> int:
+    """The current device's status word (0 = no kernel wait ran out)."""
+    word = ctypes.c_int(0)
+    rc = library().fa_device_status(ctypes.byref(word), int(bool(clear)))
+    if rc not in (FA_OK, FA_ERR_DEVICE_TIMEOUT):
+        raise FaError(rc, "fa_device_status")
+    return int(word.value)
+
+
+def fa_selftest_wait_timeout(stream=None) -> int:
+    return library().fa_selftest_wait_timeout(stream)
+
+
+def fa_release_workspace() -> None:
+    rc = library().fa_release_workspace()
+    if rc != FA_OK:
+        raise FaError(rc, "fa_release_workspace")
+
+
+# ---------------------------------------------------------------- torch convenience
+def _dtype_code(t):
+    import torch
+
+    return {torch.float16: FA_F16, torch.bfloat16: FA_BF16, torch.float32: FA_F32}[t]
+
+
+def attention(q, k, v, causal: bool = False, scale: Optional[float] = None,
+              out_dtype=None, out=None, lse=None, num_ctas: int = 0, num_splits: int = 0,
+              path: str = "auto", stream=None):
+    """O, LSE = softmax(scale * Q K^T [+ causal]) V for contiguous CUDA tensors
+    q [B,H,Nq,d], k/v [B,H,Nkv,d] (fp16 or bf16).  out_dtype: torch.float32 (default) or
+    the input dtype.  path: "auto" (decode when Nq == 1), "prefill" or "decode".
+    Enqueues on `stream` (default: torch's current stream) and returns (o, lse)."""
+    import torch
+
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("attention() takes CUDA tensors")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k and v must be contiguous [B,H,N,d]")
+    if q.dtype != k.dtype or q.dtype != v.dtype or q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("q, k, v must share one dtype, float16 or bfloat16")
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    if tuple(k.shape) != (B, H, Nkv, d) or tuple(v.shape) != (B, H, Nkv, d):
+        raise ValueError("k and v must be [B,H,Nkv,d] with q's B, H and d")
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    s = torch.cuda.current_stream(q.device) if stream is None else stream
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr())
+    ic, oc = _dtype_code(q.dtype), _dtype_code(out.dtype)
+    with torch.cuda.device(q.device):
+        if path == "decode" or (path == "auto" and Nq == 1):
+            if Nq != 1:
+                raise ValueError("the decode path takes exactly one query per head")
+            rc = fa_fwd_decode(*args, B, H, Nkv, d, scale, s.cuda_stream, ic, oc, num_splits)
+            where = "fa_fwd_decode"
+        elif path in ("prefill", "auto"):
+            rc = fa_fwd_prefill(*args, B, H, Nq, Nkv, d, scale, int(bool(causal)), s.cuda_stream,
+                                ic, oc, num_ctas)
+            where = "fa_fwd_prefill"
+        else:
+            raise ValueError(f"unknown path {path!r}")
+    if rc != FA_OK:
+        raise FaError(rc, where)
+    return out, lse

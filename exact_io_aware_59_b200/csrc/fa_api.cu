@@ -1,0 +1,320 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument checks, per-device state,
+// TMA descriptors and kernel launches.  Host code only.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool probed = false;
+  bool arch_ok = false;
+  int sm_count = 0;
+  int* status = nullptr;   // device status word (256 bytes allocated)
+  float* ws = nullptr;     // decode partials
+  size_t ws_bytes = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+thread_local int g_last_cuda_error = 0;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return FA_ERR_CUDA;
+}
+
+// Looks up (and on first use initialises) the current device's state.
+int device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    s.arch_ok = (major == 10 && minor == 0);  // the sm_100a code runs on CC 10.0 only
+    s.sm_count = sms;
+    s.probed = true;
+  }
+  if (!s.arch_ok) return FA_ERR_ARCH;
+  if (!s.status) {
+    void* p = nullptr;
+    if ((e = cudaMalloc(&p, 256)) != cudaSuccess) return e == cudaErrorMemoryAllocation ? FA_ERR_NOMEM : cuda_fail(e);
+    if ((e = cudaMemset(p, 0, 256)) != cudaSuccess || (e = cudaDeviceSynchronize()) != cudaSuccess) {
+      cudaFree(p);
+      return cuda_fail(e);
+    }
+    s.status = static_cast<int*>(p);
+  }
+  *out = &s;
+  return FA_OK;
+}
+
+int get_encoder() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_encode) return FA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(cudaErrorNotSupported);
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return FA_OK;
+}
+
+// 3-D view (d, N, B*H) of a [B,H,N,d] tensor; box (64, 128, 1) with 128-byte swizzle.
+int make_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, bool bf16) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FA_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Checks shared by every entry point.  Nothing here touches the device.
+int check_args(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int Nq, int Nkv, int d, float scale, int causal, int in_dtype, int o_dtype) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Nq < 1 || Nkv < 1) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (in_dtype != FA_F16 && in_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_F16 && o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_F32 && o_dtype != in_dtype) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return FA_ERR_INVALID_ARG;
+  if (lse && !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t qb = BH * Nq * d * 2, kvb = BH * Nkv * d * 2;
+  const size_t ob = BH * Nq * d * (o_dtype == FA_F32 ? 4 : 2), lb = BH * Nq * 4;
+  if (overlaps(o, ob, q, qb) || overlaps(o, ob, k, kvb) || overlaps(o, ob, v, kvb)) return FA_ERR_INVALID_ARG;
+  if (lse && (overlaps(lse, lb, o, ob) || overlaps(lse, lb, q, qb) || overlaps(lse, lb, k, kvb) ||
+              overlaps(lse, lb, v, kvb)))
+    return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+float scale_log2(float scale) { return static_cast<float>(static_cast<double>(scale) * 1.4426950408889634); }
+
+fa::DecodeParams decode_params(int B, int H, int Nkv, float scale, int num_splits, int sm_count) {
+  fa::DecodeParams p{};
+  p.BH = B * H;
+  p.Nkv = Nkv;
+  p.n_chunks = (Nkv + fa::kDecodeChunk - 1) / fa::kDecodeChunk;
+  p.total = static_cast<long long>(p.BH) * p.n_chunks;
+  long long g = num_splits > 0 ? num_splits : sm_count;
+  if (g > p.total) g = p.total;
+  if (g < 1) g = 1;
+  p.grid = static_cast<int>(g);
+  const long long per_cta = (p.total + p.grid - 1) / p.grid;
+  p.max_seg = static_cast<int>((per_cta + p.n_chunks - 1) / p.n_chunks + 1);
+  p.scale_log2 = scale_log2(scale);
+  return p;
+}
+
+size_t decode_ws_bytes(const fa::DecodeParams& p, int d) {
+  const size_t recs = static_cast<size_t>(p.grid) * p.max_seg * 8;  // 8 consumer warps
+  return recs * (d + 1) * sizeof(float);
+}
+
+int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                int Nq, int Nkv, int d, float scale, int causal, void* stream, int in_dtype,
+                int o_dtype, int num_ctas) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+  const bool bf16 = in_dtype == FA_BF16;
+  const long long BH = static_cast<long long>(B) * H;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map(&tq, q, Nq, BH, d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map(&tk, k, Nkv, BH, d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, Nkv, BH, d, bf16)) != FA_OK) return rc;
+  fa::PrefillParams p{};
+  p.BH = static_cast<int>(BH);
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.off = Nkv - Nq;
+  p.causal = causal;
+  p.n_qtiles = (Nq + 127) / 128;
+  p.n_pairs = (p.n_qtiles + 1) / 2;
+  p.n_kvtiles = (Nkv + 127) / 128;
+  const long long units = BH * p.n_pairs;
+  if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  p.n_units = static_cast<int>(units);
+  p.scale_log2 = scale_log2(scale);
+  long long grid = num_ctas > 0 ? num_ctas : ds->sm_count;
+  if (grid > units) grid = units;
+  if (grid < 1) grid = 1;
+  cudaError_t e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, bf16, o_dtype == FA_F32,
+                                     static_cast<int>(grid), ds->status,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int run_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int Nkv, int d, float scale, void* stream, int in_dtype, int o_dtype,
+               int num_splits) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  const fa::DecodeParams p = decode_params(B, H, Nkv, scale, num_splits, ds->sm_count);
+  const size_t need = decode_ws_bytes(p, d);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (ds->ws_bytes < need) {
+      if (ds->ws) {
+        cudaError_t e = cudaFree(ds->ws);  // synchronises: no kernel still reads it
+        ds->ws = nullptr;
+        ds->ws_bytes = 0;
+        if (e != cudaSuccess) return cuda_fail(e);
+      }
+      void* ptr = nullptr;
+      cudaError_t e = cudaMalloc(&ptr, need);
+      if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? FA_ERR_NOMEM : cuda_fail(e);
+      ds->ws = static_cast<float*>(ptr);
+      ds->ws_bytes = need;
+    }
+  }
+  float* part_o = ds->ws;
+  float* part_lse = ds->ws + static_cast<size_t>(p.grid) * p.max_seg * 8 * d;
+  cudaError_t e = fa::launch_decode(q, k, v, o, lse, p, d, in_dtype == FA_BF16, o_dtype == FA_F32,
+                                    part_o, part_lse, ds->status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+           int Nq, int Nkv, int d, float scale, int causal, void* stream, int in_dtype,
+           int o_dtype) {
+  int rc = check_args(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, in_dtype, o_dtype);
+  if (rc != FA_OK) return rc;
+  if (Nq == 1) return run_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype, 0);
+  return run_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype, o_dtype, 0);
+}
+
+int fa_fwd_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
+                   int in_dtype, int o_dtype, int num_ctas) {
+  int rc = check_args(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, in_dtype, o_dtype);
+  if (rc != FA_OK) return rc;
+  if (num_ctas < 0) return FA_ERR_INVALID_ARG;
+  return run_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype, o_dtype,
+                     num_ctas);
+}
+
+int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int H, int Nkv, int d, float scale, void* stream, int in_dtype, int o_dtype,
+                  int num_splits) {
+  int rc = check_args(q, k, v, o, lse, B, H, 1, Nkv, d, scale, 0, in_dtype, o_dtype);
+  if (rc != FA_OK) return rc;
+  if (num_splits < 0) return FA_ERR_INVALID_ARG;
+  return run_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype, num_splits);
+}
+
+int fa_decode_workspace_bytes(int B, int H, int Nkv, int d, int num_splits, size_t* bytes) {
+  if (!bytes || B < 1 || H < 1 || Nkv < 1 || num_splits < 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  int sms = 148;
+  DeviceState* ds = nullptr;
+  if (num_splits == 0) {
+    int rc = device_state(&ds);
+    if (rc != FA_OK) return rc;
+    sms = ds->sm_count;
+  }
+  *bytes = decode_ws_bytes(decode_params(B, H, Nkv, 1.0f, num_splits, sms), d);
+  return FA_OK;
+}
+
+int fa_device_status(int* status, int clear) {
+  if (!status) return FA_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  int word = 0;
+  cudaError_t e = cudaMemcpy(&word, ds->status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (clear && word != 0) {
+    e = cudaMemset(ds->status, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  *status = word;
+  return word ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+}
+
+int fa_selftest_wait_timeout(void* stream) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  cudaError_t e = fa::launch_wait_timeout_selftest(ds->status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_release_workspace(void) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (s.ws) {
+    e = cudaFree(s.ws);
+    s.ws = nullptr;
+    s.ws_bytes = 0;
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return FA_OK;
+}
+
+int fa_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_ARCH: return "device is not sm_100 (B200)";
+    case FA_ERR_CUDA: return "CUDA runtime error";
+    case FA_ERR_NOMEM: return "out of device memory";
+    case FA_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

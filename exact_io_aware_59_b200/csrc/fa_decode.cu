@@ -1,0 +1,384 @@
+// fa_decode.cu -- split-KV attention for one query per head (decode), sm_100a.
+//
+// The method ("FlashAttention 1-2-3" (myaihardware), section "Beyond FlashAttention":
+// FlashDecoding parallelises over the KV length, computes a partial softmax per chunk
+// and then reduces; "Flash Attention -- Module 12.3", section "Prefill vs Decode": one
+// query against a long KV cache): each split computes, over its own keys, the
+// normalised partial output O_s and its log-sum-exp lse_s with the online softmax; a
+// second kernel merges the splits:  M = max_s lse_s,  L = M + ln sum_s e^(lse_s - M),
+// O = sum_s e^(lse_s - L) O_s.
+//
+// The B200 mapping: decode reads every K/V byte once, so it is bound by HBM bandwidth.
+// All (b, h) heads' keys form one flat range of 64-key chunks; CTA c of G owns chunks
+// [c*T/G, (c+1)*T/G), so every SM streams the same number of bytes whatever B*H and
+// Nkv are.  One producer lane streams K and V chunks with bulk copies (L2 evict-first)
+// into a ring of shared-memory stages; eight consumer warps each take 8 keys of every
+// chunk: lanes split the head dimension for q.k (a transposing butterfly reduces 8 dot
+// products in 9 shuffles), then each lane accumulates its own d-slice of P V in fp32.
+// Each time a CTA finishes the part of a head it owns, every consumer warp writes one
+// partial record (O_s, lse_s) for the keys it saw; the combine kernel merges them all.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fa_device.cuh"
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+constexpr int kWarps = 8;                     // consumer warps
+constexpr int kThreads = (kWarps + 1) * 32;   // + one producer warp
+constexpr int kKeysPerWarp = kDecodeChunk / kWarps;
+static_assert(kKeysPerWarp == 8, "the butterfly below reduces 8 keys per warp");
+
+template <int D>
+struct DecodeCfg {
+  static constexpr int kChunkBytes = kDecodeChunk * D * 2;  // K or V part of a stage
+  static constexpr int kStages = (D == 128) ? 6 : 10;
+  static constexpr int kStageBytes = 2 * kChunkBytes;
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kAbortOff = kBarOff + 2 * kStages * 8;
+  static constexpr int kBytes = kAbortOff + 16;
+  static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ long long chunk_begin(const DecodeParams& p, int cta) {
+  return static_cast<long long>(cta) * p.total / p.grid;
+}
+
+template <int D, bool BF16>
+__device__ __forceinline__ void load_slice(const uint8_t* row, int lane, float (&x)[D / 32]) {
+  constexpr int E = D / 32;  // elements per lane
+  if constexpr (E == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(row + lane * 8);
+    unpack2<BF16>(u.x, x[0], x[1]);
+    unpack2<BF16>(u.y, x[2], x[3]);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(row + lane * 4);
+    unpack2<BF16>(u, x[0], x[1]);
+  }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_decode_split_sm100(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                          const uint16_t* __restrict__ v, float* __restrict__ part_o,
+                          float* __restrict__ part_lse, const DecodeParams p,
+                          int* __restrict__ status) {
+  using C = DecodeCfg<D>;
+  constexpr int S = C::kStages;
+  constexpr int E = D / 32;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + C::kBarOff;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kAbortOff);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bars + 8 * s, 1);             // full: producer's expect_tx + bytes
+      mbar_init(bars + 8 * (S + s), kWarps);  // empty: one arrival per consumer warp
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const long long c_begin = chunk_begin(p, blockIdx.x);
+  const long long c_end = chunk_begin(p, blockIdx.x + 1);
+
+  if (warp == kWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t policy = l2_policy_evict_first();
+      uint32_t ld = 0;
+      bool ok = true;
+      for (long long c = c_begin; c < c_end; ++c, ++ld) {
+        const int h = static_cast<int>(c / p.n_chunks);
+        const int key0 = static_cast<int>(c % p.n_chunks) * kDecodeChunk;
+        const int nk = min(kDecodeChunk, p.Nkv - key0);
+        const uint32_t bytes = static_cast<uint32_t>(nk) * D * 2;
+        const uint32_t slot = ld % S;
+        if (!mbar_wait(bars + 8 * (S + slot), ((ld / S) & 1) ^ 1, status, abort_flag,
+                       kStatusTimeoutDecode)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = bars + 8 * slot;
+        mbar_arrive_expect_tx(fb, 2 * bytes);
+        const size_t off = (static_cast<size_t>(h) * p.Nkv + key0) * D;
+        const uint32_t dst = sbase + slot * C::kStageBytes;
+        bulk_load_stream(dst, k + off, bytes, fb, policy);
+        bulk_load_stream(dst + C::kChunkBytes, v + off, bytes, fb, policy);
+      }
+      if (!ok) {
+        for (uint32_t i = (ld > (uint32_t)S ? ld - S : 0); i < ld; ++i) {
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(bars + 8 * (i % S), (i / S) & 1))
+            if (global_timer_ns() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const long long first_head = c_begin / p.n_chunks;
+    // Key (0..7 within this warp's 8) whose full dot product this lane ends up holding.
+    const int my_key = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+
+    float qv[E], acc[E];
+    float m = -INFINITY, l_lane = 0.f;
+    int cur_h = -1;
+    uint32_t ld = 0;
+    bool ok = true;
+
+    // Writes this warp's partial record for head h: its keys' normalised output and
+    // log-sum-exp.  No cross-warp synchronisation: the combine kernel merges the warps.
+    auto finish_segment = [&](int h) {
+      float l_w = l_lane;
+#pragma unroll
+      for (int s = 16; s > 0; s >>= 1) l_w += __shfl_xor_sync(0xffffffffu, l_w, s);
+      const long long rec =
+          (static_cast<long long>(blockIdx.x) * p.max_seg + (h - first_head)) * kWarps + warp;
+      const float inv = (l_w > 0.f) ? 1.0f / l_w : 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) part_o[rec * D + lane * E + e] = acc[e] * inv;
+      if (lane == 0)
+        part_lse[rec] = (l_w > 0.f) ? (m + log2f(l_w)) * 0.69314718055994531f : -INFINITY;
+    };
+
+    for (long long c = c_begin; c < c_end; ++c, ++ld) {
+      const int h = static_cast<int>(c / p.n_chunks);
+      const int key0 = static_cast<int>(c % p.n_chunks) * kDecodeChunk;
+      const int nk = min(kDecodeChunk, p.Nkv - key0);
+      if (h != cur_h) {
+        if (cur_h >= 0) finish_segment(cur_h);
+        cur_h = h;
+        float qf[E];
+        load_slice<D, BF16>(reinterpret_cast<const uint8_t*>(q + static_cast<size_t>(h) * D), lane, qf);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          qv[e] = qf[e] * p.scale_log2;  // scores come out in log2 units
+          acc[e] = 0.f;
+        }
+        m = -INFINITY;
+        l_lane = 0.f;
+      }
+      const uint32_t slot = ld % S;
+      const bool got = mbar_wait(bars + 8 * slot, (ld / S) & 1, status, abort_flag,
+                                 kStatusTimeoutDecode);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      const uint8_t* ks = smem + slot * C::kStageBytes + warp * kKeysPerWarp * D * 2;
+      const uint8_t* vs = ks + C::kChunkBytes;
+
+      // Partial dot products of this lane's d-slice with the warp's 8 keys.
+      float part[8];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        float kx[E];
+        load_slice<D, BF16>(ks + kk * D * 2, lane, kx);
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) a = fmaf(qv[e], kx[e], a);
+        part[kk] = a;
+      }
+      // Transposing butterfly: after it every lane holds the full score of key my_key.
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 16;
+        const float keep = up ? part[i + 4] : part[i];
+        const float send = up ? part[i] : part[i + 4];
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 8;
+        const float keep = up ? part[i + 2] : part[i];
+        const float send = up ? part[i] : part[i + 2];
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+      {
+        const bool up = lane & 4;
+        const float keep = up ? part[1] : part[0];
+        const float send = up ? part[0] : part[1];
+        part[0] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+      part[0] += __shfl_xor_sync(0xffffffffu, part[0], 2);
+      part[0] += __shfl_xor_sync(0xffffffffu, part[0], 1);
+      const int nvalid = nk - warp * kKeysPerWarp;  // keys of this warp inside the chunk
+      const float x = (my_key < nvalid) ? part[0] : -INFINITY;
+
+      // Online softmax over the warp's keys (eager: one exp2 for alpha per chunk).
+      float mx = x;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m, mx);
+      const float m_eff = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = ex2(m - m_eff);  // 0 when m was -inf
+      const float pe = ex2(x - m_eff);
+      l_lane = l_lane * alpha + (((lane & 3) == 0) ? pe : 0.f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] *= alpha;
+      m = m_new;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        if (kk >= nvalid) break;
+        const int src = (((kk >> 2) & 1) << 4) | (((kk >> 1) & 1) << 3) | ((kk & 1) << 2);
+        const float pk = __shfl_sync(0xffffffffu, pe, src);
+        float vx[E];
+        load_slice<D, BF16>(vs + kk * D * 2, lane, vx);
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(pk, vx[e], acc[e]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (S + slot));
+    }
+    if (ok && cur_h >= 0) finish_segment(cur_h);
+  }
+  __syncthreads();
+}
+
+template <int D, bool OF32>
+__global__ void __launch_bounds__(128)
+    fa_decode_combine(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                      void* __restrict__ o, float* __restrict__ lse, const DecodeParams p) {
+  const int h = blockIdx.x;
+  const int c = threadIdx.x;
+  // CTAs whose chunk ranges intersect head h's chunks [x0, x1].
+  const long long x0 = static_cast<long long>(h) * p.n_chunks;
+  const long long x1 = x0 + p.n_chunks - 1;
+  auto cta_of = [&](long long x) {
+    long long g = x * p.grid / p.total;
+    while (g + 1 < p.grid && chunk_begin(p, static_cast<int>(g + 1)) <= x) ++g;
+    while (g > 0 && chunk_begin(p, static_cast<int>(g)) > x) --g;
+    return static_cast<int>(g);
+  };
+  const int lo = cta_of(x0), hi = cta_of(x1);
+  float M = -INFINITY;
+  for (int g = lo; g <= hi; ++g) {
+    const long long rec0 = (static_cast<long long>(g) * p.max_seg + (h - chunk_begin(p, g) / p.n_chunks)) * kWarps;
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, part_lse[rec0 + w]);
+  }
+  float L = 0.f, acc = 0.f;
+  if (M != -INFINITY) {
+    for (int g = lo; g <= hi; ++g) {
+      const long long rec0 = (static_cast<long long>(g) * p.max_seg + (h - chunk_begin(p, g) / p.n_chunks)) * kWarps;
+      for (int w = 0; w < kWarps; ++w) {
+        const float ls = part_lse[rec0 + w];
+        const float wt = (ls == -INFINITY) ? 0.f : expf(ls - M);
+        L += wt;
+        acc = fmaf(wt, part_o[(rec0 + w) * D + c], acc);
+      }
+    }
+  }
+  const float out = (L > 0.f) ? acc / L : 0.f;
+  if constexpr (OF32) {
+    static_cast<float*>(o)[static_cast<size_t>(h) * D + c] = out;
+  }
+  if (c == 0 && lse != nullptr) lse[h] = (L > 0.f) ? M + logf(L) : -INFINITY;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(128)
+    fa_decode_combine16(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                        uint16_t* __restrict__ o, float* __restrict__ lse, const DecodeParams p) {
+  // Same merge as fa_decode_combine, output rounded to the input's 16-bit type.
+  const int h = blockIdx.x;
+  const int c = threadIdx.x;
+  const long long x0 = static_cast<long long>(h) * p.n_chunks;
+  const long long x1 = x0 + p.n_chunks - 1;
+  auto cta_of = [&](long long x) {
+    long long g = x * p.grid / p.total;
+    while (g + 1 < p.grid && chunk_begin(p, static_cast<int>(g + 1)) <= x) ++g;
+    while (g > 0 && chunk_begin(p, static_cast<int>(g)) > x) --g;
+    return static_cast<int>(g);
+  };
+  const int lo = cta_of(x0), hi = cta_of(x1);
+  float M = -INFINITY;
+  for (int g = lo; g <= hi; ++g) {
+    const long long rec0 = (static_cast<long long>(g) * p.max_seg + (h - chunk_begin(p, g) / p.n_chunks)) * kWarps;
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, part_lse[rec0 + w]);
+  }
+  float L = 0.f, acc = 0.f;
+  if (M != -INFINITY) {
+    for (int g = lo; g <= hi; ++g) {
+      const long long rec0 = (static_cast<long long>(g) * p.max_seg + (h - chunk_begin(p, g) / p.n_chunks)) * kWarps;
+      for (int w = 0; w < kWarps; ++w) {
+        const float ls = part_lse[rec0 + w];
+        const float wt = (ls == -INFINITY) ? 0.f : expf(ls - M);
+        L += wt;
+        acc = fmaf(wt, part_o[(rec0 + w) * D + c], acc);
+      }
+    }
+  }
+  const float out = (L > 0.f) ? acc / L : 0.f;
+  if constexpr (BF16) {
+    o[static_cast<size_t>(h) * D + c] = __bfloat16_as_ushort(__float2bfloat16_rn(out));
+  } else {
+    o[static_cast<size_t>(h) * D + c] = __half_as_ushort(__float2half_rn(out));
+  }
+  if (c == 0 && lse != nullptr) lse[h] = (L > 0.f) ? M + logf(L) : -INFINITY;
+}
+
+template <int D, bool BF16>
+cudaError_t launch_t(const void* q, const void* k, const void* v, void* o, float* lse,
+                     const DecodeParams& p, bool o_f32, float* part_o, float* part_lse,
+                     int* status, cudaStream_t stream) {
+  auto kern = fa_decode_split_sm100<D, BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       DecodeCfg<D>::kBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<p.grid, kThreads, DecodeCfg<D>::kBytes, stream>>>(
+      static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+      static_cast<const uint16_t*>(v), part_o, part_lse, p, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (o_f32)
+    fa_decode_combine<D, true><<<p.BH, D, 0, stream>>>(part_o, part_lse, o, lse, p);
+  else
+    fa_decode_combine16<D, BF16><<<p.BH, D, 0, stream>>>(part_o, part_lse,
+                                                          static_cast<uint16_t*>(o), lse, p);
+  return cudaGetLastError();
+}
+
+// Diagnostic: one thread waits on an mbarrier that nothing ever arrives on.  The
+// bounded wait gives up after kWaitLimitNs, records kStatusTimeoutDecode in the status
+// word and the kernel returns -- the same path a real stall would take.
+__global__ void fa_wait_timeout_selftest(int* __restrict__ status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    mbar_wait(smem_u32(&bar), 0, status, &abort_flag, kStatusTimeoutDecode);
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t stream) {
+  fa_wait_timeout_selftest<<<1, 32, 0, stream>>>(status);
+  return cudaGetLastError();
+}
+
+size_t decode_smem_bytes(int d) {
+  return d == 128 ? DecodeCfg<128>::kBytes : DecodeCfg<64>::kBytes;
+}
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const DecodeParams& p, int d, bool bf16, bool o_f32, float* part_o,
+                          float* part_lse, int* status, cudaStream_t stream) {
+  if (d == 128 && bf16) return launch_t<128, true>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream);
+  if (d == 128 && !bf16) return launch_t<128, false>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream);
+  if (d == 64 && bf16) return launch_t<64, true>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream);
+  if (d == 64 && !bf16) return launch_t<64, false>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

@@ -1,0 +1,52 @@
+// fa_internal.h -- launch interfaces shared by the host API and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+// Work description of one prefill launch (all sizes in elements / rows / tiles).
+struct PrefillParams {
+  int BH;           // B * H
+  int Nq, Nkv;
+  int off;          // Nkv - Nq: causal query i sees keys j <= i + off
+  int causal;
+  int n_qtiles;     // ceil(Nq / 128)
+  int n_pairs;      // ceil(n_qtiles / 2): a CTA work unit is two consecutive Q tiles
+  int n_kvtiles;    // ceil(Nkv / 128)
+  int n_units;      // BH * n_pairs
+  float scale_log2; // scale * log2(e)
+};
+
+// Work description of one split-KV decode launch.
+struct DecodeParams {
+  int BH;
+  int Nkv;
+  int n_chunks;       // chunks of kDecodeChunk keys per head
+  long long total;    // BH * n_chunks
+  int grid;           // CTAs: CTA c owns chunks [c*total/grid, (c+1)*total/grid)
+  int max_seg;        // most heads one CTA's chunk range can touch
+  float scale_log2;
+};
+
+constexpr int kDecodeChunk = 64;
+
+// Kernel launchers (fa_prefill.cu, fa_decode.cu).  Return the launch's cudaError_t.
+cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           void* o, float* lse, const PrefillParams& p, int d, bool bf16,
+                           bool o_f32, int grid, int* status, cudaStream_t stream);
+
+cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const DecodeParams& p, int d, bool bf16, bool o_f32, float* part_o,
+                          float* part_lse, int* status, cudaStream_t stream);
+
+// Diagnostic kernel whose only wait can never finish (see fa_selftest_wait_timeout).
+cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t stream);
+
+// Bytes of dynamic shared memory each kernel needs.
+size_t prefill_smem_bytes(int d);
+size_t decode_smem_bytes(int d);
+
+}  // namespace fa

@@ -1,0 +1,525 @@
+// fa_prefill.cu -- exact fused attention forward for Nq > 1 on sm_100a.
+//
+// The method ("FlashAttention" (fp-ai-systems), sections "The fix: tile through SRAM,
+// fuse the passes" and "Online softmax: the enabling trick"; "FlashAttention 1-2-3"
+// (myaihardware), sections "FlashAttention-1", "FlashAttention-2" and "The Math Behind
+// the Online Softmax Trick"): each Q tile owns its output and walks the K/V tiles; the
+// score tile S = Q K^T lives only on chip; a running row max m and running sum l let the
+// partial output be rescaled as new tiles arrive; O is divided by l once at the end and
+// written to HBM with the row's log-sum-exp.  Causal tiles beyond the diagonal are never
+// loaded or computed; only tiles that straddle the diagonal or the key tail are masked.
+//
+// The B200 mapping (our design, not the pages' A100/H100 sketches):
+//  * one persistent CTA per SM; a work unit is two 128-row Q tiles of one (b, h);
+//  * warp 0 (one lane) streams Q and the K/V tiles with TMA (128-byte swizzle) into a
+//    ring of shared-memory slots guarded by full/empty mbarriers;
+//  * warp 1 (one lane) issues tcgen05.mma: S_t = Q_t K^T into TMEM (fp32, 128 columns),
+//    then O_t += P_t V with P_t read from TMEM; the two Q tiles ping-pong so that one
+//    tile's softmax overlaps the other tile's matrix products;
+//  * warpgroups 1 and 2 run the softmax of tile 0 and tile 1, one thread per row: they
+//    read S from TMEM, apply scale and mask, update (m, l), write P as 16-bit into the
+//    S columns, rescale O in TMEM only when the max grows by more than 2^8 (lazy), and
+//    run the epilogue (O / l and LSE to global memory).
+//  TMEM map (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+d), O1 after it.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fa_device.cuh"
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+constexpr int BM = 128;  // query rows per tile (tcgen05 M)
+constexpr int BN = 128;  // keys per tile (tcgen05 N of S, K of P V)
+constexpr int kThreads = 384;
+constexpr int kRegsLaunch = 168;   // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsSide = 88;      // warpgroup 0 (load + MMA issue)
+constexpr int kRegsSoftmax = 208;  // warpgroups 1 and 2; 128*88 + 256*208 == 384*168
+static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+
+template <int D>
+struct PrefillCfg {
+  static constexpr int kQBytes = BM * D * 2;
+  static constexpr int kKVBytes = BN * D * 2;
+  static constexpr int kStages = (D == 128) ? 5 : 8;
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = 2 * kQBytes;
+  static constexpr int kBarOff = kRingOff + kStages * kKVBytes;
+  // mbarriers
+  static constexpr int kBarQFull = 0;
+  static constexpr int kBarQEmpty = 1;
+  static constexpr int kBarFull = 2;                 // + slot
+  static constexpr int kBarEmpty = 2 + kStages;      // + slot
+  static constexpr int kBarSFull = 2 + 2 * kStages;  // + tile
+  static constexpr int kBarPFull = kBarSFull + 2;    // + tile
+  static constexpr int kBarODone = kBarPFull + 2;    // + tile
+  static constexpr int kBarDrain = kBarODone + 2;
+  static constexpr int kBarDone = kBarDrain + 1;     // softmax warps finished with TMEM
+  static constexpr int kNumBars = kBarDone + 1;
+  static constexpr int kTmemHolderOff = kBarOff + kNumBars * 8;
+  static constexpr int kAbortOff = kTmemHolderOff + 4;
+  static constexpr int kBytes = kAbortOff + 4;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
+  static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t bars, int i) { return bars + 8u * i; }
+
+__device__ __forceinline__ void unit_coords(const PrefillParams& p, int u, int& bh, int& pair) {
+  // Heaviest first: the last Q-tile pairs (most causal work) of every head go first.
+  pair = p.n_pairs - 1 - u / p.BH;
+  bh = u % p.BH;
+}
+
+// Number of K/V tiles Q tile `qtile` must visit (0 when every row is fully masked).
+__device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, int qtile) {
+  if (qtile >= p.n_qtiles) return 0;
+  if (!p.causal) return p.n_kvtiles;
+  const int last_row = min(qtile * BM + BM - 1, p.Nq - 1);
+  const int last_key = last_row + p.off;
+  if (last_key < 0) return 0;
+  return min(p.n_kvtiles, last_key / BN + 1);
+}
+
+// Waits for TMA loads already issued, ignoring the abort flag (error path only).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) break;
+  }
+}
+
+// ---------------------------------------------------------------- producer (TMA)
+template <int D>
+__device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
+                         const PrefillParams& p, uint32_t sbase, uint32_t bars, int* status,
+                         volatile int* abort_flag) {
+  using C = PrefillCfg<D>;
+  constexpr int S = C::kStages;
+  uint32_t ld = 0, q_issued = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    int bh, pair;
+    unit_coords(p, u, bh, pair);
+    const int n0 = kv_tiles_for(p, 2 * pair), n1 = kv_tiles_for(p, 2 * pair + 1);
+    const int nmax = max(n0, n1);
+    if (nmax == 0) continue;
+    if (!mbar_wait(bar_addr(bars, C::kBarQEmpty), (q_issued & 1) ^ 1, status, abort_flag,
+                   kStatusTimeoutLoad)) {
+      ok = false;
+      break;
+    }
+    const uint32_t qf = bar_addr(bars, C::kBarQFull);
+    mbar_arrive_expect_tx(qf, ((n0 > 0) + (n1 > 0)) * C::kQBytes);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if ((t == 0 ? n0 : n1) == 0) continue;
+#pragma unroll
+      for (int sub = 0; sub < D / 64; ++sub)
+        tma_load_3d(sbase + C::kQOff + t * C::kQBytes + sub * BM * 128, tq, qf, sub * 64,
+                    (2 * pair + t) * BM, bh);
+    }
+    ++q_issued;
+    for (int j = 0; j < nmax && ok; ++j) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t slot = ld % S, ph = (ld / S) & 1;
+        if (!mbar_wait(bar_addr(bars, C::kBarEmpty + slot), ph ^ 1, status, abort_flag,
+                       kStatusTimeoutLoad)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = bar_addr(bars, C::kBarFull + slot);
+        mbar_arrive_expect_tx(fb, C::kKVBytes);
+        const uint32_t dst = sbase + C::kRingOff + slot * C::kKVBytes;
+#pragma unroll
+        for (int sub = 0; sub < D / 64; ++sub)
+          tma_load_3d(dst + sub * BN * 128, which ? tv : tk, fb, sub * 64, j * BN, bh);
+        ++ld;
+      }
+    }
+  }
+  if (!ok) {
+    // Let every copy still in flight land before the CTA's shared memory goes away.
+    for (uint32_t i = (ld > (uint32_t)S ? ld - S : 0); i < ld; ++i)
+      drain_wait(bar_addr(bars, C::kBarFull + i % S), (i / S) & 1);
+    if (q_issued) drain_wait(bar_addr(bars, C::kBarQFull), (q_issued - 1) & 1);
+  }
+}
+
+// ---------------------------------------------------------------- MMA issuer
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t qa, uint32_t ka, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    // K-major operand, 128-byte swizzle: 64-element column blocks of 128 rows x 128 B,
+    // 16 elements (32 B) per MMA step; 8-row groups 1024 B apart.
+    const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+    mma_ss(d_tmem, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+           idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t va,
+                                         uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < BN / 16; ++kk) {
+    // V is MN-major (d contiguous): 16 keys per step = two 1024-byte swizzle atoms;
+    // the second 64-column block of d lies BN*128 bytes further.
+    const uint64_t b = make_sdesc_sw128(va + kk * 16 * 128, BN * 128, 1024);
+    mma_ts(d_tmem, p_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D, bool BF16>
+__device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                           int* status, volatile int* abort_flag) {
+  using C = PrefillCfg<D>;
+  constexpr int S = C::kStages;
+  constexpr uint32_t idesc_s = make_idesc_f16(BM, BN, BF16, false);
+  constexpr uint32_t idesc_o = make_idesc_f16(BM, D, BF16, true);
+  uint32_t ld = 0, q_used = 0, pcount[2] = {0, 0};
+  bool ok = true;
+  auto wait = [&](int b, uint32_t parity) {
+    return mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutMma);
+  };
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    int bh, pair;
+    unit_coords(p, u, bh, pair);
+    const int n[2] = {kv_tiles_for(p, 2 * pair), kv_tiles_for(p, 2 * pair + 1)};
+    const int nmax = max(n[0], n[1]);
+    if (nmax == 0) continue;
+    if (!wait(C::kBarQFull, q_used & 1)) { ok = false; break; }
+    tc_fence_after();
+    // S_t(0) for both tiles from K_0.
+    const uint32_t kslot0 = ld % S;
+    if (!wait(C::kBarFull + kslot0, (ld / S) & 1)) { ok = false; break; }
+    tc_fence_after();
+    ++ld;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (n[t] == 0) continue;
+      issue_s<D>(tmem + t * 128, sbase + C::kQOff + t * C::kQBytes,
+                 sbase + C::kRingOff + kslot0 * C::kKVBytes, idesc_s);
+      tc_commit(bar_addr(bars, C::kBarSFull + t));
+    }
+    tc_commit(bar_addr(bars, C::kBarEmpty + kslot0));
+    for (int j = 0; j < nmax && ok; ++j) {
+      const uint32_t vslot = ld % S;
+      if (!wait(C::kBarFull + vslot, (ld / S) & 1)) { ok = false; break; }
+      tc_fence_after();
+      ++ld;
+      int knext = -1;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (j >= n[t]) continue;
+        if (!wait(C::kBarPFull + t, pcount[t] & 1)) { ok = false; break; }
+        ++pcount[t];
+        tc_fence_after();
+        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, sbase + C::kRingOff + vslot * C::kKVBytes,
+                    idesc_o, j > 0);
+        tc_commit(bar_addr(bars, C::kBarODone + t));
+        if (j + 1 < n[t]) {
+          if (knext < 0) {
+            knext = ld % S;
+            if (!wait(C::kBarFull + knext, (ld / S) & 1)) { ok = false; break; }
+            tc_fence_after();
+            ++ld;
+          }
+          issue_s<D>(tmem + t * 128, sbase + C::kQOff + t * C::kQBytes,
+                     sbase + C::kRingOff + knext * C::kKVBytes, idesc_s);
+          tc_commit(bar_addr(bars, C::kBarSFull + t));
+        }
+      }
+      if (!ok) break;
+      tc_commit(bar_addr(bars, C::kBarEmpty + vslot));
+      if (knext >= 0) tc_commit(bar_addr(bars, C::kBarEmpty + knext));
+    }
+    if (!ok) break;
+    tc_commit(bar_addr(bars, C::kBarQEmpty));
+    ++q_used;
+  }
+  // No MMA may still be running when the TMEM is released.
+  tc_commit(bar_addr(bars, C::kBarDrain));
+  drain_wait(bar_addr(bars, C::kBarDrain), 0);
+}
+
+// ---------------------------------------------------------------- softmax + epilogue
+template <int D, bool BF16, bool OF32>
+__device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t tmem, void* o,
+                                 float* lse, int t, int* status, volatile int* abort_flag) {
+  using C = PrefillCfg<D>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wq = warp & 3;          // this warp reaches TMEM lanes 32*wq .. 32*wq+31
+  const int r = wq * 32 + lane;     // row of the Q tile owned by this thread
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  const uint32_t tS = lane_base + t * 128;
+  const uint32_t tO = lane_base + 256 + t * D;
+  const float scale_log2 = p.scale_log2;
+  uint32_t s_seen = 0, o_seen = 0;
+  // Warp-uniform result: tcgen05.ld/st below are warp-collective, so a warp never splits
+  // on a wait that finished on some lanes and ran out on others.
+  auto wait = [&](int b, uint32_t parity) {
+    const bool ok = mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutSoftmax);
+    return __all_sync(0xffffffffu, ok);
+  };
+
+  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    int bh, pair;
+    unit_coords(p, u, bh, pair);
+    const int qtile = 2 * pair + t;
+    if (qtile >= p.n_qtiles) continue;
+    const int n_kv = kv_tiles_for(p, qtile);
+    const int row = qtile * BM + r;
+    // Last key this row may see (keys beyond Nkv are padding of the last tile).
+    const int limit = p.causal ? min(p.Nkv - 1, row + p.off) : p.Nkv - 1;
+    float m_used = -INFINITY;  // running max in log2 units (may lag the true max by <= 8)
+    float l = 0.f;             // running sum of 2^(x - m_used)
+
+    for (int j = 0; j < n_kv; ++j) {
+      if (!wait(C::kBarSFull + t, s_seen & 1)) return;
+      ++s_seen;
+      tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
+      tmem_ld_wait_only();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+
+      // x = s * scale * log2(e); masked entries -inf.
+      const int lim_c = limit - j * BN;
+      float mx = -INFINITY;
+      if (lim_c >= BN - 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = __uint_as_float(s[c][i]) * scale_log2;
+            s[c][i] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x = (c * 32 + i <= lim_c) ? __uint_as_float(s[c][i]) * scale_log2 : -INFINITY;
+            s[c][i] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+      }
+      const float m_new = fmaxf(m_used, mx);
+      // Lazy rescale: move the reference max only when it grows by more than 8 (log2),
+      // so p = 2^(x - m_used) stays <= 256.  -inf -> finite always moves; -inf -> -inf
+      // gives NaN and never moves.
+      const bool move = (m_new - m_used) > 8.0f;
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
+        // O_t still holds P V of tiles < j: wait for the last of those products.
+        if (!wait(C::kBarODone + t, (o_seen + j - 1) & 1)) return;
+        tc_fence_after();
+        const float alpha = move ? ex2(m_used - m_new) : 1.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ob[32];
+          tmem_ld_32x32b_x32(tO + cc * 32, ob);
+          tmem_ld_wait(ob);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
+          tmem_st_32x32b_x32(tO + cc * 32, ob);
+        }
+      }
+      if (move) {
+        l *= ex2(m_used - m_new);
+        m_used = m_new;
+      }
+      const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(__uint_as_float(s[c][2 * i]) - m_eff);
+          const float p1 = ex2(__uint_as_float(s[c][2 * i + 1]) - m_eff);
+          pk[i] = pack2<BF16>(p0, p1);
+          // l sums the same rounded P that the P V product uses, so a row dominated by
+          // one key normalises exactly.
+          float r0, r1;
+          unpack2<BF16>(pk[i], r0, r1);
+          rs += r0 + r1;
+        }
+        // P (16-bit, two per column) overwrites the first 64 columns of S.
+        tmem_st_32x32b_x16(tS + c * 16, pk);
+      }
+      l += rs;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_addr(bars, C::kBarPFull + t));
+    }
+
+    // Epilogue: O = O_t / l and LSE = (m + log2 l) * ln 2.
+    if (n_kv > 0) {
+      if (!wait(C::kBarODone + t, (o_seen + n_kv - 1) & 1)) return;
+      tc_fence_after();
+      o_seen += n_kv;
+    }
+    const bool valid = row < p.Nq;
+    const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+    const size_t orow = (static_cast<size_t>(bh) * p.Nq + row) * D;
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t ob[32];
+      if (n_kv > 0) {
+        tmem_ld_32x32b_x32(tO + cc * 32, ob);
+        tmem_ld_wait(ob);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ob[i] = 0u;
+      }
+      if (valid) {
+        if constexpr (OF32) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(o) + orow + cc * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(ob[4 * i]) * inv_l, __uint_as_float(ob[4 * i + 1]) * inv_l,
+                                 __uint_as_float(ob[4 * i + 2]) * inv_l, __uint_as_float(ob[4 * i + 3]) * inv_l);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(o) + orow + cc * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack2<BF16>(__uint_as_float(ob[8 * i + 2 * e]) * inv_l,
+                                 __uint_as_float(ob[8 * i + 2 * e + 1]) * inv_l);
+            dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+    if (valid && lse != nullptr)
+      lse[static_cast<size_t>(bh) * p.Nq + row] =
+          (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+  }
+}
+
+template <int D, bool BF16, bool OF32>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_prefill_sm100(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                     const __grid_constant__ CUtensorMap tv, void* __restrict__ o,
+                     float* __restrict__ lse, const PrefillParams p, int* __restrict__ status) {
+  using C = PrefillCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sbase - raw);
+  const uint32_t bars = sbase + C::kBarOff;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + C::kAbortOff);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sgen + C::kTmemHolderOff);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_addr(bars, C::kBarQFull), 1);
+    mbar_init(bar_addr(bars, C::kBarQEmpty), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar_addr(bars, C::kBarFull + s), 1);
+      mbar_init(bar_addr(bars, C::kBarEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_addr(bars, C::kBarSFull + t), 1);
+      mbar_init(bar_addr(bars, C::kBarPFull + t), 128);
+      mbar_init(bar_addr(bars, C::kBarODone + t), 1);
+    }
+    mbar_init(bar_addr(bars, C::kBarDrain), 1);
+    mbar_init(bar_addr(bars, C::kBarDone), 256);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  // Each role runs to the end of the kernel on its own path: warps with different
+  // register budgets never re-join.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
+    if (warp == 0) {
+      if (lane == 0) producer<D>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
+    } else if (warp == 1) {
+      if (lane == 0) mma_issuer<D, BF16>(p, sbase, bars, tmem, status, abort_flag);
+      __syncwarp();
+      // Release TMEM once both softmax warpgroups have finished reading it.
+      drain_wait(bar_addr(bars, C::kBarDone), 0);
+      __syncwarp();
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    softmax_epilogue<D, BF16, OF32>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+    tc_fence_before();
+    mbar_arrive(bar_addr(bars, C::kBarDone));
+  }
+}
+
+template <int D, bool BF16, bool OF32>
+cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
+                     float* lse, const PrefillParams& p, int grid, int* status,
+                     cudaStream_t stream) {
+  auto kern = fa_prefill_sm100<D, BF16, OF32>;
+  static bool configured = false;  // per template instance
+  static cudaError_t config_err = cudaSuccess;
+  if (!configured) {
+    config_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      PrefillCfg<D>::kAlloc);
+    if (config_err == cudaSuccess) {
+      cudaFuncAttributes attr;
+      config_err = cudaFuncGetAttributes(&attr, kern);
+      // setmaxnreg redistributes the registers the block was launched with; a launch
+      // with fewer would make the increase wait forever.
+      if (config_err == cudaSuccess && attr.numRegs < kRegsLaunch) config_err = cudaErrorInvalidConfiguration;
+    }
+    configured = true;
+  }
+  if (config_err != cudaSuccess) return config_err;
+  kern<<<grid, kThreads, PrefillCfg<D>::kAlloc, stream>>>(tq, tk, tv, o, lse, p, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t prefill_smem_bytes(int d) {
+  return d == 128 ? PrefillCfg<128>::kAlloc : PrefillCfg<64>::kAlloc;
+}
+
+cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           void* o, float* lse, const PrefillParams& p, int d, bool bf16,
+                           bool o_f32, int grid, int* status, cudaStream_t stream) {
+#define FA_PREFILL_CASE(D_, B_, F_) \
+  if (d == D_ && bf16 == B_ && o_f32 == F_) return launch_t<D_, B_, F_>(tq, tk, tv, o, lse, p, grid, status, stream);
+  FA_PREFILL_CASE(128, true, true)
+  FA_PREFILL_CASE(128, true, false)
+  FA_PREFILL_CASE(128, false, true)
+  FA_PREFILL_CASE(128, false, false)
+  FA_PREFILL_CASE(64, true, true)
+  FA_PREFILL_CASE(64, true, false)
+  FA_PREFILL_CASE(64, false, true)
+  FA_PREFILL_CASE(64, false, false)
+#undef FA_PREFILL_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fa

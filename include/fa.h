@@ -1,0 +1,150 @@
+/*
+ * fa.h -- C ABI of libfa_b200.so: exact fused scaled-dot-product attention forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed ("Flash Attention -- Module 12.3" (aicurriculum), section
+ * "Definition": exact softmax(Q K^T / sqrt(d)) V; "FlashAttention" (fp-ai-systems),
+ * sections "The problem: the n x n score matrix" and "The fix: tile through SRAM, fuse
+ * the passes"; "FlashAttention 1-2-3" (myaihardware), sections "FlashAttention-1",
+ * "FlashAttention-2" (causal block skipping), "The Math Behind the Online Softmax
+ * Trick" and "Beyond FlashAttention" (split-KV decoding)):
+ *
+ *     S   = scale * Q K^T            (never written to memory)
+ *     P   = softmax(S [+ causal mask]) over each row
+ *     O   = P V
+ *     LSE = per-row natural log of sum_j exp(S_ij) over the visible keys
+ *
+ * Layouts (all contiguous, d innermost, no strides):
+ *     q   [B, H, Nq,  d]   16-bit (in_dtype)
+ *     k   [B, H, Nkv, d]   16-bit (in_dtype)
+ *     v   [B, H, Nkv, d]   16-bit (in_dtype)
+ *     o   [B, H, Nq,  d]   o_dtype (FA_F32, or the same 16-bit type as the inputs)
+ *     lse [B, H, Nq]       fp32, natural log; may be NULL (then not written)
+ * All pointers are DEVICE pointers on the current CUDA device; q, k, v and o must be
+ * 16-byte aligned, lse 4-byte aligned.  K and V have H heads like Q.
+ *
+ * Causal masking: query i sees key j iff j <= i + (Nkv - Nq) (aligned bottom-right; the
+ * pages only show square masks, where this is the usual lower triangle).  A query that
+ * sees no key (only possible when Nq > Nkv) gets O = 0 and LSE = -inf.
+ *
+ * Ownership and ordering: the caller owns every buffer.  Calls only enqueue work on
+ * `stream` (a cudaStream_t; NULL = the legacy default stream) and never synchronise
+ * it; the buffers must stay valid until that work has finished.  The library keeps no
+ * pointer to caller memory after a call returns.  It owns two per-device allocations:
+ * a 256-byte device status word (allocated on the first call on a device) and, for
+ * decode, a grow-only workspace for the split partials (allocated with cudaMalloc on the
+ * first decode call that needs more; do that first call outside stream capture).
+ * Decode calls on one device share that workspace, so decode calls that can run
+ * concurrently (different streams without ordering between them) race on it.
+ *
+ * Errors: argument checks run on the host before anything is enqueued; a failed check
+ * returns its code and launches nothing.  FA_ERR_CUDA means a CUDA runtime call failed;
+ * fa_last_cuda_error() returns the cudaError_t.  Device-side faults are never raised on
+ * purpose: every wait inside the kernels is bounded (about 1 s); a wait that runs out
+ * sets bits in the device status word and the kernel returns early, leaving the outputs
+ * undefined.  Read (and clear) that word with fa_device_status() after synchronising.
+ *
+ * Determinism: tile sizes, the CTA count and the split partition depend only on the
+ * shape and the device, so equal inputs give bitwise-equal outputs.
+ */
+#ifndef FA_B200_H_
+#define FA_B200_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, misalignment, overlap, ... */
+  FA_ERR_UNSUPPORTED = 2,     /* valid request this build does not implement (d, dtype pair) */
+  FA_ERR_ARCH = 3,            /* current device is not compute capability 10.0 (B200) */
+  FA_ERR_CUDA = 4,            /* a CUDA runtime call failed: see fa_last_cuda_error() */
+  FA_ERR_NOMEM = 5,           /* a library-owned allocation failed */
+  FA_ERR_DEVICE_TIMEOUT = 6   /* fa_device_status(): a kernel's bounded wait ran out */
+};
+
+/* Element types. */
+enum { FA_F16 = 0, FA_BF16 = 1, FA_F32 = 2 };
+
+/*
+ * fa_fwd -- attention forward; the general entry point.
+ *   Nq == 1 runs the split-KV decode path (every key is visible to the single query
+ *   whatever `causal` says, by the bottom-right alignment); Nq > 1 runs the tiled
+ *   prefill path.
+ *   B, H, Nq, Nkv >= 1; d in {64, 128}; B*H <= 2^31-1; scale any finite float (use
+ *   1/sqrt(d) for the usual attention); causal 0 or 1; in_dtype FA_F16 or FA_BF16;
+ *   o_dtype FA_F32 or equal to in_dtype.  o must not overlap q, k, v or lse.
+ * Returns FA_OK once the work is enqueued.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+           int Nq, int Nkv, int d, float scale, int causal, void* stream, int in_dtype,
+           int o_dtype);
+
+/*
+ * fa_fwd_prefill -- the tiled prefill path for any Nq >= 1 (the work of fa_fwd with
+ * Nq > 1).  num_ctas: persistent CTAs to launch; 0 picks one per SM, larger values are
+ * clamped to the number of work units (pairs of 128-row query tiles).  Same arguments,
+ * layouts and errors as fa_fwd.
+ */
+int fa_fwd_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
+                   int in_dtype, int o_dtype, int num_ctas);
+
+/*
+ * fa_fwd_decode -- split-KV decode for one query per head: q [B,H,1,d], k/v [B,H,Nkv,d],
+ * o [B,H,1,d], lse [B,H,1].  num_splits: CTAs that split the flat range of all heads'
+ * 64-key chunks evenly between them (0 picks one per SM; clamped to the chunk count).
+ * Enqueues the split kernel and the fp32 log-sum-exp combine kernel on `stream`.
+ */
+int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int H, int Nkv, int d, float scale, void* stream, int in_dtype, int o_dtype,
+                  int num_splits);
+
+/* Bytes of decode workspace a fa_fwd_decode call with these arguments needs. */
+int fa_decode_workspace_bytes(int B, int H, int Nkv, int d, int num_splits, size_t* bytes);
+
+/*
+ * fa_device_status -- reads the current device's status word into *status (0 = no
+ * kernel wait ran out; otherwise FA_DEV_* bits) and clears it when clear != 0.
+ * Synchronous (a device-to-host copy on the legacy stream).  Returns FA_OK, or
+ * FA_ERR_DEVICE_TIMEOUT when the word is non-zero.
+ */
+int fa_device_status(int* status, int clear);
+
+/* Bits of the device status word. */
+enum {
+  FA_DEV_TIMEOUT_LOAD = 1,      /* prefill: a TMA producer wait ran out */
+  FA_DEV_TIMEOUT_MMA = 2,       /* prefill: the MMA issuer's wait ran out */
+  FA_DEV_TIMEOUT_SOFTMAX = 4,   /* prefill: a softmax / epilogue wait ran out */
+  FA_DEV_TIMEOUT_DECODE = 8     /* decode: a split kernel wait ran out */
+};
+
+/*
+ * fa_selftest_wait_timeout -- diagnostic for the error path above: enqueues a one-thread
+ * kernel that waits on an mbarrier nothing ever signals.  Its bounded wait gives up after
+ * about 1 s, sets FA_DEV_TIMEOUT_DECODE in the status word and returns; no fault, trap or
+ * hang.  Synchronise, then fa_device_status() reports it.
+ */
+int fa_selftest_wait_timeout(void* stream);
+
+/* Frees the current device's decode workspace (synchronises the device). */
+int fa_release_workspace(void);
+
+/* The cudaError_t behind the last FA_ERR_CUDA returned on this host thread. */
+int fa_last_cuda_error(void);
+
+/* A static, human-readable name for a status code. */
+const char* fa_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H_ */

@@ -1,0 +1,113 @@
+"""The C-ABI library: it loads, exports every symbol include/fa.h declares, and its
+host-side argument checks return the documented codes without touching a device.
+
+Pointers below are fake integers; every case is rejected before any CUDA call, so these
+tests run on a CPU-only machine (and launch nothing on a GPU machine)."""
+import math
+import subprocess
+
+import pytest
+import torch
+
+from exact_io_aware_59_b200 import binding
+from exact_io_aware_59_b200 import build as fa_build
+
+A = 1 << 20  # fake, 16-byte aligned, non-overlapping "device" addresses
+Q, K, V, O, L = A * 1, A * 2, A * 3, A * 4, A * 5
+
+
+def _fwd(**kw):
+    args = dict(q=Q, k=K, v=V, o=O, lse=L, B=1, H=2, Nq=16, Nkv=16, d=64, scale=0.125,
+                causal=0, stream=None, in_dtype=binding.FA_F16, o_dtype=binding.FA_F32)
+    args.update(kw)
+    return binding.fa_fwd(**args)
+
+
+def test_library_builds_and_loads():
+    assert fa_build.build().endswith("libfa_b200.so")
+    lib = binding.library()
+    assert lib.fa_version() == 100
+
+
+def test_every_declared_symbol_is_exported():
+    declared = binding.declared_functions()
+    assert len(declared) >= 9
+    nm = subprocess.run(["nm", "-D", "--defined-only", fa_build.LIB_PATH],
+                        capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in nm.splitlines() if " T " in line}
+    missing = [f for f in declared if f not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    lib = binding.library()
+    for f in declared:
+        assert hasattr(lib, f)
+
+
+def test_status_strings():
+    for code in range(7):
+        assert binding.status_string(code) != "unknown status"
+    assert binding.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), binding.FA_ERR_INVALID_ARG),
+    (dict(k=None), binding.FA_ERR_INVALID_ARG),
+    (dict(v=None), binding.FA_ERR_INVALID_ARG),
+    (dict(o=None), binding.FA_ERR_INVALID_ARG),
+    (dict(B=0), binding.FA_ERR_INVALID_ARG),
+    (dict(H=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(Nq=0), binding.FA_ERR_INVALID_ARG),
+    (dict(Nkv=0), binding.FA_ERR_INVALID_ARG),
+    (dict(B=1 << 16, H=1 << 16), binding.FA_ERR_INVALID_ARG),
+    (dict(causal=2), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=math.nan), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=math.inf), binding.FA_ERR_INVALID_ARG),
+    (dict(in_dtype=binding.FA_F32), binding.FA_ERR_INVALID_ARG),
+    (dict(o_dtype=7), binding.FA_ERR_INVALID_ARG),
+    (dict(in_dtype=binding.FA_F16, o_dtype=binding.FA_BF16), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=256), binding.FA_ERR_UNSUPPORTED),
+    (dict(q=Q + 8), binding.FA_ERR_INVALID_ARG),
+    (dict(k=K + 2), binding.FA_ERR_INVALID_ARG),
+    (dict(o=O + 4), binding.FA_ERR_INVALID_ARG),
+    (dict(lse=L + 2), binding.FA_ERR_INVALID_ARG),
+    (dict(o=Q), binding.FA_ERR_INVALID_ARG),                 # O overlaps Q
+    (dict(o=K + 512), binding.FA_ERR_INVALID_ARG),           # O inside K
+    (dict(lse=O + 64), binding.FA_ERR_INVALID_ARG),          # LSE inside O
+    (dict(lse=V), binding.FA_ERR_INVALID_ARG),               # LSE on V
+])
+def test_argument_checks(kw, code):
+    assert _fwd(**kw) == code
+
+
+def test_prefill_and_decode_entry_checks():
+    lib = binding
+    assert lib.fa_fwd_prefill(Q, K, V, O, L, 1, 1, 4, 4, 64, 0.1, 0, None, 0, 2, -1) == \
+        binding.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_decode(Q, K, V, O, L, 1, 1, 4, 64, 0.1, None, 0, 2, -1) == \
+        binding.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_decode(None, K, V, O, L, 1, 1, 4, 64, 0.1, None, 0, 2, 0) == \
+        binding.FA_ERR_INVALID_ARG
+    assert lib.fa_fwd_decode(Q, K, V, O, L, 1, 1, 4, 80, 0.1, None, 0, 2, 0) == \
+        binding.FA_ERR_UNSUPPORTED
+
+
+def test_decode_workspace_size_formula():
+    # 8 partial records (one per consumer warp) per CTA per head segment, d+1 floats each.
+    B, H, Nkv, d, G = 16, 32, 32768, 128, 148
+    chunks = B * H * ((Nkv + 63) // 64)
+    per_cta = -(-chunks // G)
+    max_seg = -(-per_cta // ((Nkv + 63) // 64)) + 1
+    assert binding.fa_decode_workspace_bytes(B, H, Nkv, d, G) == G * max_seg * 8 * (d + 1) * 4
+    assert binding.fa_decode_workspace_bytes(1, 1, 10, 64, 5) == 1 * 2 * 8 * 65 * 4
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_valid_call_without_device_reports_cuda_error():
+    assert _fwd() == binding.FA_ERR_CUDA
+    assert binding.library().fa_last_cuda_error() != 0
+
+
+def test_binding_rejects_host_tensors():
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        binding.attention(q, q, q)

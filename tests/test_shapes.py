@@ -1,0 +1,120 @@
+"""GPU parity on ragged and edge shapes, with guard bands around every output.
+
+Covers: Nq and Nkv not multiples of the 128-row tile (tails), Nq != Nkv with the causal
+mask aligned bottom-right, causal rows that see no key (Nq > Nkv), one query row through
+the prefill path, head dims 64 and 128, fp16 and bf16, fp32 and 16-bit O, a persistent
+grid smaller than the work (num_ctas) and decode with several split counts.
+"""
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_59_b200 import binding
+from exact_io_aware_59_b200.inputs import make_qkv
+from fa_testlib import REL_O16, compare, has_b200
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 64  # elements of canary on each side of O and LSE (keeps 16-byte alignment)
+CANARY = 1234.5
+
+
+@pytest.fixture(autouse=True)
+def _device_clean():
+    if not has_b200():
+        pytest.skip("needs a B200 (sm_100a)")
+    binding.fa_device_status(clear=True)
+    yield
+    torch.cuda.synchronize()
+    assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+
+
+def _guarded(n, dtype):
+    buf = torch.full((n + 2 * GUARD,), CANARY, dtype=dtype, device="cuda")
+    return buf, buf[GUARD:GUARD + n]
+
+
+def _check_guard(buf, n):
+    assert (buf[:GUARD] == CANARY).all() and (buf[GUARD + n:] == CANARY).all(), \
+        "write outside the output buffer"
+
+
+def _run_case(B, H, Nq, Nkv, d, dtype, causal, out_dtype=torch.float32, scale=None,
+              num_ctas=0, num_splits=0, path="auto", seed=1):
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, dtype, seed)
+    scale = d ** -0.5 if scale is None else scale
+    n_o = B * H * Nq * d
+    obuf, o = _guarded(n_o, out_dtype)
+    lbuf, lse = _guarded(B * H * Nq, torch.float32)
+    binding.attention(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale,
+                      out=o.view(B, H, Nq, d), lse=lse.view(B, H, Nq), num_ctas=num_ctas,
+                      num_splits=num_splits, path=path)
+    torch.cuda.synchronize()
+    _check_guard(obuf, n_o)
+    _check_guard(lbuf, B * H * Nq)
+    o_ref, l_ref = oracle.attention(q, k, v, scale, causal)
+    rel = REL_O16[dtype] if out_dtype != torch.float32 else 0.0
+    return compare(o.view(B, H, Nq, d), lse.view(B, H, Nq), o_ref, l_ref, rel_o=rel)
+
+
+RAGGED = [
+    # B, H, Nq, Nkv
+    (1, 1, 2, 2),
+    (1, 2, 17, 17),
+    (2, 1, 127, 127),
+    (1, 1, 129, 129),
+    (1, 3, 255, 257),
+    (1, 2, 300, 1000),   # Nq < Nkv: bottom-right causal
+    (1, 2, 1000, 300),   # Nq > Nkv: early causal rows see nothing
+    (1, 1, 383, 130),
+    (2, 2, 513, 513),
+]
+
+
+@pytest.mark.parametrize("shape", RAGGED)
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)])
+def test_ragged_prefill(shape, causal, d, dtype):
+    _run_case(*shape, d, dtype, causal)
+
+
+@pytest.mark.parametrize("d,dtype", [(64, torch.bfloat16), (128, torch.float16)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_other_dtype_pairs(d, dtype, causal):
+    _run_case(2, 3, 333, 333, d, dtype, causal)
+
+
+@pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)])
+def test_16bit_output(d, dtype):
+    _run_case(1, 3, 400, 400, d, dtype, True, out_dtype=dtype)
+
+
+@pytest.mark.parametrize("num_ctas", [1, 3, 7])
+def test_persistent_grid_smaller_than_work(num_ctas):
+    _run_case(2, 3, 700, 700, 128, torch.bfloat16, True, num_ctas=num_ctas)
+
+
+@pytest.mark.parametrize("Nkv", [1, 5, 64, 65, 1000])
+def test_prefill_path_single_query(Nkv):
+    _run_case(2, 2, 1, Nkv, 128, torch.bfloat16, True, path="prefill")
+
+
+@pytest.mark.parametrize("Nkv", [1, 7, 63, 64, 65, 129, 4097])
+@pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)])
+def test_decode_shapes(Nkv, d, dtype):
+    _run_case(2, 3, 1, Nkv, d, dtype, False)
+
+
+@pytest.mark.parametrize("num_splits", [1, 2, 5, 16, 64, 1000])
+def test_decode_split_counts(num_splits):
+    _run_case(2, 4, 1, 3000, 128, torch.bfloat16, False, num_splits=num_splits)
+
+
+def test_decode_16bit_output():
+    _run_case(3, 2, 1, 2000, 128, torch.bfloat16, False, out_dtype=torch.bfloat16)
+
+
+def test_large_negative_and_zero_scale():
+    _run_case(1, 2, 260, 260, 128, torch.bfloat16, True, scale=0.0)
+    _run_case(1, 2, 260, 260, 128, torch.bfloat16, False, scale=-0.3)
+    _run_case(2, 2, 1, 900, 128, torch.bfloat16, False, scale=-0.3)
