@@ -196,8 +196,9 @@ def make_call(w: Workload, q, k, v, o, lse, stream):
     return call
 
 
-def run_workload(w: Workload, steps, warmup, ws, stream, out_dtype):
+def run_workload(w: Workload, steps, warmup, ws, stream, out_dtype=None):
     q, k, v = workload_qkv(w, device="cuda")
+    out_dtype = w.dtype if out_dtype is None else out_dtype
     o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=out_dtype, device="cuda")
     lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device="cuda")
     call = make_call(w, q, k, v, o, lse, stream)
@@ -311,10 +312,10 @@ def arm_ours(args, ws, rank, local):
     torch.cuda.set_device(local)
     stream = torch.cuda.Stream()
     peaks, peak_src = load_peaks()
-    out_dtype = torch.bfloat16
+    out_dtype = None  # O in the inputs' 16-bit type
 
     # prefill (headline)
-    wp = WORKLOADS[PREFILL]
+    wp = WORKLOADS[args.prefill_workload]
     with ClockSampler(local) as clk:
         ms_p, tensors = run_workload(wp, args.steps, args.warmup, ws, stream, out_dtype)
     assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
@@ -322,18 +323,12 @@ def arm_ours(args, ws, rank, local):
     tflops = flops / (ms_p * 1e-3) / 1e12
     value = tflops * ws
     peak_t = peaks["bf16_tflops"]
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "prefill_traffic.json")
-    if os.path.exists(prof):
-        with open(prof) as f:
-            t = json.load(f)
-        if t.get("kernel_rev") == KERNEL_REV:
-            traffic = t.get("bytes_per_launch")
+    traffic = DRAM_TRAFFIC.get((KERNEL_REV, wp.name))
 
     # decode
     decode = None
     if not args.skip_decode:
-        wd = WORKLOADS[DECODE]
+        wd = WORKLOADS[args.decode_workload]
         dsteps = max(3, args.steps // 8)
         with ClockSampler(local) as clk_d:
             ms_d, dt_ = run_workload(wd, dsteps, args.warmup, ws, stream, out_dtype)
@@ -392,6 +387,9 @@ def arm_ours(args, ws, rank, local):
 
 # Bumped whenever the prefill kernel changes, so stale ncu traffic is not reported.
 KERNEL_REV = "prefill-v1"
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the
+# kernel at this revision (profiles/fa_prefill_sm100_<workload>.md).
+DRAM_TRAFFIC = {("prefill-v1", "long_prefill_causal"): 629.5e6}
 
 
 def main():
@@ -400,6 +398,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--prefill-workload", default=PREFILL, choices=sorted(WORKLOADS))
+    ap.add_argument("--decode-workload", default=DECODE, choices=sorted(WORKLOADS))
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")

@@ -276,7 +276,8 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     // Last key this row may see (keys beyond Nkv are padding of the last tile).
     const int limit = p.causal ? min(p.Nkv - 1, row + p.off) : p.Nkv - 1;
     float m_used = -INFINITY;  // running max in log2 units (may lag the true max by <= 8)
-    float l = 0.f;             // running sum of 2^(x - m_used)
+    float l = 0.f;             // running sum of the 16-bit-rounded 2^(x - m_used): divides O
+    float l_exact = 0.f;       // the same sum before rounding: gives LSE
 
     for (int j = 0; j < n_kv; ++j) {
       if (!wait(C::kBarSFull + t, s_seen & 1)) return;
@@ -332,11 +333,13 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
         }
       }
       if (move) {
-        l *= ex2(m_used - m_new);
+        const float a = ex2(m_used - m_new);
+        l *= a;
+        l_exact *= a;
         m_used = m_new;
       }
       const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f;
+      float rs = 0.f, rs_exact = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -345,16 +348,18 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
           const float p0 = ex2(__uint_as_float(s[c][2 * i]) - m_eff);
           const float p1 = ex2(__uint_as_float(s[c][2 * i + 1]) - m_eff);
           pk[i] = pack2<BF16>(p0, p1);
-          // l sums the same rounded P that the P V product uses, so a row dominated by
-          // one key normalises exactly.
+          // O is divided by the sum of the same rounded P that the P V product uses, so
+          // a row dominated by one key normalises exactly; LSE uses the unrounded sum.
           float r0, r1;
           unpack2<BF16>(pk[i], r0, r1);
           rs += r0 + r1;
+          rs_exact += p0 + p1;
         }
         // P (16-bit, two per column) overwrites the first 64 columns of S.
         tmem_st_32x32b_x16(tS + c * 16, pk);
       }
       l += rs;
+      l_exact += rs_exact;
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_addr(bars, C::kBarPFull + t));
@@ -402,7 +407,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     }
     if (valid && lse != nullptr)
       lse[static_cast<size_t>(bh) * p.Nq + row] =
-          (l > 0.f) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+          (l_exact > 0.f) ? (m_used + log2f(l_exact)) * 0.69314718055994531f : -INFINITY;
   }
 }
 

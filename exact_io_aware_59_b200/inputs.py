@@ -56,6 +56,11 @@ WORKLOADS = {
         Workload("long_ctx_16k", 4, 1, 16, 16384, 16384, 128, torch.bfloat16, True),
         Workload("long_ctx_32k", 4, 1, 16, 32768, 32768, 128, torch.bfloat16, True),
         Workload("decode", 5, 16, 32, 1, 32768, 128, torch.bfloat16, False),
+        # Smaller cases of the same kernels, for profiler captures (still larger than L2).
+        Workload("decode_4k", 6, 16, 32, 1, 4096, 128, torch.bfloat16, False,
+                 note="profiling size: 1 GiB of K+V"),
+        Workload("prefill_causal_4k", 7, 1, 32, 4096, 4096, 128, torch.bfloat16, True,
+                 note="profiling size"),
     ]
 }
 

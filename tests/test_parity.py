@@ -66,9 +66,22 @@ def test_full_size_sampled(name):
     assert (o.abs().amax() <= v.abs().amax().float() + 1e-3).item(), "O outside the hull of V"
 
 
-def test_decode_full_size_sampled_heads():
+@pytest.mark.parametrize("name", ["long_prefill_causal", "long_prefill_peaky"])
+def test_full_size_sampled_16bit_out(name):
+    """The benchmark's launch configuration: 16-bit O."""
+    w = WORKLOADS[name]
+    q, k, v, o, lse = _run(w, out_dtype=w.dtype)
+    rows = sample_rows(w.B, w.H, w.Nq, per_head=40, seed=w.index + 50)
+    o_ref, l_ref = oracle.attention(q.cpu(), k.cpu(), v.cpu(), w.softmax_scale, w.causal,
+                                    rows=rows)
+    idx = torch.from_numpy(rows).cuda()
+    compare(o.reshape(-1, w.d)[idx], lse.reshape(-1)[idx], o_ref, l_ref, rel_o=REL_O16[w.dtype])
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_decode_full_size_sampled_heads(out_dtype):
     w = WORKLOADS["decode"]
-    q, k, v, o, lse = _run(w)
+    q, k, v, o, lse = _run(w, out_dtype=out_dtype)
     BH = w.B * w.H
     heads = np.unique(np.concatenate([[0, 1, BH // 2, BH - 1],
                                       np.random.default_rng(5).choice(BH, 20, replace=False)]))
@@ -77,8 +90,9 @@ def test_decode_full_size_sampled_heads():
     ks = k.reshape(BH, 1, w.Nkv, w.d)[sel].reshape(1, -1, w.Nkv, w.d).cpu()
     vs = v.reshape(BH, 1, w.Nkv, w.d)[sel].reshape(1, -1, w.Nkv, w.d).cpu()
     o_ref, l_ref = oracle.attention(qs, ks, vs, w.softmax_scale, False)
+    rel = REL_O16[w.dtype] if out_dtype != torch.float32 else 0.0
     compare(o.reshape(BH, w.d)[sel], lse.reshape(BH)[sel], o_ref.reshape(-1, w.d),
-            l_ref.reshape(-1))
+            l_ref.reshape(-1), rel_o=rel)
     assert torch.isfinite(o).all() and torch.isfinite(lse).all()
 
 
