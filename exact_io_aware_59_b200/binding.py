@@ -39,6 +39,7 @@ _SIGNATURES = {
     "fa_fwd": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I],
     "fa_fwd_prefill": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I, _I],
     "fa_fwd_decode": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
+    "fa_fwd_decode_noalloc": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
     "fa_decode_workspace_bytes": [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
     "fa_device_status": [ctypes.POINTER(_I), _I],
     "fa_selftest_wait_timeout": [_VP],
@@ -95,6 +96,14 @@ def fa_fwd_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtyp
                   num_splits) -> int:
     return library().fa_fwd_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype,
                                    o_dtype, num_splits)
+
+
+def fa_fwd_decode_noalloc(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype,
+                          num_splits) -> int:
+    """fa_fwd_decode with the split partials in the library's fixed static device array
+    instead of a cudaMalloc'd workspace, for callers that cannot allocate device memory."""
+    return library().fa_fwd_decode_noalloc(q, k, v, o, lse, B, H, Nkv, d, scale, stream,
+                                           in_dtype, o_dtype, num_splits)
 
 
 def fa_decode_workspace_bytes(B, H, Nkv, d, num_splits) -> int:

@@ -214,6 +214,17 @@ int run_decode(const void* q, const void* k, const void* v, void* o, float* lse,
 
 }  // namespace
 
+namespace fa {
+int check_decode_call(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int Nkv, int d, float scale, int in_dtype, int o_dtype) {
+  return check_args(q, k, v, o, lse, B, H, 1, Nkv, d, scale, 0, in_dtype, o_dtype);
+}
+DecodeParams plan_decode(int B, int H, int Nkv, float scale, int num_splits, int sm_count) {
+  return decode_params(B, H, Nkv, scale, num_splits, sm_count);
+}
+size_t decode_workspace_bytes(const DecodeParams& p, int d) { return decode_ws_bytes(p, d); }
+}  // namespace fa
+
 extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,

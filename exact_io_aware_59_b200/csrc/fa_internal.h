@@ -45,6 +45,12 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
 // Diagnostic kernel whose only wait can never finish (see fa_selftest_wait_timeout).
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t stream);
 
+// Host-side pieces of the decode entry point, shared with other entry files (fa_api.cu).
+int check_decode_call(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int Nkv, int d, float scale, int in_dtype, int o_dtype);
+DecodeParams plan_decode(int B, int H, int Nkv, float scale, int num_splits, int sm_count);
+size_t decode_workspace_bytes(const DecodeParams& p, int d);
+
 // Bytes of dynamic shared memory each kernel needs.
 size_t prefill_smem_bytes(int d);
 size_t decode_smem_bytes(int d);

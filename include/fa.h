@@ -104,6 +104,38 @@ int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* l
                   int H, int Nkv, int d, float scale, void* stream, int in_dtype, int o_dtype,
                   int num_splits);
 
+/*
+ * fa_fwd_decode_noalloc -- fa_fwd_decode for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment variant, not part of the method.
+ *   Who needs it: fa_fwd_decode allocates its split workspace with cudaMalloc on first
+ *   use, and some callers cannot allow that -- a runtime that has handed all device
+ *   memory to its own pool, a plug-in whose host program forbids device allocations after
+ *   start-up, or latency-critical code that cannot pay for the device synchronisation
+ *   that cudaMalloc / cudaFree imply.
+ *   What it does: the same split-KV decode and combine kernels, same arguments, layouts
+ *   and results as fa_fwd_decode, with the split partials kept in one fixed static device
+ *   array of FA_NOALLOC_SCRATCH_BYTES bytes that every GPU loading this library holds
+ *   until the process exits.  The caller still passes q, k, v, o and lse.  No cudaMalloc,
+ *   cudaFree or other allocating routine is called.
+ *   Limit: a call whose partials need more than the array (G * max_seg * 8 * (d+1) * 4
+ *   bytes plus 256, see fa_decode_workspace_bytes) is refused with FA_ERR_UNSUPPORTED
+ *   before anything is enqueued.  With the default split count (one CTA per SM, 148 on
+ *   B200) that holds for B*H up to about 1,700 heads at d = 128 and 3,800 at d = 64, for
+ *   any Nkv (B=16, H=32, d=128 needs 3.1 MB).
+ *   First call: the first call on each device (made with that device current) checks the
+ *   device and looks up the array's device address; make that first call before any
+ *   stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last call's
+ *   contents.  Nothing in it needs clearing between calls.  Calls whose kernels can
+ *   overlap on the GPU (different streams without ordering between them) race on the
+ *   array.  A kernel wait that runs out is recorded in a status word inside the array,
+ *   which this entry point does not report (use fa_fwd_decode when that is needed).
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (8u << 20)
+int fa_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int Nkv, int d, float scale, void* stream,
+                          int in_dtype, int o_dtype, int num_splits);
+
 /* Bytes of decode workspace a fa_fwd_decode call with these arguments needs. */
 int fa_decode_workspace_bytes(int B, int H, int Nkv, int d, int num_splits, size_t* bytes);
 
