@@ -259,6 +259,63 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes of a row.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of x <= 8 on the FMA pipe, to take load off the SFU.  Round-to-nearest
+// argument reduction x = j + f, |f| <= 1/2, with the 1.5 * 2^23 addition trick (the sum's
+// low mantissa bits hold j); 2^f from a degree-3 polynomial whose coefficients minimise the
+// maximum relative error on [-1/2, 1/2] (computed by linear programming over a dense grid,
+// see exp2_poly.py; max relative error 7.5e-5); j is added to the exponent field with an
+// integer multiply-add.  x is clamped at -125 so the result stays a normal number.
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+__device__ __forceinline__ uint64_t exp2_poly_pair(float x0, float x1) {
+  const float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
+  const uint64_t j = f2_add(t, f2_pack(-kMagic, -kMagic));
+  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), xc);
+  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  const uint32_t r0 = __float_as_uint(t0) * (1u << 23) + __float_as_uint(p0);
+  const uint32_t r1 = __float_as_uint(t1) * (1u << 23) + __float_as_uint(p1);
+  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
+}
+
 // Two fp32 values rounded to nearest-even into one packed 16-bit pair, `lo` in the low
 // half.
 template <bool BF16>
@@ -270,6 +327,21 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   }
   return r;
+}
+
+// acc + lo + hi for a packed 16-bit pair, with mixed-precision adds (no unpacking).
+template <bool BF16>
+__device__ __forceinline__ float add_pair16(float acc, uint32_t pk) {
+  if constexpr (BF16) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %0, hi, %0;\n\t}"
+        : "+f"(acc) : "r"(pk));
+  } else {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+        "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %0, hi, %0;\n\t}"
+        : "+f"(acc) : "r"(pk));
+  }
+  return acc;
 }
 
 // Unpacks a 16-bit pair (low half first) to fp32.

@@ -149,27 +149,30 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
 }
 
 // ---------------------------------------------------------------- MMA issuer
+// Shared-memory descriptors are built once per buffer; an MMA step's operand is the
+// buffer's descriptor plus (byte offset >> 4) in the start-address field (shared-memory
+// addresses are below 2^18, so the 14-bit field never carries).
 template <int D>
-__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint32_t qa, uint32_t ka, uint32_t idesc) {
+__device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc,
+                                        uint32_t idesc) {
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     // K-major operand, 128-byte swizzle: 64-element column blocks of 128 rows x 128 B,
     // 16 elements (32 B) per MMA step; 8-row groups 1024 B apart.
-    const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-    mma_ss(d_tmem, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
-           idesc, kk > 0 ? 1u : 0u);
+    const uint32_t off16 = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+    mma_ss(d_tmem, q_desc + off16, k_desc + off16, idesc, kk > 0 ? 1u : 0u);
   }
 }
 
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t va,
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
                                          uint32_t idesc, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
     // V is MN-major (d contiguous): 16 keys per step = two 1024-byte swizzle atoms;
-    // the second 64-column block of d lies BN*128 bytes further.
-    const uint64_t b = make_sdesc_sw128(va + kk * 16 * 128, BN * 128, 1024);
-    mma_ts(d_tmem, p_tmem + kk * 8, b, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    // the second 64-column block of d lies BN*128 bytes further (the descriptor's LBO).
+    mma_ts(d_tmem, p_tmem + kk * 8, v_desc + ((kk * 16 * 128) >> 4), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -182,6 +185,12 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
   constexpr uint32_t idesc_o = make_idesc_f16(BM, D, BF16, true);
   uint32_t ld = 0, q_used = 0, pcount[2] = {0, 0};
   bool ok = true;
+  const uint64_t q_desc0 = make_sdesc_sw128(sbase + C::kQOff, 16, 1024);
+  const uint64_t kv_desc0 = make_sdesc_sw128(sbase + C::kRingOff, 16, 1024);
+  const uint64_t v_desc0 = make_sdesc_sw128(sbase + C::kRingOff, BN * 128, 1024);
+  auto q_desc = [&](int t) { return q_desc0 + ((t * C::kQBytes) >> 4); };
+  auto k_desc = [&](uint32_t slot) { return kv_desc0 + ((slot * C::kKVBytes) >> 4); };
+  auto v_desc = [&](uint32_t slot) { return v_desc0 + ((slot * C::kKVBytes) >> 4); };
   auto wait = [&](int b, uint32_t parity) {
     return mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutMma);
   };
@@ -201,8 +210,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       if (n[t] == 0) continue;
-      issue_s<D>(tmem + t * 128, sbase + C::kQOff + t * C::kQBytes,
-                 sbase + C::kRingOff + kslot0 * C::kKVBytes, idesc_s);
+      issue_s<D>(tmem + t * 128, q_desc(t), k_desc(kslot0), idesc_s);
       tc_commit(bar_addr(bars, C::kBarSFull + t));
     }
     tc_commit(bar_addr(bars, C::kBarEmpty + kslot0));
@@ -218,8 +226,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
         if (!wait(C::kBarPFull + t, pcount[t] & 1)) { ok = false; break; }
         ++pcount[t];
         tc_fence_after();
-        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, sbase + C::kRingOff + vslot * C::kKVBytes,
-                    idesc_o, j > 0);
+        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, j > 0);
         tc_commit(bar_addr(bars, C::kBarODone + t));
         if (j + 1 < n[t]) {
           if (knext < 0) {
@@ -228,8 +235,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
             tc_fence_after();
             ++ld;
           }
-          issue_s<D>(tmem + t * 128, sbase + C::kQOff + t * C::kQBytes,
-                     sbase + C::kRingOff + knext * C::kKVBytes, idesc_s);
+          issue_s<D>(tmem + t * 128, q_desc(t), k_desc(knext), idesc_s);
           tc_commit(bar_addr(bars, C::kBarSFull + t));
         }
       }
@@ -247,6 +253,75 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
+// Max (or min) of a row's 128 raw scores: eight independent chains of 3-input max.
+template <bool MAX>
+__device__ __forceinline__ float row_reduce(const uint32_t (&s)[4][32]) {
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] = __uint_as_float(s[k >> 1][(k & 1) * 16]);
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+#pragma unroll
+    for (int i = 1; i < 16; i += 2) {
+      const float a = __uint_as_float(s[k >> 1][(k & 1) * 16 + i]);
+      const float b = (i + 1 < 16) ? __uint_as_float(s[k >> 1][(k & 1) * 16 + i + 1]) : a;
+      acc[k] = MAX ? max3(acc[k], a, b) : min3(acc[k], a, b);
+    }
+  const float x = MAX ? max3(acc[0], acc[1], acc[2]) : min3(acc[0], acc[1], acc[2]);
+  const float y = MAX ? max3(acc[3], acc[4], acc[5]) : min3(acc[3], acc[4], acc[5]);
+  return MAX ? max3(x, y, fmaxf(acc[6], acc[7])) : min3(x, y, fminf(acc[6], acc[7]));
+}
+
+// p = 2^(s * scale_log2 - m) for a row's 128 scores, rounded in pairs to the 16-bit type
+// and written over the first 64 TMEM columns of S; returns the row sums of the rounded
+// and of the unrounded p.  FULL: every column visible; one pair in four takes the
+// FMA-pipe exp2, the rest the SFU.  !FULL: columns past lim_c get p = 0 (all on the SFU).
+template <bool BF16, bool FULL>
+__device__ __forceinline__ void exp_pack_store(const uint32_t (&s)[4][32], float scale_log2,
+                                               float m, int lim_c, uint32_t tS, float& sum_r,
+                                               float& sum_e) {
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  float acc_r[4] = {0.f, 0.f, 0.f, 0.f};
+  uint64_t acc_e[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) acc_e[k] = 0ull;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])),
+                                 sc2, nm2);
+      float x0, x1, p0, p1;
+      f2_unpack(x2, x0, x1);
+      if (FULL && (i & 3) == 1) {
+        f2_unpack(exp2_poly_pair(x0, x1), p0, p1);
+      } else {
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
+      if (!FULL) {
+        p0 = (c * 32 + 2 * i <= lim_c) ? p0 : 0.f;
+        p1 = (c * 32 + 2 * i + 1 <= lim_c) ? p1 : 0.f;
+      }
+      pk[i] = pack2<BF16>(p0, p1);
+      // O is divided by the sum of the same rounded P that the P V product uses, so a
+      // row dominated by one key normalises exactly; LSE uses the unrounded sum.
+      acc_r[i & 3] = add_pair16<BF16>(acc_r[i & 3], pk[i]);
+      acc_e[i & 3] = f2_add(acc_e[i & 3], f2_pack(p0, p1));
+    }
+    // P (16-bit, two per column) overwrites the first 64 columns of S.
+    tmem_st_32x32b_x16(tS + c * 16, pk);
+  }
+  sum_r = (acc_r[0] + acc_r[1]) + (acc_r[2] + acc_r[3]);
+  const uint64_t e2 = f2_add(f2_add(acc_e[0], acc_e[1]), f2_add(acc_e[2], acc_e[3]));
+  float a, b;
+  f2_unpack(e2, a, b);
+  sum_e = a + b;
+}
+
+
 template <int D, bool BF16, bool OF32>
 __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t tmem, void* o,
                                  float* lse, int t, int* status, volatile int* abort_flag) {
@@ -258,6 +333,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   const uint32_t tS = lane_base + t * 128;
   const uint32_t tO = lane_base + 256 + t * D;
   const float scale_log2 = p.scale_log2;
+  const bool neg_scale = scale_log2 < 0.f;
   uint32_t s_seen = 0, o_seen = 0;
   // Warp-uniform result: tcgen05.ld/st below are warp-collective, so a warp never splits
   // on a wait that finished on some lanes and ran out on others.
@@ -290,29 +366,21 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence(s[c]);
 
-      // x = s * scale * log2(e); masked entries -inf.
-      const int lim_c = limit - j * BN;
-      float mx = -INFINITY;
-      if (lim_c >= BN - 1) {
+      // Row max of x = s * scale * log2(e) over the visible columns, taken on the raw
+      // scores (their min when the scale is negative) and scaled once.
+      const int lim_c = limit - j * BN;  // columns c <= lim_c are visible for this row
+      const bool full = __all_sync(0xffffffffu, lim_c >= BN - 1);  // warp-uniform path
+      if (!full) {
+        const float sentinel = neg_scale ? INFINITY : -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = __uint_as_float(s[c][i]) * scale_log2;
-            s[c][i] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
-          }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float x = (c * 32 + i <= lim_c) ? __uint_as_float(s[c][i]) * scale_log2 : -INFINITY;
-            s[c][i] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
-          }
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i > lim_c) s[c][i] = __float_as_uint(sentinel);
       }
-      const float m_new = fmaxf(m_used, mx);
+      const float mr = neg_scale ? row_reduce<false>(s) : row_reduce<true>(s);
+      const float m_tile = (mr == INFINITY || mr == -INFINITY) ? -INFINITY : mr * scale_log2;
+      const float m_new = fmaxf(m_used, m_tile);
       // Lazy rescale: move the reference max only when it grows by more than 8 (log2),
       // so p = 2^(x - m_used) stays <= 256.  -inf -> finite always moves; -inf -> -inf
       // gives NaN and never moves.
@@ -339,30 +407,17 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
         m_used = m_new;
       }
       const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f, rs_exact = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(__uint_as_float(s[c][2 * i]) - m_eff);
-          const float p1 = ex2(__uint_as_float(s[c][2 * i + 1]) - m_eff);
-          pk[i] = pack2<BF16>(p0, p1);
-          // O is divided by the sum of the same rounded P that the P V product uses, so
-          // a row dominated by one key normalises exactly; LSE uses the unrounded sum.
-          float r0, r1;
-          unpack2<BF16>(pk[i], r0, r1);
-          rs += r0 + r1;
-          rs_exact += p0 + p1;
-        }
-        // P (16-bit, two per column) overwrites the first 64 columns of S.
-        tmem_st_32x32b_x16(tS + c * 16, pk);
-      }
+      float rs, rs_exact;
+      if (full)
+        exp_pack_store<BF16, true>(s, scale_log2, m_eff, lim_c, tS, rs, rs_exact);
+      else
+        exp_pack_store<BF16, false>(s, scale_log2, m_eff, lim_c, tS, rs, rs_exact);
       l += rs;
       l_exact += rs_exact;
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar_addr(bars, C::kBarPFull + t));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarPFull + t));  // one arrival per warp
     }
 
     // Epilogue: O = O_t / l and LSE = (m + log2 l) * ln 2.
@@ -435,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_addr(bars, C::kBarSFull + t), 1);
-      mbar_init(bar_addr(bars, C::kBarPFull + t), 128);
+      mbar_init(bar_addr(bars, C::kBarPFull + t), 4);  // one arrival per softmax warp
       mbar_init(bar_addr(bars, C::kBarODone + t), 1);
     }
     mbar_init(bar_addr(bars, C::kBarDrain), 1);
