@@ -56,14 +56,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Slow path of a bounded wait: spins until the phase with `parity` completes, the CTA's
-// abort flag is raised by another thread, or kWaitLimitNs passes.  On a timeout it
-// records `code` in the global status word and raises the abort flag.
+// try_wait that may suspend the thread (no instruction issue) for up to `hint_ns` while
+// the phase is incomplete; it returns as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Slow path of a bounded wait: sleeps in try_wait (so a waiting warp takes no issue slots
+// from the warps doing work) until the phase with `parity` completes, the CTA's abort flag
+// is raised by another thread, or kWaitLimitNs passes.  On a timeout it records `code` in
+// the global status word and raises the abort flag.
 __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, int* status,
                                             volatile int* abort_flag, int code) {
   const uint64_t t0 = global_timer_ns();
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       atomicOr(status, code);
@@ -291,21 +306,24 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
 
 // 2^x for a pair of x <= 8 on the FMA pipe, to take load off the SFU.  Round-to-nearest
 // argument reduction x = j + f, |f| <= 1/2, with the 1.5 * 2^23 addition trick (the sum's
-// low mantissa bits hold j); 2^f from a degree-3 polynomial whose coefficients minimise the
+// low mantissa bits hold j); 2^f from a degree-4 polynomial whose coefficients minimise the
 // maximum relative error on [-1/2, 1/2] (computed by linear programming over a dense grid,
-// see exp2_poly.py; max relative error 7.5e-5); j is added to the exponent field with an
-// integer multiply-add.  x is clamped at -125 so the result stays a normal number.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716685295105f;
+// see exp2_poly.py; max relative error 2.7e-6 in fp32, far below the 2^-9 of the bf16
+// rounding that follows); j is added to the exponent field with an integer multiply-add.
+// x is clamped at -125 so the result stays a normal number.
+constexpr float kExp2C0 = 0.9999992251396179f;
+constexpr float kExp2C1 = 0.6931217312812805f;
+constexpr float kExp2C2 = 0.24024765193462372f;
+constexpr float kExp2C3 = 0.05591819807887077f;
+constexpr float kExp2C4 = 0.009569705463945866f;
 __device__ __forceinline__ uint64_t exp2_poly_pair(float x0, float x1) {
   const float kMagic = 12582912.0f;  // 1.5 * 2^23
   const uint64_t xc = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
   const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
   const uint64_t j = f2_add(t, f2_pack(-kMagic, -kMagic));
   const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), xc);
-  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  uint64_t p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
+  p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
   p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
   p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
   float p0, p1, t0, t1;

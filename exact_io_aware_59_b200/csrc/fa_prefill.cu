@@ -72,6 +72,16 @@ __device__ __forceinline__ void unit_coords(const PrefillParams& p, int u, int& 
   bh = u % p.BH;
 }
 
+// The unit a CTA takes in round r of the persistent loop.  Units are numbered heaviest
+// first; rounds deal them out in alternating directions ("snake"), so a CTA that got a heavy
+// unit in one round gets a light one in the next.  For causal prefill this keeps the
+// busiest SM within about 2% of the mean (plain round robin: about 14%).  Every role of the
+// CTA walks the same sequence.
+__device__ __forceinline__ int unit_of_round(int r) {
+  const int G = gridDim.x, c = blockIdx.x;
+  return r * G + ((r & 1) ? (G - 1 - c) : c);
+}
+
 // Number of K/V tiles Q tile `qtile` must visit (0 when every row is fully masked).
 __device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, int qtile) {
   if (qtile >= p.n_qtiles) return 0;
@@ -99,7 +109,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
   constexpr int S = C::kStages;
   uint32_t ld = 0, q_issued = 0;
   bool ok = true;
-  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+  for (int rnd = 0, u = unit_of_round(0); u < p.n_units && ok; u = unit_of_round(++rnd)) {
     int bh, pair;
     unit_coords(p, u, bh, pair);
     const int n0 = kv_tiles_for(p, 2 * pair), n1 = kv_tiles_for(p, 2 * pair + 1);
@@ -194,7 +204,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
   auto wait = [&](int b, uint32_t parity) {
     return mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutMma);
   };
-  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+  for (int rnd = 0, u = unit_of_round(0); u < p.n_units && ok; u = unit_of_round(++rnd)) {
     int bh, pair;
     unit_coords(p, u, bh, pair);
     const int n[2] = {kv_tiles_for(p, 2 * pair), kv_tiles_for(p, 2 * pair + 1)};
@@ -342,7 +352,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     return __all_sync(0xffffffffu, ok);
   };
 
-  for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+  for (int rnd = 0, u = unit_of_round(0); u < p.n_units; u = unit_of_round(++rnd)) {
     int bh, pair;
     unit_coords(p, u, bh, pair);
     const int qtile = 2 * pair + t;
