@@ -386,7 +386,7 @@ def arm_ours(args, ws, rank, local):
 
 
 # Bumped whenever the prefill kernel changes, so stale ncu traffic is not reported.
-KERNEL_REV = "prefill-v1"
+KERNEL_REV = "prefill-v9"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the
 # kernel at this revision (profiles/fa_prefill_sm100_<workload>.md).
 DRAM_TRAFFIC = {("prefill-v1", "long_prefill_causal"): 629.5e6}

@@ -233,7 +233,8 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (j >= n[t]) continue;
-        if (!wait(C::kBarPFull + t, pcount[t] & 1)) { ok = false; break; }
+        if (!mbar_wait_spin(bar_addr(bars, C::kBarPFull + t), pcount[t] & 1, status, abort_flag,
+                            kStatusTimeoutMma)) { ok = false; break; }
         ++pcount[t];
         tc_fence_after();
         issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, j > 0);
@@ -282,57 +283,38 @@ __device__ __forceinline__ float row_reduce(const uint32_t (&s)[4][32]) {
   return MAX ? max3(x, y, fmaxf(acc[6], acc[7])) : min3(x, y, fminf(acc[6], acc[7]));
 }
 
-// p = 2^(s * scale_log2 - m) for a row's 128 scores, rounded in pairs to the 16-bit type
-// and written over the first 64 TMEM columns of S; returns the row sums of the rounded
-// and of the unrounded p.  FULL: every column visible; one pair in four takes the
-// FMA-pipe exp2, the rest the SFU.  !FULL: columns past lim_c get p = 0 (all on the SFU).
+// p = 2^(s * scale_log2 - m) for 32 scores (tile columns col0 .. col0+31), rounded in
+// pairs to the 16-bit type and stored to 16 TMEM columns at tP (two values per column);
+// adds the unrounded p to the running sums.  FULL: every column visible; one pair in four
+// takes the FMA-pipe exp2, the rest the SFU.  !FULL: columns past lim_c get p = 0.
 template <bool BF16, bool FULL>
-__device__ __forceinline__ void exp_pack_store(const uint32_t (&s)[4][32], float scale_log2,
-                                               float m, int lim_c, uint32_t tS, float& sum_r,
-                                               float& sum_e) {
-  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
-  const uint64_t nm2 = f2_pack(-m, -m);
-  float acc_r[4] = {0.f, 0.f, 0.f, 0.f};
-  uint64_t acc_e[4];
+__device__ __forceinline__ void exp_pack_store32(const uint32_t (&s)[32], uint64_t sc2, uint64_t nm2,
+                                                 int col0, int lim_c, uint32_t tP,
+                                                 uint64_t (&acc)[4]) {
+  uint32_t pk[16];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) acc_e[k] = 0ull;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[c][2 * i]), __uint_as_float(s[c][2 * i + 1])),
-                                 sc2, nm2);
-      float x0, x1, p0, p1;
-      f2_unpack(x2, x0, x1);
-      if (FULL && (i & 3) == 1) {
-        f2_unpack(exp2_poly_pair(x0, x1), p0, p1);
-      } else {
-        p0 = ex2(x0);
-        p1 = ex2(x1);
-      }
-      if (!FULL) {
-        p0 = (c * 32 + 2 * i <= lim_c) ? p0 : 0.f;
-        p1 = (c * 32 + 2 * i + 1 <= lim_c) ? p1 : 0.f;
-      }
-      pk[i] = pack2<BF16>(p0, p1);
-      // O is divided by the sum of the same rounded P that the P V product uses, so a
-      // row dominated by one key normalises exactly; LSE uses the unrounded sum.
-      acc_r[i & 3] = add_pair16<BF16>(acc_r[i & 3], pk[i]);
-      acc_e[i & 3] = f2_add(acc_e[i & 3], f2_pack(p0, p1));
+  for (int i = 0; i < 16; ++i) {
+    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2);
+    float x0, x1, p0, p1;
+    f2_unpack(x2, x0, x1);
+    if (FULL && (i & 3) == 1) {
+      f2_unpack(exp2_poly_pair(x0, x1), p0, p1);
+    } else {
+      p0 = ex2(x0);
+      p1 = ex2(x1);
     }
-    // P (16-bit, two per column) overwrites the first 64 columns of S.
-    tmem_st_32x32b_x16(tS + c * 16, pk);
+    if (!FULL) {
+      p0 = (col0 + 2 * i <= lim_c) ? p0 : 0.f;
+      p1 = (col0 + 2 * i + 1 <= lim_c) ? p1 : 0.f;
+    }
+    pk[i] = pack2<BF16>(p0, p1);
+    acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
   }
-  sum_r = (acc_r[0] + acc_r[1]) + (acc_r[2] + acc_r[3]);
-  const uint64_t e2 = f2_add(f2_add(acc_e[0], acc_e[1]), f2_add(acc_e[2], acc_e[3]));
-  float a, b;
-  f2_unpack(e2, a, b);
-  sum_e = a + b;
+  tmem_st_32x32b_x16(tP, pk);
 }
 
-
-template <int D, bool BF16, bool OF32>
+// NEG: the scale is negative, so the row maximum of scale * s comes from the minimum of s.
+template <int D, bool BF16, bool OF32, bool NEG>
 __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t tmem, void* o,
                                  float* lse, int t, int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -343,7 +325,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   const uint32_t tS = lane_base + t * 128;
   const uint32_t tO = lane_base + 256 + t * D;
   const float scale_log2 = p.scale_log2;
-  const bool neg_scale = scale_log2 < 0.f;
+  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
   uint32_t s_seen = 0, o_seen = 0;
   // Warp-uniform result: tcgen05.ld/st below are warp-collective, so a warp never splits
   // on a wait that finished on some lanes and ran out on others.
@@ -381,14 +363,14 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
       const int lim_c = limit - j * BN;  // columns c <= lim_c are visible for this row
       const bool full = __all_sync(0xffffffffu, lim_c >= BN - 1);  // warp-uniform path
       if (!full) {
-        const float sentinel = neg_scale ? INFINITY : -INFINITY;
+        const float sentinel = NEG ? INFINITY : -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i > lim_c) s[c][i] = __float_as_uint(sentinel);
       }
-      const float mr = neg_scale ? row_reduce<false>(s) : row_reduce<true>(s);
+      const float mr = row_reduce<!NEG>(s);
       const float m_tile = (mr == INFINITY || mr == -INFINITY) ? -INFINITY : mr * scale_log2;
       const float m_new = fmaxf(m_used, m_tile);
       // Lazy rescale: move the reference max only when it grows by more than 8 (log2),
@@ -417,11 +399,33 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
         m_used = m_new;
       }
       const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs, rs_exact;
-      if (full)
-        exp_pack_store<BF16, true>(s, scale_log2, m_eff, lim_c, tS, rs, rs_exact);
-      else
-        exp_pack_store<BF16, false>(s, scale_log2, m_eff, lim_c, tS, rs, rs_exact);
+      // P (16-bit, two per column) overwrites the first 64 S columns, 16 per 32 scores.
+      const uint64_t nm2 = f2_pack(-m_eff, -m_eff);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (full)
+          exp_pack_store32<BF16, true>(s[c], sc2, nm2, 32 * c, lim_c, tS + 16 * c, acc);
+        else
+          exp_pack_store32<BF16, false>(s[c], sc2, nm2, 32 * c, lim_c, tS + 16 * c, acc);
+      }
+      float rs_exact;
+      {
+        float a, b2;
+        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a, b2);
+        rs_exact = a + b2;
+      }
+      // O is divided by the row sum of the rounded P that the P V product uses, taken as the
+      // unrounded sum plus the rounding error of each tile's largest P.  That one term
+      // dominates when a row's weight sits on a few keys; the other terms' errors (relative
+      // 2^-9 for bf16, 2^-12 for fp16, either sign) average out over many comparable keys.
+      float rs = rs_exact;
+      if (m_tile != -INFINITY) {
+        const float pmax = ex2(fmaf(mr, scale_log2, -m_eff));
+        float r0, r1;
+        unpack2<BF16>(pack2<BF16>(pmax, 0.f), r0, r1);
+        rs += r0 - pmax;
+      }
       l += rs;
       l_exact += rs_exact;
       tmem_st_wait();
@@ -539,7 +543,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    softmax_epilogue<D, BF16, OF32>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+    if (p.scale_log2 < 0.f)
+      softmax_epilogue<D, BF16, OF32, true>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+    else
+      softmax_epilogue<D, BF16, OF32, false>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     tc_fence_before();
     mbar_arrive(bar_addr(bars, C::kBarDone));
   }
