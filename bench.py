@@ -153,11 +153,19 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """The largest of the ranks' x (a step time): NCCL on the GPUs, gloo on the host."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, ms_max: float, ws: int) -> float:
+    """Units all ranks processed per second: every rank runs the same independent
+    problem, and the job takes as long as its slowest rank."""
+    return units_per_rank * ws / (ms_max * 1e-3)
 
 
 def time_steps(fn, steps: int, warmup: int, ws: int, stream) -> float:
@@ -321,7 +329,7 @@ def arm_ours(args, ws, rank, local):
     assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
     flops = attention_flops(wp)
     tflops = flops / (ms_p * 1e-3) / 1e12
-    value = tflops * ws
+    value = whole_job_rate(flops, ms_p, ws) / 1e12
     peak_t = peaks["bf16_tflops"]
     traffic = DRAM_TRAFFIC.get((KERNEL_REV, wp.name))
 
@@ -337,7 +345,8 @@ def arm_ours(args, ws, rank, local):
         bytes_d = algorithmic_bytes(wd, 2)
         gbs = bytes_d / (ms_d * 1e-3) / 1e9
         decode = {
-            "workload": workload_config(wd, "bf16")["workload"], "value": gbs * ws,
+            "workload": workload_config(wd, "bf16")["workload"],
+            "value": whole_job_rate(bytes_d, ms_d, ws) / 1e9,
             "unit": "GB/s", "ms_per_step": ms_d, "steps": dsteps,
             "gpu_launches": 2 * dsteps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
@@ -352,8 +361,8 @@ def arm_ours(args, ws, rank, local):
     e2e = None
     if not args.skip_e2e:
         esteps = max(3, min(args.steps, 20))
-        ms_e, h2d, d2h = run_e2e(wp, tensors, esteps, 2, ws, stream)
-        e2e = {"value": flops / (ms_e * 1e-3) / 1e12 * ws, "unit": "TFLOP/s",
+        ms_e, h2d, d2h = run_e2e(wp, tensors, esteps, 3, ws, stream)
+        e2e = {"value": whole_job_rate(flops, ms_e, ws) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e,
                "steps": esteps}
     del tensors

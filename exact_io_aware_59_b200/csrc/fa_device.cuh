@@ -338,7 +338,7 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of x <= 8 on the FMA pipe, to take load off the SFU.  Round-to-nearest
+// 2^x for a pair of x < 127 on the FMA pipe, to take load off the SFU.  Round-to-nearest
 // argument reduction x = j + f, |f| <= 1/2, with the 1.5 * 2^23 addition trick (the sum's
 // low mantissa bits hold j); 2^f from a degree-4 polynomial whose coefficients minimise the
 // maximum relative error on [-1/2, 1/2] (computed by linear programming over a dense grid,

@@ -18,7 +18,7 @@
 //    tile's softmax overlaps the other tile's matrix products;
 //  * warpgroups 1 and 2 run the softmax of tile 0 and tile 1, one thread per row: they
 //    read S from TMEM, apply scale and mask, update (m, l), write P as 16-bit into the
-//    S columns, rescale O in TMEM only when the max grows by more than 2^8 (lazy), and
+//    S columns, rescale O in TMEM only when the max grows by more than kLazyLog2 (lazy), and
 //    run the epilogue (O / l and LSE to global memory).
 //  TMEM map (512 columns): S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+d), O1 after it.
 #include <cuda_bf16.h>
@@ -37,6 +37,11 @@ constexpr int kRegsLaunch = 168;   // 65536 / 384, rounded down to a multiple of
 constexpr int kRegsSide = 88;      // warpgroup 0 (load + MMA issue)
 constexpr int kRegsSoftmax = 208;  // warpgroups 1 and 2; 128*88 + 256*208 == 384*168
 static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+// Lazy rescale threshold in log2 units: the reference max m_used of a row moves only when
+// a tile's max exceeds it by more than this, so p = 2^(x - m_used) <= 2^15, below the fp16
+// maximum 65504 (bf16 and the fp32 O and l have far more range).  O and l share m_used,
+// so the result is the same softmax whatever the lag.
+constexpr float kLazyLog2 = 15.0f;
 
 template <int D>
 struct PrefillCfg {
@@ -284,19 +289,20 @@ __device__ __forceinline__ float row_reduce(const uint32_t (&s)[4][32]) {
 }
 
 // p = 2^(s * scale_log2 - m) for 32 scores (tile columns col0 .. col0+31), rounded in
-// pairs to the 16-bit type and stored to 16 TMEM columns at tP (two values per column);
-// adds the unrounded p to the running sums.  FULL: every column visible; one pair in four
+// pairs to the 16-bit type into pk (exp_pack_store32 also stores them to 16 TMEM columns
+// at tP, two values per column); adds the unrounded p to the running sums, and with XMAX
+// folds the exponents x = s * scale_log2 - m into two running maxima.  FULL: every column visible; one pair in four
 // takes the FMA-pipe exp2, the rest the SFU.  !FULL: columns past lim_c get p = 0.
-template <bool BF16, bool FULL>
-__device__ __forceinline__ void exp_pack_store32(const uint32_t (&s)[32], uint64_t sc2, uint64_t nm2,
-                                                 int col0, int lim_c, uint32_t tP,
-                                                 uint64_t (&acc)[4]) {
-  uint32_t pk[16];
+template <bool BF16, bool FULL, bool XMAX = false>
+__device__ __forceinline__ void exp_pack32(const uint32_t (&s)[32], uint64_t sc2, uint64_t nm2,
+                                           int col0, int lim_c, uint32_t (&pk)[16],
+                                           uint64_t (&acc)[4], float (&xmax)[2]) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1])), sc2, nm2);
     float x0, x1, p0, p1;
     f2_unpack(x2, x0, x1);
+    if (XMAX) xmax[i & 1] = max3(xmax[i & 1], x0, x1);
     if (FULL && (i & 3) == 1) {
       f2_unpack(exp2_poly_pair(x0, x1), p0, p1);
     } else {
@@ -310,6 +316,15 @@ __device__ __forceinline__ void exp_pack_store32(const uint32_t (&s)[32], uint64
     pk[i] = pack2<BF16>(p0, p1);
     acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
   }
+}
+
+template <bool BF16, bool FULL>
+__device__ __forceinline__ void exp_pack_store32(const uint32_t (&s)[32], uint64_t sc2, uint64_t nm2,
+                                                 int col0, int lim_c, uint32_t tP,
+                                                 uint64_t (&acc)[4]) {
+  uint32_t pk[16];
+  float unused[2];
+  exp_pack32<BF16, FULL>(s, sc2, nm2, col0, lim_c, pk, acc, unused);
   tmem_st_32x32b_x16(tP, pk);
 }
 
@@ -351,77 +366,109 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
       if (!wait(C::kBarSFull + t, s_seen & 1)) return;
       ++s_seen;
       tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
-      tmem_ld_wait_only();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(s[c]);
-
-      // Row max of x = s * scale * log2(e) over the visible columns, taken on the raw
-      // scores (their min when the scale is negative) and scaled once.
       const int lim_c = limit - j * BN;  // columns c <= lim_c are visible for this row
       const bool full = __all_sync(0xffffffffu, lim_c >= BN - 1);  // warp-uniform path
-      if (!full) {
-        const float sentinel = NEG ? INFINITY : -INFINITY;
+      // p = 2^(x - m_eff) for the row, stored as P over the first 64 S columns (16-bit,
+      // two per column, 16 columns per 32 scores); returns the sum of the unrounded p.
+      auto exp_pass = [&](const uint32_t (&s)[4][32], float m_eff, bool all_visible) {
+        const uint64_t nm2 = f2_pack(-m_eff, -m_eff);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 4; ++c) {
+          if (all_visible)
+            exp_pack_store32<BF16, true>(s[c], sc2, nm2, 32 * c, lim_c, tS + 16 * c, acc);
+          else
+            exp_pack_store32<BF16, false>(s[c], sc2, nm2, 32 * c, lim_c, tS + 16 * c, acc);
+        }
+        float a0, a1;
+        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+        return a0 + a1;
+      };
+      // Row max of x = s * scale * log2(e) over the visible columns, taken on the raw
+      // scores (their min when the scale is negative) and scaled once.
+      float xm, rs_exact;  // xm: largest x - m_eff of the row's visible scores (-inf if none)
+      bool done = false;
+      if (full && __all_sync(0xffffffffu, m_used != -INFINITY)) {
+        // Once a row has a finite reference max, a tile with every column visible rarely
+        // moves it: exponentiate against it straight away, taking the row max of the
+        // exponents in the same pass, so the reduction is off the path to P.  P stays in
+        // registers until the max is known; if it moved by more than kLazyLog2 anywhere in the
+        // warp, the tile is redone below from S, still intact in TMEM.
+        uint32_t s[4][32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i > lim_c) s[c][i] = __float_as_uint(sentinel);
-      }
-      const float mr = row_reduce<!NEG>(s);
-      const float m_tile = (mr == INFINITY || mr == -INFINITY) ? -INFINITY : mr * scale_log2;
-      const float m_new = fmaxf(m_used, m_tile);
-      // Lazy rescale: move the reference max only when it grows by more than 8 (log2),
-      // so p = 2^(x - m_used) stays <= 256.  -inf -> finite always moves; -inf -> -inf
-      // gives NaN and never moves.
-      const bool move = (m_new - m_used) > 8.0f;
-      if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // O_t still holds P V of tiles < j: wait for the last of those products.
-        if (!wait(C::kBarODone + t, (o_seen + j - 1) & 1)) return;
-        tc_fence_after();
-        const float alpha = move ? ex2(m_used - m_new) : 1.0f;
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t ob[32];
-          tmem_ld_32x32b_x32(tO + cc * 32, ob);
-          tmem_ld_wait(ob);
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
+        tmem_ld_wait_only();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
-          tmem_st_32x32b_x32(tO + cc * 32, ob);
+        for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+        const uint64_t nm2 = f2_pack(-m_used, -m_used);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pk[4][16];
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) exp_pack32<BF16, true, true>(s[c], sc2, nm2, 32 * c, lim_c, pk[c], acc, mx);
+        xm = fmaxf(mx[0], mx[1]);
+        done = !__any_sync(0xffffffffu, xm > kLazyLog2);
+        if (done) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_st_32x32b_x16(tS + 16 * c, pk[c]);
+          float a0, a1;
+          f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+          rs_exact = a0 + a1;
         }
       }
-      if (move) {
-        const float a = ex2(m_used - m_new);
-        l *= a;
-        l_exact *= a;
-        m_used = m_new;
-      }
-      const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-      // P (16-bit, two per column) overwrites the first 64 S columns, 16 per 32 scores.
-      const uint64_t nm2 = f2_pack(-m_eff, -m_eff);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      if (!done) {
+        uint32_t s[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (full)
-          exp_pack_store32<BF16, true>(s[c], sc2, nm2, 32 * c, lim_c, tS + 16 * c, acc);
-        else
-          exp_pack_store32<BF16, false>(s[c], sc2, nm2, 32 * c, lim_c, tS + 16 * c, acc);
-      }
-      float rs_exact;
-      {
-        float a, b2;
-        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a, b2);
-        rs_exact = a + b2;
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
+        tmem_ld_wait_only();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+        if (!full) {
+          const float sentinel = NEG ? INFINITY : -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i > lim_c) s[c][i] = __float_as_uint(sentinel);
+        }
+        const float mr = row_reduce<!NEG>(s);
+        const float m_tile = (mr == INFINITY || mr == -INFINITY) ? -INFINITY : mr * scale_log2;
+        const float m_new = fmaxf(m_used, m_tile);
+        // Lazy rescale: move the reference max only when it grows by more than kLazyLog2.
+        // -inf -> finite always moves; -inf -> -inf gives NaN and never moves.
+        const bool move = (m_new - m_used) > kLazyLog2;
+        if (j > 0 && __any_sync(0xffffffffu, move)) {
+          // O_t still holds P V of tiles < j: wait for the last of those products.
+          if (!wait(C::kBarODone + t, (o_seen + j - 1) & 1)) return;
+          tc_fence_after();
+          const float alpha = move ? ex2(m_used - m_new) : 1.0f;
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t ob[32];
+            tmem_ld_32x32b_x32(tO + cc * 32, ob);
+            tmem_ld_wait(ob);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
+            tmem_st_32x32b_x32(tO + cc * 32, ob);
+          }
+        }
+        if (move) {
+          const float a = ex2(m_used - m_new);
+          l *= a;
+          l_exact *= a;
+          m_used = m_new;
+        }
+        const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+        rs_exact = exp_pass(s, m_eff, full);
+        xm = (m_tile == -INFINITY) ? -INFINITY : fmaf(mr, scale_log2, -m_eff);
       }
       // O is divided by the row sum of the rounded P that the P V product uses, taken as the
       // unrounded sum plus the rounding error of each tile's largest P.  That one term
       // dominates when a row's weight sits on a few keys; the other terms' errors (relative
       // 2^-9 for bf16, 2^-12 for fp16, either sign) average out over many comparable keys.
       float rs = rs_exact;
-      if (m_tile != -INFINITY) {
-        const float pmax = ex2(fmaf(mr, scale_log2, -m_eff));
+      if (xm != -INFINITY) {
+        const float pmax = ex2(xm);
         float r0, r1;
         unpack2<BF16>(pack2<BF16>(pmax, 0.f), r0, r1);
         rs += r0 - pmax;

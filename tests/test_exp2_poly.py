@@ -13,7 +13,7 @@ def test_header_constants_are_the_minimax_fit():
 
 def test_emulated_exp2_accuracy_over_the_softmax_range():
     c = exp2_poly.header_coefficients()
-    x = np.concatenate([np.linspace(-125.0, 8.5, 400001, dtype=np.float32),
+    x = np.concatenate([np.linspace(-125.0, 16.0, 400001, dtype=np.float32),
                         np.array([0.0, -0.5, 0.5, 1.0, -1.0, 8.0, -125.0], dtype=np.float32)])
     got = exp2_poly.exp2_emulated(x, c).astype(np.float64)
     ref = np.exp2(x.astype(np.float64))

@@ -213,7 +213,7 @@ def test_rows_subset_and_threads(oracle_mod):
     assert np.array_equal(orow, of[rows]) and np.array_equal(lrow, lf[rows])
 
 
-@pytest.mark.parametrize("tau", [0.0, 8.0])
+@pytest.mark.parametrize("tau", [0.0, 8.0, 15.0])
 @pytest.mark.parametrize("causal", [False, True])
 def test_online_blockwise_equals_two_pass(oracle_mod, tau, causal):
     """The tiled online softmax (the method) reaches the two-pass definition."""

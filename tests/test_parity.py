@@ -4,14 +4,16 @@ Small workloads are compared on every output; the full-size ones (the same launc
 configuration the benchmark times) on sampled rows that the oracle computes one by one.
 Tolerances: max|dO| <= 1e-2, mean|dO| <= 1e-3, max|dLSE| <= 1e-3 (fp32 O).
 """
+import math
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from exact_io_aware_59_b200 import binding
-from exact_io_aware_59_b200.inputs import WORKLOADS, workload_qkv
-from fa_testlib import REL_O16, compare, has_b200, sample_rows
+from exact_io_aware_59_b200.inputs import WORKLOADS, randn, workload_qkv
+from fa_testlib import REL_O16, compare, has_b200, sample_rows, scale_for
 
 pytestmark = pytest.mark.gpu
 
@@ -104,4 +106,28 @@ def test_decode_small_full_compare():
     o, lse = binding.attention(q.cuda(), k.cuda(), v.cuda(), scale=0.09)
     torch.cuda.synchronize()
     o_ref, l_ref = oracle.attention(q, k, v, 0.09, False)
+    compare(o, lse, o_ref, l_ref)
+
+
+@pytest.mark.parametrize("growth", [12.0, 20.0, -20.0])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)])
+def test_running_max_growing_along_keys(growth, causal, d, dtype):
+    """Scores that rise (or fall) by `growth` log2 units per 128-key tile, plus noise.
+    Rising by 20 moves every row's reference max on every tile (rescale of O, and the
+    early exponentiation against the old max is redone); rising by 12 makes the reference
+    max lag the true one without moving it, so p reaches ~2^12 (close to the fp16 limit
+    for the lag); falling leaves the first tile's max in charge."""
+    B, H, N = 1, 2, 1000
+    scale = scale_for(d)
+    g = growth / (128 * scale * math.log2(math.e))
+    q = randn((B, H, N, d), 71, torch.float32, 0.3)
+    k = randn((B, H, N, d), 72, torch.float32, 0.3)
+    v = randn((B, H, N, d), 73, dtype)
+    q[..., 0] = 1.0
+    k[..., 0] = g * torch.arange(N, dtype=torch.float32)
+    q, k = q.to(dtype), k.to(dtype)
+    o, lse = binding.attention(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.attention(q, k, v, scale, causal)
     compare(o, lse, o_ref, l_ref)
