@@ -229,6 +229,9 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
       tc_commit(bar_addr(bars, C::kBarSFull + t));
     }
     tc_commit(bar_addr(bars, C::kBarEmpty + kslot0));
+    // The Q tiles are free once the last S that reads them completes: release them then,
+    // so the next unit's Q load overlaps this unit's last softmax and P V products.
+    if (nmax == 1) tc_commit(bar_addr(bars, C::kBarQEmpty));
     for (int j = 0; j < nmax && ok; ++j) {
       const uint32_t vslot = ld % S;
       if (!wait(C::kBarFull + vslot, (ld / S) & 1)) { ok = false; break; }
@@ -258,9 +261,9 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
       if (!ok) break;
       tc_commit(bar_addr(bars, C::kBarEmpty + vslot));
       if (knext >= 0) tc_commit(bar_addr(bars, C::kBarEmpty + knext));
+      if (j == nmax - 2) tc_commit(bar_addr(bars, C::kBarQEmpty));  // last S was issued above
     }
     if (!ok) break;
-    tc_commit(bar_addr(bars, C::kBarQEmpty));
     ++q_used;
   }
   // No MMA may still be running when the TMEM is released.
@@ -384,45 +387,46 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
         f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
         return a0 + a1;
       };
-      // Row max of x = s * scale * log2(e) over the visible columns, taken on the raw
-      // scores (their min when the scale is negative) and scaled once.
+      uint32_t s[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
+      tmem_ld_wait_only();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(s[c]);
       float xm, rs_exact;  // xm: largest x - m_eff of the row's visible scores (-inf if none)
       bool done = false;
       if (full && __all_sync(0xffffffffu, m_used != -INFINITY)) {
         // Once a row has a finite reference max, a tile with every column visible rarely
         // moves it: exponentiate against it straight away, taking the row max of the
-        // exponents in the same pass, so the reduction is off the path to P.  P stays in
-        // registers until the max is known; if it moved by more than kLazyLog2 anywhere in the
-        // warp, the tile is redone below from S, still intact in TMEM.
-        uint32_t s[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
-        tmem_ld_wait_only();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+        // exponents in the same pass, so the reduction is off the path to P, and store each
+        // chunk of P as soon as it is packed.  P overwrites S columns 0-63 (score chunks 0
+        // and 1, which stay in registers); chunks 2 and 3 stay intact in TMEM.  If the max
+        // moved by more than kLazyLog2 anywhere in the warp, the tile is redone below from
+        // those; P has not been released yet.
         const uint64_t nm2 = f2_pack(-m_used, -m_used);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pk[4][16];
         float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) exp_pack32<BF16, true, true>(s[c], sc2, nm2, 32 * c, lim_c, pk[c], acc, mx);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+          exp_pack32<BF16, true, true>(s[c], sc2, nm2, 32 * c, lim_c, pk, acc, mx);
+          tmem_st_32x32b_x16(tS + 16 * c, pk);
+        }
         xm = fmaxf(mx[0], mx[1]);
         done = !__any_sync(0xffffffffu, xm > kLazyLog2);
         if (done) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_st_32x32b_x16(tS + 16 * c, pk[c]);
           float a0, a1;
           f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
           rs_exact = a0 + a1;
+        } else {
+#pragma unroll
+          for (int c = 2; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
+          tmem_ld_wait_only();
+#pragma unroll
+          for (int c = 2; c < 4; ++c) reg_fence(s[c]);
         }
       }
       if (!done) {
-        uint32_t s[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
-        tmem_ld_wait_only();
-#pragma unroll
-        for (int c = 0; c < 4; ++c) reg_fence(s[c]);
         if (!full) {
           const float sentinel = NEG ? INFINITY : -INFINITY;
 #pragma unroll
@@ -437,11 +441,20 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
         // Lazy rescale: move the reference max only when it grows by more than kLazyLog2.
         // -inf -> finite always moves; -inf -> -inf gives NaN and never moves.
         const bool move = (m_new - m_used) > kLazyLog2;
+        const float alpha = move ? ex2(m_used - m_new) : 1.0f;
+        if (move) {
+          l *= alpha;
+          l_exact *= alpha;
+          m_used = m_new;
+        }
+        const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+        rs_exact = exp_pass(s, m_eff, full);
+        xm = (m_tile == -INFINITY) ? -INFINITY : fmaf(mr, scale_log2, -m_eff);
         if (j > 0 && __any_sync(0xffffffffu, move)) {
-          // O_t still holds P V of tiles < j: wait for the last of those products.
+          // O_t still holds P V of tiles < j: wait for the last of those products, then
+          // bring it to the new reference (before P is released to the next product).
           if (!wait(C::kBarODone + t, (o_seen + j - 1) & 1)) return;
           tc_fence_after();
-          const float alpha = move ? ex2(m_used - m_new) : 1.0f;
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t ob[32];
@@ -452,15 +465,6 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
             tmem_st_32x32b_x32(tO + cc * 32, ob);
           }
         }
-        if (move) {
-          const float a = ex2(m_used - m_new);
-          l *= a;
-          l_exact *= a;
-          m_used = m_new;
-        }
-        const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-        rs_exact = exp_pass(s, m_eff, full);
-        xm = (m_tile == -INFINITY) ? -INFINITY : fmaf(mr, scale_log2, -m_eff);
       }
       // O is divided by the row sum of the rounded P that the P V product uses, taken as the
       // unrounded sum plus the rounding error of each tile's largest P.  That one term
