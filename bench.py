@@ -350,7 +350,8 @@ def arm_ours(args, ws, rank, local):
             "unit": "GB/s", "ms_per_step": ms_d, "steps": dsteps,
             "gpu_launches": 2 * dsteps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                         "traffic": DECODE_TRAFFIC.get((DECODE_REV, wd.name)),
                          "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": bytes_d},
             "clocks": clk_d.summary(),
@@ -395,10 +396,14 @@ def arm_ours(args, ws, rank, local):
 
 
 # Bumped whenever the prefill kernel changes, so stale ncu traffic is not reported.
-KERNEL_REV = "prefill-v9"
+KERNEL_REV = "prefill-v12"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the
 # kernel at this revision (profiles/fa_prefill_sm100_<workload>.md).
-DRAM_TRAFFIC = {("prefill-v1", "long_prefill_causal"): 629.5e6}
+DRAM_TRAFFIC = {("prefill-v12", "long_prefill_causal"): 590.5e6}
+# The decode kernel's traffic per launch, taken on decode_4k (B16 H32 Nkv4096: 1.0816 GB)
+# and scaled by the keys streamed (x8 for Nkv 32768): the kernel reads each key once.
+DECODE_REV = "decode-v1"
+DECODE_TRAFFIC = {("decode-v1", "decode"): 8 * 1.0816e9}
 
 
 def main():
