@@ -37,6 +37,11 @@ constexpr int kRegsLaunch = 168;   // 65536 / 384, rounded down to a multiple of
 constexpr int kRegsSide = 88;      // warpgroup 0 (load + MMA issue)
 constexpr int kRegsSoftmax = 208;  // warpgroups 1 and 2; 128*88 + 256*208 == 384*168
 static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+// One score pair in kFmaExp2Every takes 2^x on the FMA pipe (exp2_poly_pair) instead of the
+// SFU; 0 sends every score to the SFU.  Timed back to back at the boosted clock, one pair in
+// four and none ran equally fast; timed for seconds under the 1 kW power cap, where the
+// polynomial's extra instructions cost clock, the SFU alone was 2.8% faster.
+constexpr int kFmaExp2Every = 0;
 // Lazy rescale threshold in log2 units: the reference max m_used of a row moves only when
 // a tile's max exceeds it by more than this, so p = 2^(x - m_used) <= 2^15, below the fp16
 // maximum 65504 (bf16 and the fp32 O and l have far more range).  O and l share m_used,
@@ -294,8 +299,9 @@ __device__ __forceinline__ float row_reduce(const uint32_t (&s)[4][32]) {
 // p = 2^(s * scale_log2 - m) for 32 scores (tile columns col0 .. col0+31), rounded in
 // pairs to the 16-bit type into pk (exp_pack_store32 also stores them to 16 TMEM columns
 // at tP, two values per column); adds the unrounded p to the running sums, and with XMAX
-// folds the exponents x = s * scale_log2 - m into two running maxima.  FULL: every column visible; one pair in four
-// takes the FMA-pipe exp2, the rest the SFU.  !FULL: columns past lim_c get p = 0.
+// folds the exponents x = s * scale_log2 - m into two running maxima.  FULL: every column
+// visible (and, with kFmaExp2Every > 0, one pair in kFmaExp2Every takes the FMA-pipe
+// exp2).  !FULL: columns past lim_c get p = 0.
 template <bool BF16, bool FULL, bool XMAX = false>
 __device__ __forceinline__ void exp_pack32(const uint32_t (&s)[32], uint64_t sc2, uint64_t nm2,
                                            int col0, int lim_c, uint32_t (&pk)[16],
@@ -306,7 +312,7 @@ __device__ __forceinline__ void exp_pack32(const uint32_t (&s)[32], uint64_t sc2
     float x0, x1, p0, p1;
     f2_unpack(x2, x0, x1);
     if (XMAX) xmax[i & 1] = max3(xmax[i & 1], x0, x1);
-    if (FULL && (i & 3) == 1) {
+    if (FULL && kFmaExp2Every > 0 && (i % (kFmaExp2Every > 0 ? kFmaExp2Every : 1)) == 1) {
       f2_unpack(exp2_poly_pair(x0, x1), p0, p1);
     } else {
       p0 = ex2(x0);
