@@ -147,6 +147,39 @@ def attention(q, k, v, scale: float, causal: bool, rows: Optional[Sequence[int]]
     return o, lse
 
 
+def paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, scale: float,
+                           nthreads: int = 0, lib=None):
+    """Decode (one query per head) against a paged KV cache, in fp64.
+
+    q: [B,H,d]; k_cache, v_cache: [num_pages, H, page_size, d]; block_table: [B, P]
+    integers; seq_lens: [B].  Logical key i of sequence b is slot i mod page_size of page
+    block_table[b, i // page_size] -- the KV-cache pages of PagedAttention ("FlashAttention
+    1-2-3" (myaihardware), section "FlashAttention in production": vLLM's PagedAttention
+    over KV cache blocks).  The keys of each sequence are gathered in logical order and the
+    result is attention() over them (no mask: the query follows every cached key).  A
+    sequence with no keys gives O = 0 and LSE = -inf.  Returns (o [B,H,d], lse [B,H]).
+    """
+    import torch
+    B, H, d = q.shape
+    ps = k_cache.shape[2]
+    o = np.zeros((B, H, d), dtype=np.float64)
+    lse = np.full((B, H), -np.inf, dtype=np.float64)
+    bt = torch.as_tensor(block_table).to(torch.int64).cpu()
+    for b in range(B):
+        L = int(seq_lens[b])
+        if L == 0:
+            continue
+        pages = bt[b, : (L + ps - 1) // ps]
+        kb = k_cache[pages].permute(1, 0, 2, 3).reshape(H, -1, d)[:, :L]
+        vb = v_cache[pages].permute(1, 0, 2, 3).reshape(H, -1, d)[:, :L]
+        ob, lb = attention(q[b].reshape(1, H, 1, d), kb.reshape(1, H, L, d).contiguous(),
+                           vb.reshape(1, H, L, d).contiguous(), scale, False,
+                           nthreads=nthreads, lib=lib)
+        o[b] = ob[0, :, 0]
+        lse[b] = lb[0, :, 0]
+    return o, lse
+
+
 def _f64(x):
     try:
         import torch

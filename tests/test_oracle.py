@@ -273,3 +273,60 @@ def test_golden_byte_counts(oracle_mod):
                 assert abs(t["total"] / 1e6 - val) < 2
             else:
                 assert round(t[term] / 1e6) == val
+
+
+# ---------------------------------------------------------------- paged KV cache (decode)
+def _scatter_pages(K, V, page_size, num_pages, rng, dtype):
+    """Writes contiguous K, V [B,H,Lmax,d] into pages [num_pages,H,page_size,d] in a random
+    page order (unused pages and slots hold other random values); returns the caches and
+    the block table."""
+    B, H, Lmax, d = K.shape
+    P = (Lmax + page_size - 1) // page_size
+    perm = rng.permutation(num_pages)[: B * P].reshape(B, P)
+    kc = torch.randn(num_pages, H, page_size, d).to(dtype)
+    vc = torch.randn(num_pages, H, page_size, d).to(dtype)
+    for b in range(B):
+        for i in range(P):
+            n = min(page_size, Lmax - i * page_size)
+            kc[perm[b, i], :, :n] = K[b, :, i * page_size: i * page_size + n]
+            vc[perm[b, i], :, :n] = V[b, :, i * page_size: i * page_size + n]
+    return kc, vc, torch.from_numpy(perm.astype(np.int32))
+
+
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_paged_decode_equals_contiguous(oracle_mod, page_size):
+    """Pages in a random order, ragged lengths (0, 1, a page, a page + 1, full): the
+    paged oracle equals attention() over each sequence's contiguous keys."""
+    rng = np.random.default_rng(page_size)
+    B, H, Lmax, d = 6, 3, 200, 32
+    q = make_qkv(B, H, 1, 1, d, torch.bfloat16, 500)[0][:, :, 0]
+    _, K, V = make_qkv(B, H, 1, Lmax, d, torch.bfloat16, 510)
+    kc, vc, bt = _scatter_pages(K, V, page_size, 96, rng, torch.bfloat16)
+    lens = [0, 1, page_size, page_size + 1, 137, Lmax]
+    o, lse = oracle_mod.paged_decode_attention(q, kc, vc, bt, lens, 0.3)
+    for b, L in enumerate(lens):
+        if L == 0:
+            assert (o[b] == 0).all() and np.isneginf(lse[b]).all()
+            continue
+        o_ref, l_ref = oracle_mod.attention(q[b].reshape(1, H, 1, d), K[b:b + 1, :, :L].contiguous(),
+                                            V[b:b + 1, :, :L].contiguous(), 0.3, False)
+        np.testing.assert_allclose(o[b], o_ref[0, :, 0], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], l_ref[0, :, 0], rtol=0, atol=1e-12)
+
+
+def test_paged_decode_pin_sees_a_wrong_page():
+    """Negative control for the pin above: pointing one block-table entry at a page the
+    sequence does not own changes the result, so a mis-indexed page would be caught.
+    (Reordering a sequence's own pages would not: without a mask the keys form a set.)"""
+    import oracle
+    rng = np.random.default_rng(3)
+    B, H, Lmax, d, ps = 1, 2, 128, 16, 16
+    q = make_qkv(B, H, 1, 1, d, torch.bfloat16, 520)[0][:, :, 0]
+    _, K, V = make_qkv(B, H, 1, Lmax, d, torch.bfloat16, 530)
+    kc, vc, bt = _scatter_pages(K, V, ps, 16, rng, torch.bfloat16)
+    unused = sorted(set(range(16)) - set(bt[0].tolist()))[0]
+    bt2 = bt.clone()
+    bt2[0, 2] = unused
+    o1, _ = oracle.paged_decode_attention(q, kc, vc, bt, [Lmax - 20], 1.0)
+    o2, _ = oracle.paged_decode_attention(q, kc, vc, bt2, [Lmax - 20], 1.0)
+    assert np.isfinite(o1).all() and not np.allclose(o1, o2, atol=1e-6)
