@@ -4,7 +4,10 @@ One step = one pass of the hot path over one batch of synthetic input:
   * the headline line times the long causal prefill (B=1, H=32, N=8192, d=128, bf16), one
     fa_fwd call per step;
   * the "decode" object times the split-KV decode (B=16, H=32, Nq=1, Nkv=32768, d=128,
-    bf16), one fa_fwd call (split kernel + combine kernel) per step.
+    bf16), one fa_fwd call (split kernel + combine kernel) per step;
+  * the "decode_paged" object times the same decode against a paged KV cache (64-key
+    pages scattered over the pool by a seeded random block table), one
+    fa_fwd_decode_paged call per step.
 Inputs are resident in HBM and larger than L2 (126 MB) when the timed region starts.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -31,7 +34,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_io_aware_59_b200 import binding  # noqa: E402
-from exact_io_aware_59_b200.inputs import WORKLOADS, Workload, workload_qkv  # noqa: E402
+from exact_io_aware_59_b200.inputs import (WORKLOADS, Workload, paged_decode_inputs,  # noqa: E402
+                                           workload_qkv)
 
 METRIC = "attention fwd TFLOP/s at 1 B200 (% of dense bf16 peak); decode HBM GB/s"
 PREFILL = "long_prefill_causal"
@@ -358,6 +362,42 @@ def arm_ours(args, ws, rank, local):
         }
         torch.cuda.empty_cache()
 
+    # decode against a paged KV cache (same shape as the decode workload)
+    decode_paged = None
+    if not args.skip_decode:
+        wd = WORKLOADS[args.decode_workload]
+        ps = 64
+        pq, kc, vc, table, sl = paged_decode_inputs(wd.B, wd.H, wd.Nkv, wd.d, ps, wd.dtype,
+                                                    1000 * wd.index + 500, device="cuda")
+        po = torch.empty((wd.B, wd.H, wd.d), dtype=wd.dtype, device="cuda")
+        pl = torch.empty((wd.B, wd.H), dtype=torch.float32, device="cuda")
+        pargs = (pq.data_ptr(), kc.data_ptr(), vc.data_ptr(), table.data_ptr(), sl.data_ptr(),
+                 po.data_ptr(), pl.data_ptr(), wd.B, wd.H, wd.d, ps, table.shape[1], kc.shape[0],
+                 float(wd.softmax_scale), stream.cuda_stream, binding._dtype_code(wd.dtype),
+                 binding._dtype_code(wd.dtype), 0)
+
+        def paged_call():
+            check(binding.fa_fwd_decode_paged(*pargs), "fa_fwd_decode_paged")
+
+        psteps = max(3, args.steps // 8)
+        with ClockSampler(local) as clk_p, torch.cuda.stream(stream):
+            ms_pd = time_steps(paged_call, psteps, args.warmup, ws, stream)
+        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+        bytes_pd = algorithmic_bytes(wd, 2)
+        gbs_pd = bytes_pd / (ms_pd * 1e-3) / 1e9
+        decode_paged = {
+            "workload": f"{wd.name} in a paged cache: {ps}-key pages, block table a seeded "
+                        f"random permutation of {kc.shape[0]} pages",
+            "value": whole_job_rate(bytes_pd, ms_pd, ws) / 1e9, "unit": "GB/s",
+            "ms_per_step": ms_pd, "steps": psteps, "gpu_launches": 2 * psteps,
+            "roofline": {"bound": "hbm", "achieved": gbs_pd, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs_pd / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": peak_src, "algorithmic_bytes_per_launch": bytes_pd},
+            "clocks": clk_p.summary(),
+        }
+        del pq, kc, vc, table, sl, po, pl
+        torch.cuda.empty_cache()
+
     # end to end through the C ABI with host buffers
     e2e = None
     if not args.skip_e2e:
@@ -389,6 +429,7 @@ def arm_ours(args, ws, rank, local):
                          "frac_of_sustained": tflops / peaks.get("bf16_tflops_sustained", peak_t)},
             "clocks": clk.summary(),
             "decode": decode,
+            "decode_paged": decode_paged,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

@@ -19,6 +19,7 @@ from . import build as _build
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ARCH = 0, 1, 2, 3
 FA_ERR_CUDA, FA_ERR_NOMEM, FA_ERR_DEVICE_TIMEOUT = 4, 5, 6
 FA_F16, FA_BF16, FA_F32 = 0, 1, 2
+FA_DEV_BAD_INPUT = 16
 
 HEADER = os.path.join(_build.INCLUDE, "fa.h")
 
@@ -40,6 +41,8 @@ _SIGNATURES = {
     "fa_fwd_prefill": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I, _I],
     "fa_fwd_decode": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
     "fa_fwd_decode_noalloc": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
+    "fa_fwd_decode_paged": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP,
+                            _I, _I, _I],
     "fa_decode_workspace_bytes": [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
     "fa_device_status": [ctypes.POINTER(_I), _I],
     "fa_selftest_wait_timeout": [_VP],
@@ -104,6 +107,14 @@ def fa_fwd_decode_noalloc(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype
     instead of a cudaMalloc'd workspace, for callers that cannot allocate device memory."""
     return library().fa_fwd_decode_noalloc(q, k, v, o, lse, B, H, Nkv, d, scale, stream,
                                            in_dtype, o_dtype, num_splits)
+
+
+def fa_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, H, d, page_size,
+                        max_pages_per_seq, num_pages, scale, stream, in_dtype, o_dtype,
+                        num_splits) -> int:
+    return library().fa_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, H,
+                                         d, page_size, max_pages_per_seq, num_pages, scale,
+                                         stream, in_dtype, o_dtype, num_splits)
 
 
 def fa_decode_workspace_bytes(B, H, Nkv, d, num_splits) -> int:
@@ -183,3 +194,38 @@ def attention(q, k, v, causal: bool = False, scale: Optional[float] = None,
     if rc != FA_OK:
         raise FaError(rc, where)
     return out, lse
+
+
+def paged_decode(q, k_cache, v_cache, block_table, seq_lens, scale: Optional[float] = None,
+                 out_dtype=None, num_splits: int = 0, stream=None):
+    """Decode against a paged KV cache: q [B,H,d]; k_cache, v_cache
+    [num_pages,H,page_size,d] (q's fp16/bf16 type); block_table int32 [B,P]; seq_lens int32
+    [B] -- all contiguous CUDA tensors.  Returns (o [B,H,d], lse [B,H]); out_dtype
+    torch.float32 (default) or q's dtype."""
+    import torch
+
+    ts = (q, k_cache, v_cache, block_table, seq_lens)
+    if not all(t.is_cuda and t.is_contiguous() for t in ts):
+        raise ValueError("paged_decode() takes contiguous CUDA tensors")
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    B, H, d = q.shape
+    num_pages, Hc, page_size, dc = k_cache.shape
+    if (Hc, dc) != (H, d) or tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("caches must be [num_pages, H, page_size, d] with q's H and d")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("block_table must be [B, P] and seq_lens [B]")
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    s = torch.cuda.current_stream(q.device) if stream is None else stream
+    with torch.cuda.device(q.device):
+        rc = fa_fwd_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                 block_table.data_ptr(), seq_lens.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr(), B, H, d, page_size, block_table.shape[1],
+                                 num_pages, scale, s.cuda_stream, _dtype_code(q.dtype),
+                                 _dtype_code(o.dtype), num_splits)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_decode_paged")
+    return o, lse

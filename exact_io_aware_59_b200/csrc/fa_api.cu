@@ -183,7 +183,7 @@ int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse
 
 int run_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                int Nkv, int d, float scale, void* stream, int in_dtype, int o_dtype,
-               int num_splits) {
+               int num_splits, const fa::PagedKV* paged = nullptr) {
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != FA_OK) return rc;
@@ -208,8 +208,40 @@ int run_decode(const void* q, const void* k, const void* v, void* o, float* lse,
   float* part_o = ds->ws;
   float* part_lse = ds->ws + static_cast<size_t>(p.grid) * p.max_seg * 8 * d;
   cudaError_t e = fa::launch_decode(q, k, v, o, lse, p, d, in_dtype == FA_BF16, o_dtype == FA_F32,
-                                    part_o, part_lse, ds->status, static_cast<cudaStream_t>(stream));
+                                    part_o, part_lse, ds->status, static_cast<cudaStream_t>(stream),
+                                    paged);
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+// Host checks of fa_fwd_decode_paged (everything but the device-resident table and lengths).
+int check_paged_args(const void* q, const void* kc, const void* vc, const int* table,
+                     const int* lens, void* o, float* lse, int B, int H, int d, int page_size,
+                     int max_pages, int num_pages, float scale, int in_dtype, int o_dtype,
+                     int num_splits) {
+  if (!q || !kc || !vc || !table || !lens || !o) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || max_pages < 1 || num_pages < 1 || num_splits < 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (page_size < 16 || page_size > 1024 || (page_size & (page_size - 1)) != 0) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_pages) * page_size > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (in_dtype != FA_F16 && in_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_F16 && o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_F32 && o_dtype != in_dtype) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(o, 16)) return FA_ERR_INVALID_ARG;
+  if (!aligned(table, 4) || !aligned(lens, 4) || (lse && !aligned(lse, 4))) return FA_ERR_INVALID_ARG;
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t qb = BH * d * 2, ob = BH * d * (o_dtype == FA_F32 ? 4 : 2), lb = BH * 4;
+  const size_t cb = static_cast<size_t>(num_pages) * H * page_size * d * 2;
+  const size_t tb = static_cast<size_t>(B) * max_pages * 4, sb = static_cast<size_t>(B) * 4;
+  const void* ins[5] = {q, kc, vc, table, lens};
+  const size_t in_bytes[5] = {qb, cb, cb, tb, sb};
+  for (int i = 0; i < 5; ++i) {
+    if (overlaps(o, ob, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+    if (lse && overlaps(lse, lb, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+  }
+  if (lse && overlaps(lse, lb, o, ob)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
 }
 
 }  // namespace
@@ -253,6 +285,23 @@ int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* l
   if (rc != FA_OK) return rc;
   if (num_splits < 0) return FA_ERR_INVALID_ARG;
   return run_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype, num_splits);
+}
+
+int fa_fwd_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                        const int* block_table, const int* seq_lens, void* o, float* lse,
+                        int B, int H, int d, int page_size, int max_pages_per_seq,
+                        int num_pages, float scale, void* stream, int in_dtype, int o_dtype,
+                        int num_splits) {
+  const int rc = check_paged_args(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, H, d,
+                                  page_size, max_pages_per_seq, num_pages, scale, in_dtype,
+                                  o_dtype, num_splits);
+  if (rc != FA_OK) return rc;
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  const fa::PagedKV pk{block_table, seq_lens, H, shift, max_pages_per_seq, num_pages};
+  // Every head gets the table's capacity of key slots; the kernels skip the empty ones.
+  return run_decode(q, k_cache, v_cache, o, lse, B, H, max_pages_per_seq * page_size, d, scale,
+                    stream, in_dtype, o_dtype, num_splits, &pk);
 }
 
 int fa_decode_workspace_bytes(int B, int H, int Nkv, int d, int num_splits, size_t* bytes) {

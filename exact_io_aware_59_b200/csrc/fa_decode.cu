@@ -17,6 +17,12 @@
 // products in 9 shuffles), then each lane accumulates its own d-slice of P V in fp32.
 // Each time a CTA finishes the part of a head it owns, every consumer warp writes one
 // partial record (O_s, lse_s) for the keys it saw; the combine kernel merges them all.
+//
+// Paged KV cache ("FlashAttention 1-2-3" (myaihardware), section "Integration in Major
+// Inference Engines"): the same kernels, with each head given the table's capacity of
+// 64-key chunk slots.  A chunk's keys are gathered page by page (one bulk copy per page
+// it touches) from [num_pages, H, page_size, d] caches through the block table; slots
+// past a sequence's length are skipped by producer and consumers alike.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -46,6 +52,26 @@ __device__ __forceinline__ long long chunk_begin(const DecodeParams& p, int cta)
   return static_cast<long long>(cta) * p.total / p.grid;
 }
 
+// Chunk c of the flat range: its head, first key and number of keys (<= 0: an empty slot
+// past the sequence's length).  With a paged cache the length comes from seq_lens,
+// clamped to [0, capacity]; `flag` (the producer) records a clamp in the status word.
+template <bool PAGED>
+__device__ __forceinline__ void chunk_info(const DecodeParams& p, const PagedKV& pk, long long c,
+                                           int& h, int& key0, int& nk, int* status, bool flag) {
+  h = static_cast<int>(c / p.n_chunks);
+  key0 = static_cast<int>(c % p.n_chunks) * kDecodeChunk;
+  int len = p.Nkv;
+  if constexpr (PAGED) {
+    const int cap = pk.max_pages << pk.page_shift;
+    len = pk.seq_lens[h / pk.H];
+    if (len < 0 || len > cap) {
+      if (flag) atomicOr(status, kStatusBadInput);
+      len = len < 0 ? 0 : cap;
+    }
+  }
+  nk = min(kDecodeChunk, len - key0);
+}
+
 template <int D, bool BF16>
 __device__ __forceinline__ void load_slice(const uint8_t* row, int lane, float (&x)[D / 32]) {
   constexpr int E = D / 32;  // elements per lane
@@ -59,11 +85,11 @@ __device__ __forceinline__ void load_slice(const uint8_t* row, int lane, float (
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_decode_split_sm100(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                           const uint16_t* __restrict__ v, float* __restrict__ part_o,
-                          float* __restrict__ part_lse, const DecodeParams p,
+                          float* __restrict__ part_lse, const DecodeParams p, const PagedKV pk,
                           int* __restrict__ status) {
   using C = DecodeCfg<D>;
   constexpr int S = C::kStages;
@@ -93,10 +119,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t policy = l2_policy_evict_first();
       uint32_t ld = 0;
       bool ok = true;
-      for (long long c = c_begin; c < c_end; ++c, ++ld) {
-        const int h = static_cast<int>(c / p.n_chunks);
-        const int key0 = static_cast<int>(c % p.n_chunks) * kDecodeChunk;
-        const int nk = min(kDecodeChunk, p.Nkv - key0);
+      for (long long c = c_begin; c < c_end; ++c) {
+        int h, key0, nk;
+        chunk_info<PAGED>(p, pk, c, h, key0, nk, status, true);
+        if (nk <= 0) continue;  // empty slot: no stage, the consumers skip it too
         const uint32_t bytes = static_cast<uint32_t>(nk) * D * 2;
         const uint32_t slot = ld % S;
         if (!mbar_wait(bars + 8 * (S + slot), ((ld / S) & 1) ^ 1, status, abort_flag,
@@ -106,10 +132,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t fb = bars + 8 * slot;
         mbar_arrive_expect_tx(fb, 2 * bytes);
-        const size_t off = (static_cast<size_t>(h) * p.Nkv + key0) * D;
         const uint32_t dst = sbase + slot * C::kStageBytes;
-        bulk_load_stream(dst, k + off, bytes, fb, policy);
-        bulk_load_stream(dst + C::kChunkBytes, v + off, bytes, fb, policy);
+        if constexpr (PAGED) {
+          // One copy per page the chunk touches: [key, key + seg) lies in logical page
+          // key >> page_shift of sequence b, at slot key & (page_size - 1).
+          const int b = h / pk.H, hh = h % pk.H;
+          const int ps = 1 << pk.page_shift;
+          for (int key = key0; key < key0 + nk;) {
+            const int in_page = key & (ps - 1);
+            const int seg = min(key0 + nk - key, ps - in_page);
+            int page = pk.block_table[static_cast<size_t>(b) * pk.max_pages + (key >> pk.page_shift)];
+            if (page < 0 || page >= pk.num_pages) {
+              atomicOr(status, kStatusBadInput);
+              page = 0;
+            }
+            const size_t off = ((static_cast<size_t>(page) * pk.H + hh) * ps + in_page) * D;
+            const uint32_t sb = static_cast<uint32_t>(seg) * D * 2;
+            const uint32_t so = static_cast<uint32_t>(key - key0) * D * 2;
+            bulk_load_stream(dst + so, k + off, sb, fb, policy);
+            bulk_load_stream(dst + C::kChunkBytes + so, v + off, sb, fb, policy);
+            key += seg;
+          }
+        } else {
+          const size_t off = (static_cast<size_t>(h) * p.Nkv + key0) * D;
+          bulk_load_stream(dst, k + off, bytes, fb, policy);
+          bulk_load_stream(dst + C::kChunkBytes, v + off, bytes, fb, policy);
+        }
+        ++ld;
       }
       if (!ok) {
         for (uint32_t i = (ld > (uint32_t)S ? ld - S : 0); i < ld; ++i) {
@@ -146,10 +195,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         part_lse[rec] = (l_w > 0.f) ? (m + log2f(l_w)) * 0.69314718055994531f : -INFINITY;
     };
 
-    for (long long c = c_begin; c < c_end; ++c, ++ld) {
-      const int h = static_cast<int>(c / p.n_chunks);
-      const int key0 = static_cast<int>(c % p.n_chunks) * kDecodeChunk;
-      const int nk = min(kDecodeChunk, p.Nkv - key0);
+    for (long long c = c_begin; c < c_end; ++c) {
+      int h, key0, nk;
+      chunk_info<PAGED>(p, pk, c, h, key0, nk, status, false);
       if (h != cur_h) {
         if (cur_h >= 0) finish_segment(cur_h);
         cur_h = h;
@@ -163,6 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = -INFINITY;
         l_lane = 0.f;
       }
+      // An empty slot still opens its head (so every segment gets its records), but has
+      // no stage to read.
+      if (nk <= 0) continue;
       const uint32_t slot = ld % S;
       const bool got = mbar_wait(bars + 8 * slot, (ld / S) & 1, status, abort_flag,
                                  kStatusTimeoutDecode);
@@ -235,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + 8 * (S + slot));
+      ++ld;
     }
     if (ok && cur_h >= 0) finish_segment(cur_h);
   }
@@ -326,14 +378,15 @@ __global__ void __launch_bounds__(128)
 template <int D, bool BF16>
 cudaError_t launch_t(const void* q, const void* k, const void* v, void* o, float* lse,
                      const DecodeParams& p, bool o_f32, float* part_o, float* part_lse,
-                     int* status, cudaStream_t stream) {
-  auto kern = fa_decode_split_sm100<D, BF16>;
+                     int* status, cudaStream_t stream, const PagedKV* paged) {
+  auto kern = paged ? fa_decode_split_sm100<D, BF16, true> : fa_decode_split_sm100<D, BF16, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        DecodeCfg<D>::kBytes);
   if (e != cudaSuccess) return e;
+  const PagedKV pk = paged ? *paged : PagedKV{nullptr, nullptr, 1, 0, 0, 0};
   kern<<<p.grid, kThreads, DecodeCfg<D>::kBytes, stream>>>(
       static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
-      static_cast<const uint16_t*>(v), part_o, part_lse, p, status);
+      static_cast<const uint16_t*>(v), part_o, part_lse, p, pk, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (o_f32)
@@ -373,11 +426,12 @@ size_t decode_smem_bytes(int d) {
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                           const DecodeParams& p, int d, bool bf16, bool o_f32, float* part_o,
-                          float* part_lse, int* status, cudaStream_t stream) {
-  if (d == 128 && bf16) return launch_t<128, true>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream);
-  if (d == 128 && !bf16) return launch_t<128, false>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream);
-  if (d == 64 && bf16) return launch_t<64, true>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream);
-  if (d == 64 && !bf16) return launch_t<64, false>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream);
+                          float* part_lse, int* status, cudaStream_t stream,
+                          const PagedKV* paged) {
+  if (d == 128 && bf16) return launch_t<128, true>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream, paged);
+  if (d == 128 && !bf16) return launch_t<128, false>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream, paged);
+  if (d == 64 && bf16) return launch_t<64, true>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream, paged);
+  if (d == 64 && !bf16) return launch_t<64, false>(q, k, v, o, lse, p, o_f32, part_o, part_lse, status, stream, paged);
   return cudaErrorInvalidValue;
 }
 

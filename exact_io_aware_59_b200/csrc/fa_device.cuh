@@ -15,6 +15,7 @@ enum : int {
   kStatusTimeoutMma = 1 << 1,       // the MMA issuer's wait ran out
   kStatusTimeoutSoftmax = 1 << 2,   // a softmax / epilogue wait ran out
   kStatusTimeoutDecode = 1 << 3,    // a split-KV decode wait ran out
+  kStatusBadInput = 1 << 4,         // paged decode: table entry or length out of range
 };
 
 // A wait that has not finished after this long is treated as a hang.

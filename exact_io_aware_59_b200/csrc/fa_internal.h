@@ -33,6 +33,16 @@ struct DecodeParams {
 
 constexpr int kDecodeChunk = 64;
 
+// Paged KV cache of a decode launch (null block_table: contiguous [B,H,Nkv,d] K/V).
+struct PagedKV {
+  const int* block_table;  // [B, max_pages] physical page of each logical page
+  const int* seq_lens;     // [B] keys per sequence
+  int H;                   // heads per sequence (flat head = b * H + h)
+  int page_shift;          // log2(page_size)
+  int max_pages;           // logical pages per sequence (table row length)
+  int num_pages;           // physical pages in the caches
+};
+
 // Kernel launchers (fa_prefill.cu, fa_decode.cu).  Return the launch's cudaError_t.
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            void* o, float* lse, const PrefillParams& p, int d, bool bf16,
@@ -40,7 +50,8 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                           const DecodeParams& p, int d, bool bf16, bool o_f32, float* part_o,
-                          float* part_lse, int* status, cudaStream_t stream);
+                          float* part_lse, int* status, cudaStream_t stream,
+                          const PagedKV* paged = nullptr);
 
 // Diagnostic kernel whose only wait can never finish (see fa_selftest_wait_timeout).
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t stream);

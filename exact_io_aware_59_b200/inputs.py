@@ -86,3 +86,20 @@ def make_qkv(B, H, Nq, Nkv, d, dtype, seed_base: int, q_std: float = 1.0, device
 
 def workload_qkv(w: Workload, device="cpu"):
     return make_qkv(w.B, w.H, w.Nq, w.Nkv, w.d, w.dtype, 1000 * w.index, w.q_std, device)
+
+
+def paged_decode_inputs(B: int, H: int, L: int, d: int, page_size: int, dtype: torch.dtype,
+                        seed_base: int, device="cpu"):
+    """A paged KV cache holding B sequences of L keys each: q [B,H,d]; k_cache, v_cache
+    [B*ceil(L/page_size), H, page_size, d] iid N(0,1) rounded to `dtype`; block_table
+    int32 [B, P] a seeded random permutation of all pages (so a sequence's pages are
+    scattered over the pool); seq_lens int32 [B] all L.  Seeds seed_base + 0..3."""
+    P = (L + page_size - 1) // page_size
+    q = randn((B, H, d), seed_base + 0, dtype, 1.0, device)
+    k_cache = randn((B * P, H, page_size, d), seed_base + 1, dtype, 1.0, device)
+    v_cache = randn((B * P, H, page_size, d), seed_base + 2, dtype, 1.0, device)
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed_base + 3))
+    table = torch.randperm(B * P, generator=g, device=device).to(torch.int32).reshape(B, P)
+    seq_lens = torch.full((B,), L, dtype=torch.int32, device=device)
+    return q, k_cache, v_cache, table.contiguous(), seq_lens

@@ -136,6 +136,35 @@ int fa_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* o, 
                           int B, int H, int Nkv, int d, float scale, void* stream,
                           int in_dtype, int o_dtype, int num_splits);
 
+/*
+ * fa_fwd_decode_paged -- split-KV decode for one query per head against a paged KV cache
+ * ("FlashAttention 1-2-3" (myaihardware), section "Integration in Major Inference
+ * Engines": each KV-cache page of vLLM's PagedAttention is a block the kernel tiles over;
+ * with the FlashDecoding split of section "Beyond FlashAttention").
+ *   q [B,H,d] and o [B,H,d] (o fp32 or q's 16-bit type), lse [B,H] fp32 (may be NULL).
+ *   k_cache, v_cache: [num_pages, H, page_size, d] in q's 16-bit type; the page_size x d
+ *   block of one head in one page is contiguous.
+ *   block_table: int32 [B, max_pages_per_seq]; logical key i of sequence b is slot
+ *   i % page_size of page block_table[b * max_pages_per_seq + i / page_size].
+ *   seq_lens: int32 [B], keys of each sequence, 0 <= seq_lens[b] <= max_pages_per_seq *
+ *   page_size; a sequence with no keys gets O = 0 and LSE = -inf.
+ *   All pointers are device memory owned by the caller and must stay valid until the
+ *   enqueued work completes; q, the caches and o 16-byte aligned, the rest 4-byte.
+ *   page_size: a power of two from 16 to 1024.  num_splits as for fa_fwd_decode; the
+ *   split covers max_pages_per_seq * page_size key slots per head, and slots past a
+ *   sequence's length cost nothing but their share of the split.
+ *   Errors: FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED for arguments checkable on the host
+ *   (nothing is enqueued).  Table entries and lengths live on the device: an entry
+ *   outside [0, num_pages) is replaced by page 0 and a length outside its range is
+ *   clamped, and FA_DEV_BAD_INPUT is set in the status word (fa_device_status); no
+ *   out-of-bounds read happens.  Same workspace as fa_fwd_decode.
+ */
+int fa_fwd_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                        const int* block_table, const int* seq_lens, void* o, float* lse,
+                        int B, int H, int d, int page_size, int max_pages_per_seq,
+                        int num_pages, float scale, void* stream, int in_dtype, int o_dtype,
+                        int num_splits);
+
 /* Bytes of decode workspace a fa_fwd_decode call with these arguments needs. */
 int fa_decode_workspace_bytes(int B, int H, int Nkv, int d, int num_splits, size_t* bytes);
 
@@ -152,7 +181,8 @@ enum {
   FA_DEV_TIMEOUT_LOAD = 1,      /* prefill: a TMA producer wait ran out */
   FA_DEV_TIMEOUT_MMA = 2,       /* prefill: the MMA issuer's wait ran out */
   FA_DEV_TIMEOUT_SOFTMAX = 4,   /* prefill: a softmax / epilogue wait ran out */
-  FA_DEV_TIMEOUT_DECODE = 8     /* decode: a split kernel wait ran out */
+  FA_DEV_TIMEOUT_DECODE = 8,    /* decode: a split kernel wait ran out */
+  FA_DEV_BAD_INPUT = 16         /* paged decode: a block-table entry or length out of range */
 };
 
 /*

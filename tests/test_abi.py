@@ -111,3 +111,34 @@ def test_binding_rejects_host_tensors():
     q = torch.zeros(1, 1, 4, 64, dtype=torch.float16)
     with pytest.raises(ValueError):
         binding.attention(q, q, q)
+
+
+def _paged(**kw):
+    a = dict(q=Q, kc=K, vc=V, table=L + 64, lens=L + 128, o=O, lse=L, B=1, H=1, d=64,
+             page_size=16, max_pages=4, num_pages=8, scale=0.1, stream=None, in_dtype=0,
+             o_dtype=2, num_splits=0)
+    a.update(kw)
+    return binding.fa_fwd_decode_paged(a["q"], a["kc"], a["vc"], a["table"], a["lens"], a["o"],
+                                       a["lse"], a["B"], a["H"], a["d"], a["page_size"],
+                                       a["max_pages"], a["num_pages"], a["scale"], a["stream"],
+                                       a["in_dtype"], a["o_dtype"], a["num_splits"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(table=None), binding.FA_ERR_INVALID_ARG),
+    (dict(lens=None), binding.FA_ERR_INVALID_ARG),
+    (dict(kc=None), binding.FA_ERR_INVALID_ARG),
+    (dict(page_size=8), binding.FA_ERR_INVALID_ARG),      # below 16
+    (dict(page_size=48), binding.FA_ERR_INVALID_ARG),     # not a power of two
+    (dict(page_size=2048), binding.FA_ERR_INVALID_ARG),
+    (dict(max_pages=0), binding.FA_ERR_INVALID_ARG),
+    (dict(num_pages=0), binding.FA_ERR_INVALID_ARG),
+    (dict(max_pages=1 << 22, page_size=1024), binding.FA_ERR_INVALID_ARG),  # > 2^31 keys
+    (dict(num_splits=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(table=L + 66), binding.FA_ERR_INVALID_ARG),     # misaligned int32 table
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(in_dtype=0, o_dtype=1), binding.FA_ERR_UNSUPPORTED),
+    (dict(o=K), binding.FA_ERR_INVALID_ARG),              # O on the key cache
+])
+def test_paged_decode_argument_checks(kw, code):
+    assert _paged(**kw) == code
