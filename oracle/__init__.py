@@ -154,8 +154,8 @@ def paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, scale: fl
     q: [B,H,d]; k_cache, v_cache: [num_pages, H, page_size, d]; block_table: [B, P]
     integers; seq_lens: [B].  Logical key i of sequence b is slot i mod page_size of page
     block_table[b, i // page_size] -- the KV-cache pages of PagedAttention ("FlashAttention
-    1-2-3" (myaihardware), section "FlashAttention in production": vLLM's PagedAttention
-    over KV cache blocks).  The keys of each sequence are gathered in logical order and the
+    1-2-3" (myaihardware), section "Integration in Major Inference Engines": each KV cache
+    page is a block the attention kernel tiles over).  The keys of each sequence are gathered in logical order and the
     result is attention() over them (no mask: the query follows every cached key).  A
     sequence with no keys gives O = 0 and LSE = -inf.  Returns (o [B,H,d], lse [B,H]).
     """
@@ -177,6 +177,37 @@ def paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, scale: fl
                            nthreads=nthreads, lib=lib)
         o[b] = ob[0, :, 0]
         lse[b] = lb[0, :, 0]
+    return o, lse
+
+
+def varlen_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: bool,
+                     nthreads: int = 0, lib=None):
+    """Attention over a batch of sequences of different lengths, packed token-major.
+
+    q: [total_q, H, d], k/v: [total_k, H, d]; sequence b owns query tokens
+    cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and key tokens cu_seqlens_k[b] ..
+    cu_seqlens_k[b+1]-1, and attends only to its own keys (causal alignment per sequence,
+    bottom-right as in attention()).  This is attention() applied sequence by sequence --
+    the "batch of independent problems" the pages tile over ("FlashAttention 1-2-3"
+    (myaihardware), section "When FlashAttention Doesn't Help": each query in the batch
+    processed independently).  Query tokens of a sequence with no keys, or fully masked,
+    get O = 0 and LSE = -inf.  Returns (o [total_q,H,d], lse [total_q,H]) in float64.
+    """
+    total_q, H, d = q.shape
+    o = np.zeros((total_q, H, d), dtype=np.float64)
+    lse = np.full((total_q, H), -np.inf, dtype=np.float64)
+    cq = [int(x) for x in cu_seqlens_q]
+    ck = [int(x) for x in cu_seqlens_k]
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0 or k1 == k0:
+            continue
+        qb = q[q0:q1].permute(1, 0, 2).reshape(1, H, q1 - q0, d).contiguous()
+        kb = k[k0:k1].permute(1, 0, 2).reshape(1, H, k1 - k0, d).contiguous()
+        vb = v[k0:k1].permute(1, 0, 2).reshape(1, H, k1 - k0, d).contiguous()
+        ob, lb = attention(qb, kb, vb, scale, causal, nthreads=nthreads, lib=lib)
+        o[q0:q1] = ob[0].transpose(1, 0, 2)
+        lse[q0:q1] = lb[0].T
     return o, lse
 
 

@@ -330,3 +330,54 @@ def test_paged_decode_pin_sees_a_wrong_page():
     o1, _ = oracle.paged_decode_attention(q, kc, vc, bt, [Lmax - 20], 1.0)
     o2, _ = oracle.paged_decode_attention(q, kc, vc, bt2, [Lmax - 20], 1.0)
     assert np.isfinite(o1).all() and not np.allclose(o1, o2, atol=1e-6)
+
+
+# ---------------------------------------------------------------- varlen (packed batches)
+def _pack(x):
+    """[B,H,L,d] -> token-major [B*L,H,d]."""
+    B, H, L, d = x.shape
+    return x.permute(0, 2, 1, 3).reshape(B * L, H, d).contiguous()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equal_lengths_is_the_batched_oracle(oracle_mod, causal):
+    """Equal lengths: the packed token-major batch gives attention() of the [B,H,L,d]
+    batch, row for row (pins the token-major indexing and the per-sequence split)."""
+    B, H, L, d = 3, 2, 50, 16
+    q, k, v = make_qkv(B, H, L, L, d, torch.float16, 600)
+    cu = [0, L, 2 * L, 3 * L]
+    o, lse = oracle_mod.varlen_attention(_pack(q), _pack(k), _pack(v), cu, cu, 0.4, causal)
+    o_ref, l_ref = oracle_mod.attention(q, k, v, 0.4, causal)
+    np.testing.assert_array_equal(o, o_ref.transpose(0, 2, 1, 3).reshape(B * L, H, d))
+    np.testing.assert_array_equal(lse, l_ref.transpose(0, 2, 1).reshape(B * L, H))
+
+
+def test_varlen_sequences_are_isolated(oracle_mod):
+    """Changing one sequence's keys and values changes only that sequence's rows; ragged
+    and empty sequences, Nq != Nkv with bottom-right causal alignment."""
+    H, d = 2, 16
+    lq, lk = [5, 0, 40, 7, 3], [9, 4, 40, 0, 12]
+    cq = np.concatenate([[0], np.cumsum(lq)]).tolist()
+    ck = np.concatenate([[0], np.cumsum(lk)]).tolist()
+    q = randn((cq[-1], H, d), 700, torch.bfloat16)
+    k = randn((ck[-1], H, d), 701, torch.bfloat16)
+    v = randn((ck[-1], H, d), 702, torch.bfloat16)
+    o1, l1 = oracle_mod.varlen_attention(q, k, v, cq, ck, 0.5, True)
+    k2, v2 = k.clone(), v.clone()
+    k2[ck[2]:ck[3]] = randn((lk[2], H, d), 703, torch.bfloat16)
+    v2[ck[2]:ck[3]] = randn((lk[2], H, d), 704, torch.bfloat16)
+    o2, l2 = oracle_mod.varlen_attention(q, k2, v2, cq, ck, 0.5, True)
+    other = np.r_[0:cq[2], cq[3]:cq[-1]]
+    np.testing.assert_array_equal(o1[other], o2[other])
+    np.testing.assert_array_equal(l1[other], l2[other])
+    assert not np.allclose(o1[cq[2]:cq[3]], o2[cq[2]:cq[3]])
+    # sequence 3 has no keys: O = 0, LSE = -inf
+    assert (o1[cq[3]:cq[4]] == 0).all() and np.isneginf(l1[cq[3]:cq[4]]).all()
+    # sequence 4: 3 queries, 12 keys, causal bottom-right: query i sees keys <= i + 9
+    qb = q[cq[4]:cq[5]].permute(1, 0, 2).reshape(1, H, 3, d)
+    kb = k[ck[4]:ck[5]].permute(1, 0, 2).reshape(1, H, 12, d)
+    vb = v[ck[4]:ck[5]].permute(1, 0, 2).reshape(1, H, 12, d)
+    s = torch.einsum("bhqd,bhkd->bhqk", qb.double(), kb.double()) * 0.5
+    s = s.masked_fill(torch.arange(12)[None, :] > torch.arange(3)[:, None] + 9, float("-inf"))
+    ref = torch.softmax(s, -1) @ vb.double()
+    np.testing.assert_allclose(o1[cq[4]:cq[5]], ref[0].permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
