@@ -41,6 +41,8 @@ _SIGNATURES = {
     "fa_fwd_prefill": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I, _I],
     "fa_fwd_decode": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
     "fa_fwd_decode_noalloc": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
+    "fa_fwd_varlen": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP,
+                      _I, _I],
     "fa_fwd_decode_paged": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP,
                             _I, _I, _I],
     "fa_decode_workspace_bytes": [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
@@ -107,6 +109,12 @@ def fa_fwd_decode_noalloc(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype
     instead of a cudaMalloc'd workspace, for callers that cannot allocate device memory."""
     return library().fa_fwd_decode_noalloc(q, k, v, o, lse, B, H, Nkv, d, scale, stream,
                                            in_dtype, o_dtype, num_splits)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q, max_k, d, scale,
+                  causal, stream, in_dtype, o_dtype) -> int:
+    return library().fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q,
+                                   max_k, d, scale, causal, stream, in_dtype, o_dtype)
 
 
 def fa_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, H, d, page_size,
@@ -228,4 +236,40 @@ def paged_decode(q, k_cache, v_cache, block_table, seq_lens, scale: Optional[flo
                                  _dtype_code(o.dtype), num_splits)
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd_decode_paged")
+    return o, lse
+
+
+def varlen_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                     causal: bool = False, scale: Optional[float] = None, out_dtype=None,
+                     stream=None):
+    """Attention over a packed batch: q [total_q,H,d], k/v [total_k,H,d] (fp16/bf16),
+    cu_seqlens_q/k int32 [B+1] -- all contiguous CUDA tensors.  Returns
+    (o [total_q,H,d], lse [total_q,H])."""
+    import torch
+
+    ts = (q, k, v, cu_seqlens_q, cu_seqlens_k)
+    if not all(t.is_cuda and t.is_contiguous() for t in ts):
+        raise ValueError("varlen_attention() takes contiguous CUDA tensors")
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise ValueError("cu_seqlens must be int32")
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    if tuple(k.shape) != (total_k, H, d) or tuple(v.shape) != (total_k, H, d):
+        raise ValueError("k and v must be [total_k, H, d] with q's H and d")
+    B = cu_seqlens_q.numel() - 1
+    if B < 1 or cu_seqlens_k.numel() != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B+1 entries")
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((total_q, H, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((total_q, H), dtype=torch.float32, device=q.device)
+    s = torch.cuda.current_stream(q.device) if stream is None else stream
+    with torch.cuda.device(q.device):
+        rc = fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q,
+                           total_k, int(max_seqlen_q), int(max_seqlen_k), d, scale,
+                           int(bool(causal)), s.cuda_stream, _dtype_code(q.dtype),
+                           _dtype_code(o.dtype))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_varlen")
     return o, lse

@@ -92,6 +92,22 @@ int make_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, bool
   return FA_OK;
 }
 
+// 3-D view (d, H, tokens) of a packed [tokens, H, d] tensor; box (64, 1, 128): the same
+// 128 rows x 128 B shared-memory tile as above, rows being tokens of one head.
+int make_map_packed(CUtensorMap* map, const void* ptr, long long tokens, int H, int d, bool bf16) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                        3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FA_OK;
+}
+
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
   return x < y + nb && y < x + na;
@@ -171,6 +187,8 @@ int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse
   const long long units = BH * p.n_pairs;
   if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
   p.n_units = static_cast<int>(units);
+  p.cu_q = p.cu_k = nullptr;
+  p.H = H;
   p.scale_log2 = scale_log2(scale);
   long long grid = num_ctas > 0 ? num_ctas : ds->sm_count;
   if (grid > units) grid = units;
@@ -179,6 +197,75 @@ int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse
                                      static_cast<int>(grid), ds->status,
                                      static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int run_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_q,
+               const int* cu_k, int B, int H, int total_q, int total_k, int max_q, int max_k,
+               int d, float scale, int causal, void* stream, int in_dtype, int o_dtype) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+  const bool bf16 = in_dtype == FA_BF16;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map_packed(&tq, q, total_q, H, d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map_packed(&tk, k, total_k, H, d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map_packed(&tv, v, total_k, H, d, bf16)) != FA_OK) return rc;
+  fa::PrefillParams p{};
+  p.BH = B * H;
+  p.Nq = max_q;
+  p.Nkv = max_k;
+  p.off = 0;  // per sequence in the kernel
+  p.causal = causal;
+  p.n_qtiles = (max_q + 127) / 128;
+  p.n_pairs = (p.n_qtiles + 1) / 2;
+  p.n_kvtiles = (max_k + 127) / 128;
+  const long long units = static_cast<long long>(p.BH) * p.n_pairs;
+  if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  p.n_units = static_cast<int>(units);
+  p.scale_log2 = scale_log2(scale);
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.H = H;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  long long grid = ds->sm_count;
+  if (grid > units) grid = units;
+  if (grid < 1) grid = 1;
+  cudaError_t e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, bf16, o_dtype == FA_F32,
+                                     static_cast<int>(grid), ds->status,
+                                     static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int check_varlen_args(const void* q, const void* k, const void* v, void* o, float* lse,
+                      const int* cu_q, const int* cu_k, int B, int H, int total_q, int total_k,
+                      int max_q, int max_k, int d, float scale, int causal, int in_dtype,
+                      int o_dtype) {
+  if (!q || !k || !v || !o || !cu_q || !cu_k) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || total_q < 1 || total_k < 1 || max_q < 1 || max_k < 1) return FA_ERR_INVALID_ARG;
+  if (max_q > total_q || max_k > total_k) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (in_dtype != FA_F16 && in_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_F16 && o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_F32 && o_dtype != in_dtype) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return FA_ERR_INVALID_ARG;
+  if (!aligned(cu_q, 4) || !aligned(cu_k, 4) || (lse && !aligned(lse, 4))) return FA_ERR_INVALID_ARG;
+  const size_t qb = static_cast<size_t>(total_q) * H * d * 2;
+  const size_t kb = static_cast<size_t>(total_k) * H * d * 2;
+  const size_t ob = static_cast<size_t>(total_q) * H * d * (o_dtype == FA_F32 ? 4 : 2);
+  const size_t lb = static_cast<size_t>(total_q) * H * 4, cb = static_cast<size_t>(B + 1) * 4;
+  const void* ins[5] = {q, k, v, cu_q, cu_k};
+  const size_t in_bytes[5] = {qb, kb, kb, cb, cb};
+  for (int i = 0; i < 5; ++i) {
+    if (overlaps(o, ob, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+    if (lse && overlaps(lse, lb, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+  }
+  if (lse && overlaps(lse, lb, o, ob)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
 }
 
 int run_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -285,6 +372,18 @@ int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* l
   if (rc != FA_OK) return rc;
   if (num_splits < 0) return FA_ERR_INVALID_ARG;
   return run_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype, num_splits);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int total_q,
+                  int total_k, int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal,
+                  void* stream, int in_dtype, int o_dtype) {
+  const int rc = check_varlen_args(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q,
+                                   total_k, max_seqlen_q, max_seqlen_k, d, scale, causal,
+                                   in_dtype, o_dtype);
+  if (rc != FA_OK) return rc;
+  return run_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k,
+                    max_seqlen_q, max_seqlen_k, d, scale, causal, stream, in_dtype, o_dtype);
 }
 
 int fa_fwd_decode_paged(const void* q, const void* k_cache, const void* v_cache,

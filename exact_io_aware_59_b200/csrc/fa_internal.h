@@ -18,6 +18,13 @@ struct PrefillParams {
   int n_kvtiles;    // ceil(Nkv / 128)
   int n_units;      // BH * n_pairs
   float scale_log2; // scale * log2(e)
+  // Packed variable-length batches (null cu_q: the [B,H,N,d] layout above).  Then
+  // Nq / Nkv are the longest query / key sequences, q/o are [total_q, H, d], k/v
+  // [total_k, H, d], and sequence b owns tokens cu[b] .. cu[b+1]-1.
+  const int* cu_q;
+  const int* cu_k;
+  int H;            // heads per sequence (bh = b * H + h)
+  int total_q, total_k;
 };
 
 // Work description of one split-KV decode launch.

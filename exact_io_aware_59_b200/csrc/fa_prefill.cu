@@ -92,14 +92,69 @@ __device__ __forceinline__ int unit_of_round(int r) {
   return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
-// Number of K/V tiles Q tile `qtile` must visit (0 when every row is fully masked).
-__device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, int qtile) {
-  if (qtile >= p.n_qtiles) return 0;
-  if (!p.causal) return p.n_kvtiles;
-  const int last_row = min(qtile * BM + BM - 1, p.Nq - 1);
-  const int last_key = last_row + p.off;
+// One work unit: its (b*H + h, Q-tile pair) and the sequence it belongs to.  For a packed
+// variable-length batch the sequence's token ranges come from cu_q / cu_k, which live
+// on the device: a range outside [0, total] or longer than the longest sequence the
+// caller declared is clamped and, when `flag`, reported in the status word.
+struct Unit {
+  int bh, pair;
+  int Lq, Lk;  // queries and keys of the sequence
+  int q0, k0;  // first query / key token of the sequence (packed layout)
+  int h;       // head within the sequence (packed layout)
+};
+
+__device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u, int* status, bool flag) {
+  Unit x;
+  unit_coords(p, u, x.bh, x.pair);
+  if (p.cu_q == nullptr) {
+    x.Lq = p.Nq;
+    x.Lk = p.Nkv;
+    x.q0 = x.k0 = x.h = 0;
+    return x;
+  }
+  const int b = x.bh / p.H;
+  x.h = x.bh % p.H;
+  int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+  const bool bad = q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
+                   k1 > p.total_k || k1 - k0 > p.Nkv;
+  if (bad) {
+    if (flag) atomicOr(status, kStatusBadInput);
+    q0 = min(max(q0, 0), p.total_q);
+    q1 = min(max(q1, q0), min(p.total_q, q0 + p.Nq));
+    k0 = min(max(k0, 0), p.total_k);
+    k1 = min(max(k1, k0), min(p.total_k, k0 + p.Nkv));
+  }
+  x.q0 = q0;
+  x.Lq = q1 - q0;
+  x.k0 = k0;
+  x.Lk = k1 - k0;
+  return x;
+}
+
+// Number of K/V tiles Q tile `qtile` of unit x must visit (0 when every row is fully
+// masked or the tile lies past the sequence's queries).
+__device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, const Unit& x, int qtile) {
+  if (qtile * BM >= x.Lq) return 0;
+  const int ntk = (x.Lk + BN - 1) / BN;
+  if (!p.causal) return ntk;
+  const int last_row = min(qtile * BM + BM - 1, x.Lq - 1);
+  const int last_key = last_row + x.Lk - x.Lq;  // bottom-right alignment per sequence
   if (last_key < 0) return 0;
-  return min(p.n_kvtiles, last_key / BN + 1);
+  return min(ntk, last_key / BN + 1);
+}
+
+// TMA coordinates (beyond the 64-column block) of the tile whose first row is `first`
+// (a query row or a key row of the unit's sequence): (row, b*H + h) in the [B,H,N,d]
+// view, (h, token) in the packed [tokens, H, d] view.
+__device__ __forceinline__ void tile_coords(const PrefillParams& p, const Unit& x, int first,
+                                            bool query, int& c1, int& c2) {
+  if (p.cu_q == nullptr) {
+    c1 = first;
+    c2 = x.bh;
+  } else {
+    c1 = x.h;
+    c2 = (query ? x.q0 : x.k0) + first;
+  }
 }
 
 // Waits for TMA loads already issued, ignoring the abort flag (error path only).
@@ -120,9 +175,9 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
   uint32_t ld = 0, q_issued = 0;
   bool ok = true;
   for (int rnd = 0, u = unit_of_round(0); u < p.n_units && ok; u = unit_of_round(++rnd)) {
-    int bh, pair;
-    unit_coords(p, u, bh, pair);
-    const int n0 = kv_tiles_for(p, 2 * pair), n1 = kv_tiles_for(p, 2 * pair + 1);
+    const Unit x = unit_of(p, u, status, true);
+    const int pair = x.pair;
+    const int n0 = kv_tiles_for(p, x, 2 * pair), n1 = kv_tiles_for(p, x, 2 * pair + 1);
     const int nmax = max(n0, n1);
     if (nmax == 0) continue;
     if (!mbar_wait(bar_addr(bars, C::kBarQEmpty), (q_issued & 1) ^ 1, status, abort_flag,
@@ -135,10 +190,11 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       if ((t == 0 ? n0 : n1) == 0) continue;
+      int c1, c2;
+      tile_coords(p, x, (2 * pair + t) * BM, true, c1, c2);
 #pragma unroll
       for (int sub = 0; sub < D / 64; ++sub)
-        tma_load_3d(sbase + C::kQOff + t * C::kQBytes + sub * BM * 128, tq, qf, sub * 64,
-                    (2 * pair + t) * BM, bh);
+        tma_load_3d(sbase + C::kQOff + t * C::kQBytes + sub * BM * 128, tq, qf, sub * 64, c1, c2);
     }
     ++q_issued;
     for (int j = 0; j < nmax && ok; ++j) {
@@ -153,9 +209,11 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
         const uint32_t fb = bar_addr(bars, C::kBarFull + slot);
         mbar_arrive_expect_tx(fb, C::kKVBytes);
         const uint32_t dst = sbase + C::kRingOff + slot * C::kKVBytes;
+        int c1, c2;
+        tile_coords(p, x, j * BN, false, c1, c2);
 #pragma unroll
         for (int sub = 0; sub < D / 64; ++sub)
-          tma_load_3d(dst + sub * BN * 128, which ? tv : tk, fb, sub * 64, j * BN, bh);
+          tma_load_3d(dst + sub * BN * 128, which ? tv : tk, fb, sub * 64, c1, c2);
         ++ld;
       }
     }
@@ -215,9 +273,8 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
     return mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutMma);
   };
   for (int rnd = 0, u = unit_of_round(0); u < p.n_units && ok; u = unit_of_round(++rnd)) {
-    int bh, pair;
-    unit_coords(p, u, bh, pair);
-    const int n[2] = {kv_tiles_for(p, 2 * pair), kv_tiles_for(p, 2 * pair + 1)};
+    const Unit x = unit_of(p, u, status, false);
+    const int n[2] = {kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)};
     const int nmax = max(n[0], n[1]);
     if (nmax == 0) continue;
     if (!wait(C::kBarQFull, q_used & 1)) { ok = false; break; }
@@ -359,14 +416,14 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   };
 
   for (int rnd = 0, u = unit_of_round(0); u < p.n_units; u = unit_of_round(++rnd)) {
-    int bh, pair;
-    unit_coords(p, u, bh, pair);
-    const int qtile = 2 * pair + t;
-    if (qtile >= p.n_qtiles) continue;
-    const int n_kv = kv_tiles_for(p, qtile);
+    const Unit x = unit_of(p, u, status, false);
+    const int qtile = 2 * x.pair + t;
+    if (qtile * BM >= x.Lq) continue;
+    const int n_kv = kv_tiles_for(p, x, qtile);
     const int row = qtile * BM + r;
-    // Last key this row may see (keys beyond Nkv are padding of the last tile).
-    const int limit = p.causal ? min(p.Nkv - 1, row + p.off) : p.Nkv - 1;
+    // Last key this row may see (keys beyond the sequence's are padding of its last tile,
+    // or the next sequence's in a packed batch).
+    const int limit = p.causal ? min(x.Lk - 1, row + x.Lk - x.Lq) : x.Lk - 1;
     float m_used = -INFINITY;  // running max in log2 units (may lag the true max by <= 8)
     float l = 0.f;             // running sum of the 16-bit-rounded 2^(x - m_used): divides O
     float l_exact = 0.f;       // the same sum before rounding: gives LSE
@@ -497,9 +554,13 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
       tc_fence_after();
       o_seen += n_kv;
     }
-    const bool valid = row < p.Nq;
+    const bool valid = row < x.Lq;
+    // Output row: (b*H + h, row) in [B,H,Nq,d]; (token, h) in the packed [tokens, H, d].
+    const size_t orow_i = p.cu_q == nullptr
+                              ? static_cast<size_t>(x.bh) * p.Nq + row
+                              : (static_cast<size_t>(x.q0) + row) * p.H + x.h;
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
-    const size_t orow = (static_cast<size_t>(bh) * p.Nq + row) * D;
+    const size_t orow = orow_i * D;
 #pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t ob[32];
@@ -532,7 +593,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
       }
     }
     if (valid && lse != nullptr)
-      lse[static_cast<size_t>(bh) * p.Nq + row] =
+      lse[orow_i] =
           (l_exact > 0.f) ? (m_used + log2f(l_exact)) * 0.69314718055994531f : -INFINITY;
   }
 }

@@ -137,6 +137,29 @@ int fa_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* o, 
                           int in_dtype, int o_dtype, int num_splits);
 
 /*
+ * fa_fwd_varlen -- prefill over a packed batch of sequences of different lengths
+ * ("FlashAttention 1-2-3" (myaihardware), section "When FlashAttention Doesn't Help":
+ * continuous batching, each sequence of the batch an independent problem).
+ *   q [total_q, H, d], k/v [total_k, H, d] (token-major, fp16/bf16), o [total_q, H, d]
+ *   (fp32 or q's 16-bit type), lse [total_q, H] fp32 (may be NULL).
+ *   cu_seqlens_q / cu_seqlens_k: int32 [B+1] device arrays, non-decreasing, starting at
+ *   0 and ending at total_q / total_k: sequence b owns query tokens cu_seqlens_q[b] ..
+ *   cu_seqlens_q[b+1]-1 and key tokens likewise, and attends to its own keys only
+ *   (causal mask aligned bottom-right per sequence, as for fa_fwd).  max_seqlen_q /
+ *   max_seqlen_k bound every sequence's length (they size the work).  A query token
+ *   whose sequence has no visible key gets O = 0 and LSE = -inf.
+ *   All pointers are device memory owned by the caller, valid until the work completes;
+ *   q, k, v, o 16-byte aligned, the rest 4-byte.
+ *   Errors: FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED for what the host can check (nothing
+ *   is enqueued).  The offsets live on the device: a range outside [0, total] or longer
+ *   than its max_seqlen is clamped and FA_DEV_BAD_INPUT is set in the status word.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int H, int total_q,
+                  int total_k, int max_seqlen_q, int max_seqlen_k, int d, float scale, int causal,
+                  void* stream, int in_dtype, int o_dtype);
+
+/*
  * fa_fwd_decode_paged -- split-KV decode for one query per head against a paged KV cache
  * ("FlashAttention 1-2-3" (myaihardware), section "Integration in Major Inference
  * Engines": each KV-cache page of vLLM's PagedAttention is a block the kernel tiles over;
@@ -182,7 +205,7 @@ enum {
   FA_DEV_TIMEOUT_MMA = 2,       /* prefill: the MMA issuer's wait ran out */
   FA_DEV_TIMEOUT_SOFTMAX = 4,   /* prefill: a softmax / epilogue wait ran out */
   FA_DEV_TIMEOUT_DECODE = 8,    /* decode: a split kernel wait ran out */
-  FA_DEV_BAD_INPUT = 16         /* paged decode: a block-table entry or length out of range */
+  FA_DEV_BAD_INPUT = 16         /* paged decode / varlen: a device-side table or offset out of range */
 };
 
 /*

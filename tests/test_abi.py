@@ -142,3 +142,29 @@ def _paged(**kw):
 ])
 def test_paged_decode_argument_checks(kw, code):
     assert _paged(**kw) == code
+
+
+def _varlen(**kw):
+    a = dict(q=Q, k=K, v=V, o=O, lse=L, cq=L + 4096, ck=L + 8192, B=2, H=2, tq=100, tk=100,
+             mq=60, mk=60, d=64, scale=0.1, causal=1, stream=None, in_dtype=0, o_dtype=2)
+    a.update(kw)
+    return binding.fa_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cq"], a["ck"],
+                                 a["B"], a["H"], a["tq"], a["tk"], a["mq"], a["mk"], a["d"],
+                                 a["scale"], a["causal"], a["stream"], a["in_dtype"],
+                                 a["o_dtype"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cq=None), binding.FA_ERR_INVALID_ARG),
+    (dict(ck=None), binding.FA_ERR_INVALID_ARG),
+    (dict(B=0), binding.FA_ERR_INVALID_ARG),
+    (dict(tq=0), binding.FA_ERR_INVALID_ARG),
+    (dict(mk=0), binding.FA_ERR_INVALID_ARG),
+    (dict(mq=101), binding.FA_ERR_INVALID_ARG),        # longer than the whole batch
+    (dict(causal=3), binding.FA_ERR_INVALID_ARG),
+    (dict(cq=L + 4098), binding.FA_ERR_INVALID_ARG),   # misaligned int32 offsets
+    (dict(d=32), binding.FA_ERR_UNSUPPORTED),
+    (dict(o=Q), binding.FA_ERR_INVALID_ARG),           # O on Q
+])
+def test_varlen_argument_checks(kw, code):
+    assert _varlen(**kw) == code
