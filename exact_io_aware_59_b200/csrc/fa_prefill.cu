@@ -103,32 +103,34 @@ struct Unit {
   int h;       // head within the sequence (packed layout)
 };
 
+template <bool VARLEN>
 __device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u, int* status, bool flag) {
   Unit x;
   unit_coords(p, u, x.bh, x.pair);
-  if (p.cu_q == nullptr) {
+  if constexpr (!VARLEN) {
     x.Lq = p.Nq;
     x.Lk = p.Nkv;
     x.q0 = x.k0 = x.h = 0;
     return x;
+  } else {
+    const int b = x.bh / p.H;
+    x.h = x.bh % p.H;
+    int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+    const bool bad = q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
+                     k1 > p.total_k || k1 - k0 > p.Nkv;
+    if (bad) {
+      if (flag) atomicOr(status, kStatusBadInput);
+      q0 = min(max(q0, 0), p.total_q);
+      q1 = min(max(q1, q0), min(p.total_q, q0 + p.Nq));
+      k0 = min(max(k0, 0), p.total_k);
+      k1 = min(max(k1, k0), min(p.total_k, k0 + p.Nkv));
+    }
+    x.q0 = q0;
+    x.Lq = q1 - q0;
+    x.k0 = k0;
+    x.Lk = k1 - k0;
+    return x;
   }
-  const int b = x.bh / p.H;
-  x.h = x.bh % p.H;
-  int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
-  const bool bad = q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
-                   k1 > p.total_k || k1 - k0 > p.Nkv;
-  if (bad) {
-    if (flag) atomicOr(status, kStatusBadInput);
-    q0 = min(max(q0, 0), p.total_q);
-    q1 = min(max(q1, q0), min(p.total_q, q0 + p.Nq));
-    k0 = min(max(k0, 0), p.total_k);
-    k1 = min(max(k1, k0), min(p.total_k, k0 + p.Nkv));
-  }
-  x.q0 = q0;
-  x.Lq = q1 - q0;
-  x.k0 = k0;
-  x.Lk = k1 - k0;
-  return x;
 }
 
 // Number of K/V tiles Q tile `qtile` of unit x must visit (0 when every row is fully
@@ -146,9 +148,10 @@ __device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, const Unit& 
 // TMA coordinates (beyond the 64-column block) of the tile whose first row is `first`
 // (a query row or a key row of the unit's sequence): (row, b*H + h) in the [B,H,N,d]
 // view, (h, token) in the packed [tokens, H, d] view.
+template <bool VARLEN>
 __device__ __forceinline__ void tile_coords(const PrefillParams& p, const Unit& x, int first,
                                             bool query, int& c1, int& c2) {
-  if (p.cu_q == nullptr) {
+  if constexpr (!VARLEN) {
     c1 = first;
     c2 = x.bh;
   } else {
@@ -166,7 +169,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- producer (TMA)
-template <int D>
+template <int D, bool VARLEN>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                          const PrefillParams& p, uint32_t sbase, uint32_t bars, int* status,
                          volatile int* abort_flag) {
@@ -175,7 +178,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
   uint32_t ld = 0, q_issued = 0;
   bool ok = true;
   for (int rnd = 0, u = unit_of_round(0); u < p.n_units && ok; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of(p, u, status, true);
+    const Unit x = unit_of<VARLEN>(p, u, status, true);
     const int pair = x.pair;
     const int n0 = kv_tiles_for(p, x, 2 * pair), n1 = kv_tiles_for(p, x, 2 * pair + 1);
     const int nmax = max(n0, n1);
@@ -191,7 +194,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     for (int t = 0; t < 2; ++t) {
       if ((t == 0 ? n0 : n1) == 0) continue;
       int c1, c2;
-      tile_coords(p, x, (2 * pair + t) * BM, true, c1, c2);
+      tile_coords<VARLEN>(p, x, (2 * pair + t) * BM, true, c1, c2);
 #pragma unroll
       for (int sub = 0; sub < D / 64; ++sub)
         tma_load_3d(sbase + C::kQOff + t * C::kQBytes + sub * BM * 128, tq, qf, sub * 64, c1, c2);
@@ -210,7 +213,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
         mbar_arrive_expect_tx(fb, C::kKVBytes);
         const uint32_t dst = sbase + C::kRingOff + slot * C::kKVBytes;
         int c1, c2;
-        tile_coords(p, x, j * BN, false, c1, c2);
+        tile_coords<VARLEN>(p, x, j * BN, false, c1, c2);
 #pragma unroll
         for (int sub = 0; sub < D / 64; ++sub)
           tma_load_3d(dst + sub * BN * 128, which ? tv : tk, fb, sub * 64, c1, c2);
@@ -254,7 +257,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint6
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool VARLEN>
 __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                            int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -273,7 +276,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
     return mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutMma);
   };
   for (int rnd = 0, u = unit_of_round(0); u < p.n_units && ok; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of(p, u, status, false);
+    const Unit x = unit_of<VARLEN>(p, u, status, false);
     const int n[2] = {kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)};
     const int nmax = max(n[0], n[1]);
     if (nmax == 0) continue;
@@ -395,7 +398,7 @@ __device__ __forceinline__ void exp_pack_store32(const uint32_t (&s)[32], uint64
 }
 
 // NEG: the scale is negative, so the row maximum of scale * s comes from the minimum of s.
-template <int D, bool BF16, bool OF32, bool NEG>
+template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN>
 __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t tmem, void* o,
                                  float* lse, int t, int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -416,7 +419,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   };
 
   for (int rnd = 0, u = unit_of_round(0); u < p.n_units; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of(p, u, status, false);
+    const Unit x = unit_of<VARLEN>(p, u, status, false);
     const int qtile = 2 * x.pair + t;
     if (qtile * BM >= x.Lq) continue;
     const int n_kv = kv_tiles_for(p, x, qtile);
@@ -556,9 +559,8 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     }
     const bool valid = row < x.Lq;
     // Output row: (b*H + h, row) in [B,H,Nq,d]; (token, h) in the packed [tokens, H, d].
-    const size_t orow_i = p.cu_q == nullptr
-                              ? static_cast<size_t>(x.bh) * p.Nq + row
-                              : (static_cast<size_t>(x.q0) + row) * p.H + x.h;
+    const size_t orow_i = !VARLEN ? static_cast<size_t>(x.bh) * p.Nq + row
+                                  : (static_cast<size_t>(x.q0) + row) * p.H + x.h;
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
     const size_t orow = orow_i * D;
 #pragma unroll 1
@@ -598,7 +600,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   }
 }
 
-template <int D, bool BF16, bool OF32>
+template <int D, bool BF16, bool OF32, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_prefill_sm100(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, void* __restrict__ o,
@@ -649,9 +651,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
     if (warp == 0) {
-      if (lane == 0) producer<D>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
+      if (lane == 0) producer<D, VARLEN>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D, BF16>(p, sbase, bars, tmem, status, abort_flag);
+      if (lane == 0) mma_issuer<D, BF16, VARLEN>(p, sbase, bars, tmem, status, abort_flag);
       __syncwarp();
       // Release TMEM once both softmax warpgroups have finished reading it.
       drain_wait(bar_addr(bars, C::kBarDone), 0);
@@ -662,19 +664,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     if (p.scale_log2 < 0.f)
-      softmax_epilogue<D, BF16, OF32, true>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, true, VARLEN>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     else
-      softmax_epilogue<D, BF16, OF32, false>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, false, VARLEN>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     tc_fence_before();
     mbar_arrive(bar_addr(bars, C::kBarDone));
   }
 }
 
-template <int D, bool BF16, bool OF32>
+template <int D, bool BF16, bool OF32, bool VARLEN>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                      float* lse, const PrefillParams& p, int grid, int* status,
                      cudaStream_t stream) {
-  auto kern = fa_prefill_sm100<D, BF16, OF32>;
+  auto kern = fa_prefill_sm100<D, BF16, OF32, VARLEN>;
   static bool configured = false;  // per template instance
   static cudaError_t config_err = cudaSuccess;
   if (!configured) {
@@ -703,8 +705,10 @@ size_t prefill_smem_bytes(int d) {
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            void* o, float* lse, const PrefillParams& p, int d, bool bf16,
                            bool o_f32, int grid, int* status, cudaStream_t stream) {
-#define FA_PREFILL_CASE(D_, B_, F_) \
-  if (d == D_ && bf16 == B_ && o_f32 == F_) return launch_t<D_, B_, F_>(tq, tk, tv, o, lse, p, grid, status, stream);
+#define FA_PREFILL_CASE(D_, B_, F_)                                                          \
+  if (d == D_ && bf16 == B_ && o_f32 == F_)                                                   \
+    return p.cu_q ? launch_t<D_, B_, F_, true>(tq, tk, tv, o, lse, p, grid, status, stream)   \
+                  : launch_t<D_, B_, F_, false>(tq, tk, tv, o, lse, p, grid, status, stream);
   FA_PREFILL_CASE(128, true, true)
   FA_PREFILL_CASE(128, true, false)
   FA_PREFILL_CASE(128, false, true)
