@@ -7,7 +7,10 @@ One step = one pass of the hot path over one batch of synthetic input:
     bf16), one fa_fwd call (split kernel + combine kernel) per step;
   * the "decode_paged" object times the same decode against a paged KV cache (64-key
     pages scattered over the pool by a seeded random block table), one
-    fa_fwd_decode_paged call per step.
+    fa_fwd_decode_paged call per step;
+  * the "prefill_varlen" object times a packed ragged causal batch (16 sequences,
+    seeded log-uniform lengths in [512, 8192], H=32, d=128, bf16), one fa_fwd_varlen
+    call per step.
 Inputs are resident in HBM and larger than L2 (126 MB) when the timed region starts.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -35,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 from exact_io_aware_59_b200 import binding  # noqa: E402
 from exact_io_aware_59_b200.inputs import (WORKLOADS, Workload, paged_decode_inputs,  # noqa: E402
-                                           workload_qkv)
+                                           varlen_inputs, varlen_lengths, workload_qkv)
 
 METRIC = "attention fwd TFLOP/s at 1 B200 (% of dense bf16 peak); decode HBM GB/s"
 PREFILL = "long_prefill_causal"
@@ -362,6 +365,41 @@ def arm_ours(args, ws, rank, local):
         }
         torch.cuda.empty_cache()
 
+    # packed variable-length prefill: a ragged causal batch
+    prefill_varlen = None
+    if not args.skip_decode:
+        lens = varlen_lengths(16, 512, 8192, 4242)
+        Hv, dv = 32, 128
+        vq, vk, vv, vcu = varlen_inputs(lens, Hv, dv, torch.bfloat16, 8000, device="cuda")
+        vo = torch.empty_like(vq)
+        vlse = torch.empty((vq.shape[0], Hv), dtype=torch.float32, device="cuda")
+        vargs = (vq.data_ptr(), vk.data_ptr(), vv.data_ptr(), vo.data_ptr(), vlse.data_ptr(),
+                 vcu.data_ptr(), vcu.data_ptr(), len(lens), Hv, vq.shape[0], vk.shape[0],
+                 max(lens), max(lens), dv, float(dv ** -0.5), 1, stream.cuda_stream,
+                 binding.FA_BF16, binding.FA_BF16)
+
+        def varlen_call():
+            check(binding.fa_fwd_varlen(*vargs), "fa_fwd_varlen")
+
+        vsteps = max(3, args.steps // 4)
+        with ClockSampler(local) as clk_v, torch.cuda.stream(stream):
+            ms_v = time_steps(varlen_call, vsteps, args.warmup, ws, stream)
+        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+        flops_v = sum(4 * dv * Hv * causal_pairs(n, n) for n in lens)
+        tf_v = flops_v / (ms_v * 1e-3) / 1e12
+        prefill_varlen = {
+            "workload": f"packed causal batch of {len(lens)} sequences, {sum(lens)} tokens "
+                        f"(lengths log-uniform in [512, 8192], seeded), H={Hv} d={dv} bf16",
+            "value": whole_job_rate(flops_v, ms_v, ws) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms_v, "steps": vsteps, "gpu_launches": vsteps,
+            "roofline": {"bound": "tensor", "achieved": tf_v, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": tf_v / peak_t, "traffic": None, "peak_source": peak_src,
+                         "flops_per_launch": flops_v},
+            "clocks": clk_v.summary(),
+        }
+        del vq, vk, vv, vcu, vo, vlse
+        torch.cuda.empty_cache()
+
     # decode against a paged KV cache (same shape as the decode workload)
     decode_paged = None
     if not args.skip_decode:
@@ -430,6 +468,7 @@ def arm_ours(args, ws, rank, local):
             "clocks": clk.summary(),
             "decode": decode,
             "decode_paged": decode_paged,
+            "prefill_varlen": prefill_varlen,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
@@ -437,7 +476,7 @@ def arm_ours(args, ws, rank, local):
 
 
 # Bumped whenever the prefill kernel changes, so stale ncu traffic is not reported.
-KERNEL_REV = "prefill-v19"
+KERNEL_REV = "prefill-v21"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the
 # kernel at this revision (profiles/fa_prefill_sm100_<workload>.md).
 DRAM_TRAFFIC = {("prefill-v19", "long_prefill_causal"): 588.0e6}

@@ -103,3 +103,26 @@ def paged_decode_inputs(B: int, H: int, L: int, d: int, page_size: int, dtype: t
     table = torch.randperm(B * P, generator=g, device=device).to(torch.int32).reshape(B, P)
     seq_lens = torch.full((B,), L, dtype=torch.int32, device=device)
     return q, k_cache, v_cache, table.contiguous(), seq_lens
+
+
+def varlen_lengths(n: int, lo: int, hi: int, seed: int):
+    """n sequence lengths drawn log-uniformly from [lo, hi] with a seeded generator (a
+    mix of short and long requests, as in a continuously batched prefill)."""
+    g = torch.Generator()
+    g.manual_seed(int(seed))
+    u = torch.rand(n, generator=g, dtype=torch.float64)
+    import math
+    return [int(round(math.exp(math.log(lo) + float(x) * (math.log(hi) - math.log(lo))))) for x in u]
+
+
+def varlen_inputs(lengths, H: int, d: int, dtype: torch.dtype, seed_base: int, device="cpu"):
+    """A packed batch: q, k, v [sum(lengths), H, d] iid N(0,1) rounded to `dtype` (seeds
+    seed_base + 0, 1, 2) and cu_seqlens int32 [len(lengths)+1]."""
+    total = int(sum(lengths))
+    q = randn((total, H, d), seed_base + 0, dtype, 1.0, device)
+    k = randn((total, H, d), seed_base + 1, dtype, 1.0, device)
+    v = randn((total, H, d), seed_base + 2, dtype, 1.0, device)
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    return q, k, v, torch.tensor(cu, dtype=torch.int32, device=device)
