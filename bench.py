@@ -479,7 +479,7 @@ def arm_ours(args, ws, rank, local):
 KERNEL_REV = "prefill-v21"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the
 # kernel at this revision (profiles/fa_prefill_sm100_<workload>.md).
-DRAM_TRAFFIC = {("prefill-v19", "long_prefill_causal"): 588.0e6}
+DRAM_TRAFFIC = {("prefill-v21", "long_prefill_causal"): 581.4e6}
 # The decode kernel's traffic per launch, taken on decode_4k (B16 H32 Nkv4096: 1.0816 GB)
 # and scaled by the keys streamed (x8 for Nkv 32768): the kernel reads each key once.
 DECODE_REV = "decode-v1"
