@@ -211,6 +211,41 @@ def varlen_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, scale: float, causal: 
     return o, lse
 
 
+def e4m3_to_f64(bits):
+    """Values of FP8 E4M3 codes (uint8 array or tensor): sign bit, 4 exponent bits with
+    bias 7, 3 mantissa bits; exponent 0 is subnormal (m * 2^-9); S.1111.111 is NaN and
+    there is no infinity (the "fn" variant used for FP8 tensor-core inputs).  Returns
+    numpy float64."""
+    try:
+        import torch
+        if isinstance(bits, torch.Tensor):
+            bits = bits.detach().cpu().view(torch.uint8).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    out = sign * mag
+    return np.where((e == 15) & ((b & 7) == 7), np.nan, out)
+
+
+def fp8_qk_attention(q8, k8, v, q_scale: float, k_scale: float, scale: float, causal: bool,
+                     rows=None, nthreads: int = 0, lib=None):
+    """Attention with FP8 queries and keys ("FlashAttention 1-2-3" (myaihardware), section
+    "FlashAttention-3: FP8, Async Warp Overlap, and Hopper-Specific Optimizations": FP8
+    tensor-core inputs).  q8 [B,H,Nq,d] and k8 [B,H,Nkv,d] hold E4M3
+    codes; the tensors they stand for are q_scale * decode(q8) and k_scale * decode(k8)
+    (per-tensor scales).  v [B,H,Nkv,d] in its own type.  The result is attention() of
+    those values in fp64, same layout and conventions."""
+    import torch
+    qf = torch.from_numpy(e4m3_to_f64(q8) * float(q_scale))
+    kf = torch.from_numpy(e4m3_to_f64(k8) * float(k_scale))
+    vf = torch.as_tensor(v).detach().cpu().to(torch.float64)
+    return attention(qf, kf, vf, scale, causal, rows=rows, nthreads=nthreads, lib=lib)
+
+
 def _f64(x):
     try:
         import torch

@@ -381,3 +381,36 @@ def test_varlen_sequences_are_isolated(oracle_mod):
     s = s.masked_fill(torch.arange(12)[None, :] > torch.arange(3)[:, None] + 9, float("-inf"))
     ref = torch.softmax(s, -1) @ vb.double()
     np.testing.assert_allclose(o1[cq[4]:cq[5]], ref[0].permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) queries and keys
+def test_e4m3_decode_matches_torch_for_every_code(oracle_mod):
+    """All 256 E4M3 codes decode to the values of torch.float8_e4m3fn (a library
+    routine), NaN codes included."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ours = oracle_mod.e4m3_to_f64(codes)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref)) and np.isnan(ours).sum() == 2
+    fin = ~np.isnan(ref)
+    np.testing.assert_array_equal(ours[fin], ref[fin])
+    assert ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9 and ours[0x38] == 1.0
+
+
+def test_fp8_attention_is_attention_of_the_dequantised_tensors(oracle_mod):
+    """The FP8 reference equals attention() on q_scale * Q and k_scale * K given as fp64,
+    and the scales act as one factor on the scores (q_scale*k_scale*scale fixed)."""
+    B, H, N, d = 1, 2, 40, 32
+    qf = randn((B, H, N, d), 800, torch.float32, 3.0)
+    kf = randn((B, H, N, d), 801, torch.float32, 3.0)
+    v = randn((B, H, N, d), 802, torch.bfloat16)
+    q8 = qf.to(torch.float8_e4m3fn).view(torch.uint8)
+    k8 = kf.to(torch.float8_e4m3fn).view(torch.uint8)
+    o, lse = oracle_mod.fp8_qk_attention(q8, k8, v, 0.5, 0.25, 0.1, True)
+    qd = q8.view(torch.float8_e4m3fn).to(torch.float64) * 0.5
+    kd = k8.view(torch.float8_e4m3fn).to(torch.float64) * 0.25
+    o_ref, l_ref = oracle_mod.attention(qd, kd, v.to(torch.float64), 0.1, True)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(lse, l_ref)
+    o2, l2 = oracle_mod.fp8_qk_attention(q8, k8, v, 1.0, 1.0, 0.1 * 0.5 * 0.25, True)
+    np.testing.assert_allclose(o2, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2, lse, rtol=0, atol=1e-12)
