@@ -8,6 +8,8 @@ One step = one pass of the hot path over one batch of synthetic input:
   * the "decode_paged" object times the same decode against a paged KV cache (64-key
     pages scattered over the pool by a seeded random block table), one
     fa_fwd_decode_paged call per step;
+  * the "prefill_fp8" object times the headline shape with Q and K in E4M3, one
+    fa_fwd_fp8 call per step;
   * the "prefill_varlen" object times a packed ragged causal batch (16 sequences,
     seeded log-uniform lengths in [512, 8192], H=32, d=128, bf16), one fa_fwd_varlen
     call per step.
@@ -365,6 +367,46 @@ def arm_ours(args, ws, rank, local):
         }
         torch.cuda.empty_cache()
 
+    # prefill with E4M3 queries and keys (the headline shape)
+    prefill_fp8 = None
+    if not args.skip_decode:
+        q, k, v = tensors[0], tensors[1], tensors[2]
+        q_s = float(q.abs().amax()) / 448.0
+        k_s = float(k.abs().amax()) / 448.0
+        q8 = (q.float() / q_s).to(torch.float8_e4m3fn).view(torch.uint8)
+        k8 = (k.float() / k_s).to(torch.float8_e4m3fn).view(torch.uint8)
+        o8 = torch.empty_like(tensors[3])
+        l8 = torch.empty_like(tensors[4])
+        fargs = (q8.data_ptr(), k8.data_ptr(), v.data_ptr(), o8.data_ptr(), l8.data_ptr(),
+                 wp.B, wp.H, wp.Nq, wp.Nkv, wp.d, float(wp.softmax_scale), int(wp.causal),
+                 stream.cuda_stream, q_s, k_s, binding._dtype_code(wp.dtype),
+                 binding._dtype_code(o8.dtype))
+
+        def fp8_call():
+            check(binding.fa_fwd_fp8(*fargs), "fa_fwd_fp8")
+
+        fsteps = max(3, args.steps // 4)
+        with ClockSampler(local) as clk_f, torch.cuda.stream(stream):
+            ms_f = time_steps(fp8_call, fsteps, args.warmup, ws, stream)
+        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+        tf_f = flops / (ms_f * 1e-3) / 1e12
+        # Half the FLOPs (Q K^T) run at the E4M3 rate, nominally twice bf16; half (P V) at bf16.
+        peak_f = peak_t * 4.0 / 3.0
+        prefill_fp8 = {
+            "workload": workload_config(wp, "bf16")["workload"] + ", Q and K in E4M3 "
+                        "(per-tensor scales), V and P bf16",
+            "value": whole_job_rate(flops, ms_f, ws) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms_f, "steps": fsteps, "gpu_launches": fsteps,
+            "roofline": {"bound": "tensor", "achieved": tf_f, "peak": peak_f, "unit": "TFLOP/s",
+                         "frac": tf_f / peak_f, "traffic": None,
+                         "peak_source": "blend of half E4M3 (2x measured bf16, the nominal "
+                                        "ratio) and half measured bf16: 4/3 x " + peak_src,
+                         "frac_of_bf16_peak": tf_f / peak_t, "flops_per_launch": flops},
+            "clocks": clk_f.summary(),
+        }
+        del q8, k8, o8, l8
+        torch.cuda.empty_cache()
+
     # packed variable-length prefill: a ragged causal batch
     prefill_varlen = None
     if not args.skip_decode:
@@ -469,6 +511,7 @@ def arm_ours(args, ws, rank, local):
             "decode": decode,
             "decode_paged": decode_paged,
             "prefill_varlen": prefill_varlen,
+            "prefill_fp8": prefill_fp8,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

@@ -41,6 +41,7 @@ _SIGNATURES = {
     "fa_fwd_prefill": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I, _I],
     "fa_fwd_decode": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
     "fa_fwd_decode_noalloc": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
+    "fa_fwd_fp8": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _F, _F, _I, _I],
     "fa_fwd_varlen": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP,
                       _I, _I],
     "fa_fwd_decode_paged": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP,
@@ -109,6 +110,12 @@ def fa_fwd_decode_noalloc(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype
     instead of a cudaMalloc'd workspace, for callers that cannot allocate device memory."""
     return library().fa_fwd_decode_noalloc(q, k, v, o, lse, B, H, Nkv, d, scale, stream,
                                            in_dtype, o_dtype, num_splits)
+
+
+def fa_fwd_fp8(q8, k8, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, q_scale, k_scale,
+               v_dtype, o_dtype) -> int:
+    return library().fa_fwd_fp8(q8, k8, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream,
+                                q_scale, k_scale, v_dtype, o_dtype)
 
 
 def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q, max_k, d, scale,
@@ -272,4 +279,38 @@ def varlen_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max
                            _dtype_code(o.dtype))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd_varlen")
+    return o, lse
+
+
+def fp8_attention(q8, k8, v, q_scale: float, k_scale: float, causal: bool = False,
+                  scale: Optional[float] = None, out_dtype=None, stream=None):
+    """Attention with E4M3 queries and keys: q8 [B,H,Nq,128], k8 [B,H,Nkv,128] as uint8 (or
+    torch.float8_e4m3fn) codes standing for q_scale * Q and k_scale * K; v [B,H,Nkv,128]
+    fp16/bf16.  Returns (o, lse) like attention()."""
+    import torch
+
+    if q8.dtype == torch.float8_e4m3fn:
+        q8 = q8.view(torch.uint8)
+    if k8.dtype == torch.float8_e4m3fn:
+        k8 = k8.view(torch.uint8)
+    ts = (q8, k8, v)
+    if not all(t.is_cuda and t.is_contiguous() for t in ts):
+        raise ValueError("fp8_attention() takes contiguous CUDA tensors")
+    if q8.dtype != torch.uint8 or k8.dtype != torch.uint8:
+        raise ValueError("q8 and k8 must hold E4M3 codes (uint8 or float8_e4m3fn)")
+    B, H, Nq, d = q8.shape
+    Nkv = k8.shape[2]
+    if tuple(k8.shape) != (B, H, Nkv, d) or tuple(v.shape) != (B, H, Nkv, d):
+        raise ValueError("k8 and v must be [B,H,Nkv,d] with q8's B, H and d")
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((B, H, Nq, d), dtype=out_dtype, device=v.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=v.device)
+    s = torch.cuda.current_stream(v.device) if stream is None else stream
+    with torch.cuda.device(v.device):
+        rc = fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                        B, H, Nq, Nkv, d, scale, int(bool(causal)), s.cuda_stream,
+                        float(q_scale), float(k_scale), _dtype_code(v.dtype), _dtype_code(o.dtype))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_fp8")
     return o, lse

@@ -92,6 +92,22 @@ int make_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, bool
   return FA_OK;
 }
 
+// 3-D view (d, N, B*H) of a [B,H,N,d] tensor of one-byte codes (d = 128); box
+// (128, 128, 1): one 128-byte row per query or key, 128-byte swizzle.
+int make_map_u8(CUtensorMap* map, const void* ptr, int N, long long BH, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N) * d};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return FA_OK;
+}
+
 // 3-D view (d, H, tokens) of a packed [tokens, H, d] tensor; box (64, 1, 128): the same
 // 128 rows x 128 B shared-memory tile as above, rows being tokens of one head.
 int make_map_packed(CUtensorMap* map, const void* ptr, long long tokens, int H, int d, bool bf16) {
@@ -372,6 +388,64 @@ int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* l
   if (rc != FA_OK) return rc;
   if (num_splits < 0) return FA_ERR_INVALID_ARG;
   return run_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype, num_splits);
+}
+
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v, void* o, float* lse, int B,
+               int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
+               float q_scale, float k_scale, int v_dtype, int o_dtype) {
+  if (!q8 || !k8 || !v || !o) return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Nq < 1 || Nkv < 1) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !std::isfinite(q_scale) || !std::isfinite(k_scale)) return FA_ERR_INVALID_ARG;
+  const float s_all = scale * q_scale * k_scale;
+  if (!std::isfinite(s_all)) return FA_ERR_INVALID_ARG;
+  if (v_dtype != FA_F16 && v_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_F16 && o_dtype != FA_BF16 && o_dtype != FA_F32) return FA_ERR_INVALID_ARG;
+  if (o_dtype != FA_F32 && o_dtype != v_dtype) return FA_ERR_UNSUPPORTED;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v, 16) || !aligned(o, 16)) return FA_ERR_INVALID_ARG;
+  if (lse && !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t qb = BH * Nq * d, kb = BH * Nkv * d, vb = BH * Nkv * d * 2;
+  const size_t ob = BH * Nq * d * (o_dtype == FA_F32 ? 4 : 2), lb = BH * Nq * 4;
+  const void* ins[3] = {q8, k8, v};
+  const size_t in_bytes[3] = {qb, kb, vb};
+  for (int i = 0; i < 3; ++i) {
+    if (overlaps(o, ob, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+    if (lse && overlaps(lse, lb, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+  }
+  if (lse && overlaps(lse, lb, o, ob)) return FA_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if ((rc = make_map_u8(&tq, q8, Nq, static_cast<long long>(BH), d)) != FA_OK) return rc;
+  if ((rc = make_map_u8(&tk, k8, Nkv, static_cast<long long>(BH), d)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, Nkv, static_cast<long long>(BH), d, v_dtype == FA_BF16)) != FA_OK) return rc;
+  fa::PrefillParams p{};
+  p.BH = static_cast<int>(BH);
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.off = Nkv - Nq;
+  p.causal = causal;
+  p.n_qtiles = (Nq + 127) / 128;
+  p.n_pairs = (p.n_qtiles + 1) / 2;
+  p.n_kvtiles = (Nkv + 127) / 128;
+  const long long units = static_cast<long long>(BH) * p.n_pairs;
+  if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  p.n_units = static_cast<int>(units);
+  p.scale_log2 = scale_log2(s_all);  // the per-tensor scales fold into the score scale
+  p.cu_q = p.cu_k = nullptr;
+  p.H = H;
+  long long grid = ds->sm_count;
+  if (grid > units) grid = units;
+  if (grid < 1) grid = 1;
+  cudaError_t e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, v_dtype == FA_BF16,
+                                     o_dtype == FA_F32, static_cast<int>(grid), ds->status,
+                                     static_cast<cudaStream_t>(stream), true);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

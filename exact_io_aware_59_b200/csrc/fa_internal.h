@@ -51,9 +51,11 @@ struct PagedKV {
 };
 
 // Kernel launchers (fa_prefill.cu, fa_decode.cu).  Return the launch's cudaError_t.
+// qk8: tq / tk hold E4M3 codes (d = 128, box 128 x 128 bytes); bf16 then names V's type.
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            void* o, float* lse, const PrefillParams& p, int d, bool bf16,
-                           bool o_f32, int grid, int* status, cudaStream_t stream);
+                           bool o_f32, int grid, int* status, cudaStream_t stream,
+                           bool qk8 = false);
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                           const DecodeParams& p, int d, bool bf16, bool o_f32, float* part_o,

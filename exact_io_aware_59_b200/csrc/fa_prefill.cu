@@ -169,7 +169,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- producer (TMA)
-template <int D, bool VARLEN>
+// QK8: Q and K hold one-byte E4M3 codes, one 128-byte row per query / key (d = 128), so a
+// Q or K tile is a single 128 x 128 B box in the first half of its slot.
+template <int D, bool VARLEN, bool QK8>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                          const PrefillParams& p, uint32_t sbase, uint32_t bars, int* status,
                          volatile int* abort_flag) {
@@ -189,15 +191,20 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
       break;
     }
     const uint32_t qf = bar_addr(bars, C::kBarQFull);
-    mbar_arrive_expect_tx(qf, ((n0 > 0) + (n1 > 0)) * C::kQBytes);
+    constexpr uint32_t kQLoad = QK8 ? BM * 128 : C::kQBytes;
+    mbar_arrive_expect_tx(qf, ((n0 > 0) + (n1 > 0)) * kQLoad);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       if ((t == 0 ? n0 : n1) == 0) continue;
       int c1, c2;
       tile_coords<VARLEN>(p, x, (2 * pair + t) * BM, true, c1, c2);
+      if constexpr (QK8) {
+        tma_load_3d(sbase + C::kQOff + t * C::kQBytes, tq, qf, 0, c1, c2);
+      } else {
 #pragma unroll
-      for (int sub = 0; sub < D / 64; ++sub)
-        tma_load_3d(sbase + C::kQOff + t * C::kQBytes + sub * BM * 128, tq, qf, sub * 64, c1, c2);
+        for (int sub = 0; sub < D / 64; ++sub)
+          tma_load_3d(sbase + C::kQOff + t * C::kQBytes + sub * BM * 128, tq, qf, sub * 64, c1, c2);
+      }
     }
     ++q_issued;
     for (int j = 0; j < nmax && ok; ++j) {
@@ -210,13 +217,18 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
           break;
         }
         const uint32_t fb = bar_addr(bars, C::kBarFull + slot);
-        mbar_arrive_expect_tx(fb, C::kKVBytes);
+        const bool k8 = QK8 && which == 0;
+        mbar_arrive_expect_tx(fb, k8 ? BN * 128 : C::kKVBytes);
         const uint32_t dst = sbase + C::kRingOff + slot * C::kKVBytes;
         int c1, c2;
         tile_coords<VARLEN>(p, x, j * BN, false, c1, c2);
+        if (k8) {
+          tma_load_3d(dst, tk, fb, 0, c1, c2);
+        } else {
 #pragma unroll
-        for (int sub = 0; sub < D / 64; ++sub)
-          tma_load_3d(dst + sub * BN * 128, which ? tv : tk, fb, sub * 64, c1, c2);
+          for (int sub = 0; sub < D / 64; ++sub)
+            tma_load_3d(dst + sub * BN * 128, which ? tv : tk, fb, sub * 64, c1, c2);
+        }
         ++ld;
       }
     }
@@ -233,9 +245,16 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
 // Shared-memory descriptors are built once per buffer; an MMA step's operand is the
 // buffer's descriptor plus (byte offset >> 4) in the start-address field (shared-memory
 // addresses are below 2^18, so the 14-bit field never carries).
-template <int D>
+template <int D, bool QK8>
 __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc,
                                         uint32_t idesc) {
+  if constexpr (QK8) {
+    // One-byte codes: a row is one 128-byte swizzle row; 32 elements (32 B) per step.
+#pragma unroll
+    for (int kk = 0; kk < D / 32; ++kk)
+      mma_ss_f8(d_tmem, q_desc + ((kk * 32) >> 4), k_desc + ((kk * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
+    return;
+  }
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     // K-major operand, 128-byte swizzle: 64-element column blocks of 128 rows x 128 B,
@@ -257,12 +276,12 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint6
   }
 }
 
-template <int D, bool BF16, bool VARLEN>
+template <int D, bool BF16, bool VARLEN, bool QK8>
 __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                            int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
   constexpr int S = C::kStages;
-  constexpr uint32_t idesc_s = make_idesc_f16(BM, BN, BF16, false);
+  constexpr uint32_t idesc_s = QK8 ? make_idesc_e4m3(BM, BN) : make_idesc_f16(BM, BN, BF16, false);
   constexpr uint32_t idesc_o = make_idesc_f16(BM, D, BF16, true);
   uint32_t ld = 0, q_used = 0, pcount[2] = {0, 0};
   bool ok = true;
@@ -290,7 +309,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       if (n[t] == 0) continue;
-      issue_s<D>(tmem + t * 128, q_desc(t), k_desc(kslot0), idesc_s);
+      issue_s<D, QK8>(tmem + t * 128, q_desc(t), k_desc(kslot0), idesc_s);
       tc_commit(bar_addr(bars, C::kBarSFull + t));
     }
     tc_commit(bar_addr(bars, C::kBarEmpty + kslot0));
@@ -319,7 +338,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
             tc_fence_after();
             ++ld;
           }
-          issue_s<D>(tmem + t * 128, q_desc(t), k_desc(knext), idesc_s);
+          issue_s<D, QK8>(tmem + t * 128, q_desc(t), k_desc(knext), idesc_s);
           tc_commit(bar_addr(bars, C::kBarSFull + t));
         }
       }
@@ -600,7 +619,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   }
 }
 
-template <int D, bool BF16, bool OF32, bool VARLEN>
+template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_prefill_sm100(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, void* __restrict__ o,
@@ -651,9 +670,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
     if (warp == 0) {
-      if (lane == 0) producer<D, VARLEN>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
+      if (lane == 0) producer<D, VARLEN, QK8>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D, BF16, VARLEN>(p, sbase, bars, tmem, status, abort_flag);
+      if (lane == 0) mma_issuer<D, BF16, VARLEN, QK8>(p, sbase, bars, tmem, status, abort_flag);
       __syncwarp();
       // Release TMEM once both softmax warpgroups have finished reading it.
       drain_wait(bar_addr(bars, C::kBarDone), 0);
@@ -672,11 +691,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool BF16, bool OF32, bool VARLEN>
+template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                      float* lse, const PrefillParams& p, int grid, int* status,
                      cudaStream_t stream) {
-  auto kern = fa_prefill_sm100<D, BF16, OF32, VARLEN>;
+  auto kern = fa_prefill_sm100<D, BF16, OF32, VARLEN, QK8>;
   static bool configured = false;  // per template instance
   static cudaError_t config_err = cudaSuccess;
   if (!configured) {
@@ -704,11 +723,18 @@ size_t prefill_smem_bytes(int d) {
 
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            void* o, float* lse, const PrefillParams& p, int d, bool bf16,
-                           bool o_f32, int grid, int* status, cudaStream_t stream) {
-#define FA_PREFILL_CASE(D_, B_, F_)                                                          \
-  if (d == D_ && bf16 == B_ && o_f32 == F_)                                                   \
-    return p.cu_q ? launch_t<D_, B_, F_, true>(tq, tk, tv, o, lse, p, grid, status, stream)   \
-                  : launch_t<D_, B_, F_, false>(tq, tk, tv, o, lse, p, grid, status, stream);
+                           bool o_f32, int grid, int* status, cudaStream_t stream, bool qk8) {
+  if (qk8) {  // E4M3 queries and keys: d = 128, [B,H,N,d] layout
+    if (d != 128 || p.cu_q) return cudaErrorInvalidValue;
+    if (bf16 && o_f32) return launch_t<128, true, true, false, true>(tq, tk, tv, o, lse, p, grid, status, stream);
+    if (bf16) return launch_t<128, true, false, false, true>(tq, tk, tv, o, lse, p, grid, status, stream);
+    if (o_f32) return launch_t<128, false, true, false, true>(tq, tk, tv, o, lse, p, grid, status, stream);
+    return launch_t<128, false, false, false, true>(tq, tk, tv, o, lse, p, grid, status, stream);
+  }
+#define FA_PREFILL_CASE(D_, B_, F_)                                                               \
+  if (d == D_ && bf16 == B_ && o_f32 == F_)                                                        \
+    return p.cu_q ? launch_t<D_, B_, F_, true, false>(tq, tk, tv, o, lse, p, grid, status, stream) \
+                  : launch_t<D_, B_, F_, false, false>(tq, tk, tv, o, lse, p, grid, status, stream);
   FA_PREFILL_CASE(128, true, true)
   FA_PREFILL_CASE(128, true, false)
   FA_PREFILL_CASE(128, false, true)

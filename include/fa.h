@@ -137,6 +137,22 @@ int fa_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* o, 
                           int in_dtype, int o_dtype, int num_splits);
 
 /*
+ * fa_fwd_fp8 -- prefill with FP8 queries and keys ("FlashAttention 1-2-3" (myaihardware),
+ * section "FlashAttention-3: FP8, Async Warp Overlap, and Hopper-Specific Optimizations":
+ * FP8 inputs to the tensor cores for Q K^T).
+ *   q8 [B,H,Nq,d] and k8 [B,H,Nkv,d] hold E4M3 codes (one byte each, the "fn" variant:
+ *   no infinities); they stand for q_scale * Q and k_scale * K (per-tensor scales).
+ *   v [B,H,Nkv,d] in v_dtype (FA_F16 or FA_BF16), o [B,H,Nq,d] in FA_F32 or v_dtype,
+ *   lse [B,H,Nq] fp32 (may be NULL).  S = Q K^T runs on tcgen05 kind::f8f6f4 (E4M3 x
+ *   E4M3, fp32 accumulate); P is rounded to v_dtype for P V as in fa_fwd.  The result is
+ *   softmax(scale * q_scale * k_scale * Q8 K8^T [+ causal]) V.  d must be 128.
+ *   Same ownership, alignment (16 bytes for q8, k8, v, o) and error rules as fa_fwd.
+ */
+int fa_fwd_fp8(const void* q8, const void* k8, const void* v, void* o, float* lse, int B,
+               int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
+               float q_scale, float k_scale, int v_dtype, int o_dtype);
+
+/*
  * fa_fwd_varlen -- prefill over a packed batch of sequences of different lengths
  * ("FlashAttention 1-2-3" (myaihardware), section "When FlashAttention Doesn't Help":
  * continuous batching, each sequence of the batch an independent problem).

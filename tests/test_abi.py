@@ -168,3 +168,22 @@ def _varlen(**kw):
 ])
 def test_varlen_argument_checks(kw, code):
     assert _varlen(**kw) == code
+
+
+def test_fp8_entry_checks():
+    f = binding.fa_fwd_fp8
+    args = dict(q8=Q, k8=K, v=V, o=O, lse=L, B=1, H=1, Nq=4, Nkv=4, d=128, scale=0.1, causal=0,
+                stream=None, qs=1.0, ks=1.0, vd=1, od=2)
+
+    def call(**kw):
+        a = dict(args)
+        a.update(kw)
+        return f(a["q8"], a["k8"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Nq"], a["Nkv"],
+                 a["d"], a["scale"], a["causal"], a["stream"], a["qs"], a["ks"], a["vd"], a["od"])
+
+    assert call(d=64) == binding.FA_ERR_UNSUPPORTED
+    assert call(q8=None) == binding.FA_ERR_INVALID_ARG
+    assert call(qs=math.inf) == binding.FA_ERR_INVALID_ARG
+    assert call(vd=2) == binding.FA_ERR_INVALID_ARG          # V must be 16-bit
+    assert call(vd=0, od=1) == binding.FA_ERR_UNSUPPORTED     # 16-bit O must be V's type
+    assert call(k8=K + 8) == binding.FA_ERR_INVALID_ARG       # misaligned

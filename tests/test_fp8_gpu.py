@@ -1,0 +1,98 @@
+"""GPU parity of the FP8-Q/K prefill (fa_fwd_fp8) against the fp64 oracle
+(oracle.fp8_qk_attention: attention() of the dequantised E4M3 tensors, pinned on the CPU).
+P stays in V's 16-bit type, so the bf16 tolerances apply unchanged."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_59_b200 import binding
+from exact_io_aware_59_b200.inputs import randn
+from fa_testlib import REL_O16, compare, has_b200, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _device_clean():
+    if not has_b200():
+        pytest.skip("needs a B200 (sm_100a)")
+    binding.fa_device_status(clear=True)
+    yield
+    torch.cuda.synchronize()
+    assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+
+
+def _quantise(x):
+    """Per-tensor scale to the E4M3 range, then round to E4M3 codes."""
+    s = float(x.abs().max()) / 448.0
+    return (x / s).to(torch.float8_e4m3fn).view(torch.uint8), s
+
+
+def _inputs(B, H, Nq, Nkv, vdtype, seed, std=1.0):
+    qf = randn((B, H, Nq, 128), seed, torch.float32, std)
+    kf = randn((B, H, Nkv, 128), seed + 1, torch.float32, std)
+    v = randn((B, H, Nkv, 128), seed + 2, vdtype)
+    q8, qs = _quantise(qf)
+    k8, ks = _quantise(kf)
+    return q8, qs, k8, ks, v
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("vdtype", [torch.bfloat16, torch.float16])
+def test_fp8_matches_oracle(causal, vdtype):
+    B, H, Nq, Nkv = 2, 3, 300, 333
+    q8, qs, k8, ks, v = _inputs(B, H, Nq, Nkv, vdtype, 1200)
+    o, lse = binding.fp8_attention(q8.cuda(), k8.cuda(), v.cuda(), qs, ks, causal=causal,
+                                   scale=128 ** -0.5)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.fp8_qk_attention(q8, k8, v, qs, ks, 128 ** -0.5, causal)
+    compare(o, lse, o_ref, l_ref)
+
+
+def test_fp8_16bit_out_peaky():
+    """Larger scores (Q std 4 before quantisation), 16-bit O."""
+    B, H, N = 1, 2, 520
+    q8, qs, k8, ks, v = _inputs(B, H, N, N, torch.bfloat16, 1300, std=4.0)
+    o, lse = binding.fp8_attention(q8.cuda(), k8.cuda(), v.cuda(), qs, ks, causal=True,
+                                   scale=128 ** -0.5, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.fp8_qk_attention(q8, k8, v, qs, ks, 128 ** -0.5, True)
+    compare(o, lse, o_ref, l_ref, rel_o=REL_O16[torch.bfloat16])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_equals_bf16_path_on_exact_values(causal):
+    """Small integers are exact in E4M3 and bf16 and their dot products are exact in
+    fp32, so S, and with it the whole result, must equal fa_fwd's bit for bit."""
+    B, H, N = 1, 2, 384
+    g = torch.Generator().manual_seed(31)
+    qi = torch.randint(-3, 4, (B, H, N, 128), generator=g).float()
+    ki = torch.randint(-3, 4, (B, H, N, 128), generator=g).float()
+    v = randn((B, H, N, 128), 1400, torch.bfloat16)
+    q8 = qi.to(torch.float8_e4m3fn).view(torch.uint8)
+    k8 = ki.to(torch.float8_e4m3fn).view(torch.uint8)
+    o8, l8 = binding.fp8_attention(q8.cuda(), k8.cuda(), v.cuda(), 1.0, 1.0, causal=causal,
+                                   scale=0.02)
+    o16, l16 = binding.attention(qi.to(torch.bfloat16).cuda(), ki.to(torch.bfloat16).cuda(),
+                                 v.cuda(), causal=causal, scale=0.02)
+    torch.cuda.synchronize()
+    assert torch.equal(o8, o16) and torch.equal(l8, l16)
+
+
+def test_fp8_full_size_sampled():
+    """The long causal prefill shape (B=1, H=32, N=8192) with E4M3 Q and K, sampled rows."""
+    B, H, N = 1, 32, 8192
+    qf = randn((B, H, N, 128), 1500, torch.float32, device="cuda")
+    kf = randn((B, H, N, 128), 1501, torch.float32, device="cuda")
+    v = randn((B, H, N, 128), 1502, torch.bfloat16, device="cuda")
+    q8, qs = _quantise(qf)
+    k8, ks = _quantise(kf)
+    del qf, kf
+    o, lse = binding.fp8_attention(q8, k8, v, qs, ks, causal=True, scale=128 ** -0.5)
+    torch.cuda.synchronize()
+    rows = sample_rows(B, H, N, per_head=24, seed=15)
+    o_ref, l_ref = oracle.fp8_qk_attention(q8.cpu(), k8.cpu(), v.cpu(), qs, ks, 128 ** -0.5,
+                                           True, rows=rows)
+    idx = torch.from_numpy(rows).cuda()
+    compare(o.reshape(-1, 128)[idx], lse.reshape(-1)[idx], o_ref, l_ref)
