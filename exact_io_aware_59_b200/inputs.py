@@ -126,3 +126,9 @@ def varlen_inputs(lengths, H: int, d: int, dtype: torch.dtype, seed_base: int, d
     for n in lengths:
         cu.append(cu[-1] + int(n))
     return q, k, v, torch.tensor(cu, dtype=torch.int32, device=device)
+
+
+def make_grad_out(B: int, H: int, Nq: int, d: int, dtype: torch.dtype, seed: int, device="cpu"):
+    """Upstream gradient dO [B,H,Nq,d] for the backward pass: iid N(0,1) rounded to
+    `dtype`.  Workloads seed it with 1000*index + 3 (after Q, K, V)."""
+    return randn((B, H, Nq, d), seed, dtype, 1.0, device)

@@ -21,6 +21,13 @@ Contents
                               enabling trick").  An optional threshold tau keeps a stale
                               max until the new one exceeds it by more than tau (log2
                               units); the result is the same in exact arithmetic.
+``attention_backward``        dQ, dK, dV of attention() for an upstream gradient dO: the
+                              gradient of the definition, written out with the whole
+                              score matrix of a head in numpy fp64 ("Flash Attention --
+                              Module 12.3" section "Prefill vs Decode", "Training").
+``paged_decode_attention``,   attention() over a paged KV cache, over a packed batch of
+``varlen_attention``,         sequences, and over FP8 (E4M3) queries and keys decoded
+``fp8_qk_attention``          from the format's definition (``e4m3_to_f64``).
 ``lse_combine``               merges partial results over disjoint key sets by their
                               log-sum-exp, the reduction step of split-KV decoding
                               ("FlashAttention 1-2-3" section "Beyond FlashAttention":
@@ -244,6 +251,62 @@ def fp8_qk_attention(q8, k8, v, q_scale: float, k_scale: float, scale: float, ca
     kf = torch.from_numpy(e4m3_to_f64(k8) * float(k_scale))
     vf = torch.as_tensor(v).detach().cpu().to(torch.float64)
     return attention(qf, kf, vf, scale, causal, rows=rows, nthreads=nthreads, lib=lib)
+
+
+def attention_backward(q, k, v, do, scale: float, causal: bool, heads=None):
+    """Gradients dQ, dK, dV of attention() for an upstream gradient dO, in fp64.
+
+    The pages say only that training runs a backward pass that is IO-aware as the forward
+    is ("Flash Attention -- Module 12.3", section "Prefill vs Decode", "Training"), and
+    that the forward keeps per-row softmax statistics so that nothing N x N has to be
+    stored ("FlashAttention 1-2-3" (myaihardware), section "FlashAttention-1: Tiling,
+    Recomputation, and Online Softmax").  What it must compute is the gradient of the
+    definition O = softmax(scale * Q K^T [+ causal mask]) V, written out here with the
+    whole score matrix of one head (numpy matmuls as the only library step):
+
+        P    = softmax of the masked, scaled scores, row by row (masked entries 0)
+        dV   = P^T dO
+        dP   = dO V^T
+        D_i  = sum_j P_ij dP_ij            (equal to dO_i . O_i)
+        dS   = P * (dP - D)                (the softmax Jacobian applied row by row)
+        dQ   = scale * dS K
+        dK   = scale * dS^T Q
+
+    q, do: [B,H,Nq,d]; k, v: [B,H,Nkv,d] (torch tensors of any float type, or numpy).
+    Causal masking is aligned bottom-right as in attention(); a query row that sees no key
+    has P = 0 and contributes nothing.  heads: optional list of flat head ids b*H + h;
+    only those heads are computed (the others stay 0).  Returns numpy float64
+    (dq [B,H,Nq,d], dk [B,H,Nkv,d], dv [B,H,Nkv,d]).
+    """
+    qf, kf, vf, gf = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, Nq, d = qf.shape
+    Nkv = kf.shape[2]
+    assert kf.shape == (B, H, Nkv, d) and vf.shape == (B, H, Nkv, d) and gf.shape == qf.shape
+    dq = np.zeros_like(qf)
+    dk = np.zeros_like(kf)
+    dv = np.zeros_like(vf)
+    if Nq == 0 or Nkv == 0:
+        return dq, dk, dv
+    visible = np.ones((Nq, Nkv), dtype=bool)
+    if causal:
+        visible = np.arange(Nkv)[None, :] <= np.arange(Nq)[:, None] + (Nkv - Nq)
+    ids = range(B * H) if heads is None else heads
+    for bh in ids:
+        b, h = divmod(int(bh), H)
+        Q, K, V, G = qf[b, h], kf[b, h], vf[b, h], gf[b, h]
+        s = np.where(visible, scale * (Q @ K.T), -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        m = np.where(np.isfinite(m), m, 0.0)
+        e = np.where(visible, np.exp(s - m), 0.0)
+        z = e.sum(axis=1, keepdims=True)
+        P = e / np.where(z > 0, z, 1.0)
+        dv[b, h] = P.T @ G
+        dP = G @ V.T
+        D = (P * dP).sum(axis=1, keepdims=True)
+        dS = P * (dP - D)
+        dq[b, h] = scale * (dS @ K)
+        dk[b, h] = scale * (dS.T @ Q)
+    return dq, dk, dv
 
 
 def _f64(x):

@@ -414,3 +414,120 @@ def test_fp8_attention_is_attention_of_the_dequantised_tensors(oracle_mod):
     o2, l2 = oracle_mod.fp8_qk_attention(q8, k8, v, 1.0, 1.0, 0.1 * 0.5 * 0.25, True)
     np.testing.assert_allclose(o2, o, rtol=0, atol=1e-12)
     np.testing.assert_allclose(l2, lse, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- backward pass
+def _bwd_inputs(B, H, Nq, Nkv, d, seed, dtype=torch.float64):
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, torch.float32, seed)
+    g = randn((B, H, Nq, d), seed + 3, torch.float32)
+    return q.to(dtype), k.to(dtype), v.to(dtype), g.to(dtype)
+
+
+@pytest.mark.parametrize("causal,Nq,Nkv", [(False, 6, 9), (True, 6, 9), (True, 9, 9),
+                                           (False, 9, 4)])
+def test_backward_matches_autograd_of_the_definition(oracle_mod, causal, Nq, Nkv):
+    """torch autograd (fp64) of softmax(scale Q K^T + mask) V, a library derivation of the
+    same gradients, agrees with the written-out formulas."""
+    B, H, d = 2, 2, 5
+    q, k, v, g = _bwd_inputs(B, H, Nq, Nkv, d, 41)
+    scale = 0.37
+    qa, ka, va = (t.clone().requires_grad_(True) for t in (q, k, v))
+    s = scale * qa @ ka.transpose(-1, -2)
+    if causal:
+        s = s.masked_fill(~torch.from_numpy(_visible_mask(Nq, Nkv, True)), float("-inf"))
+    (torch.softmax(s, dim=-1) @ va).backward(g)
+    dq, dk, dv = oracle_mod.attention_backward(q, k, v, g, scale, causal)
+    for ours, ref in ((dq, qa.grad), (dk, ka.grad), (dv, va.grad)):
+        np.testing.assert_allclose(ours, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_backward_matches_finite_differences_of_the_forward_oracle(oracle_mod):
+    """Central differences of L = sum(dO * O), O from the C forward oracle, against the
+    backward formulas: every element of Q, K and V on a tiny causal case with Nq != Nkv."""
+    B, H, Nq, Nkv, d = 1, 2, 3, 4, 3
+    q, k, v, g = _bwd_inputs(B, H, Nq, Nkv, d, 57)
+    scale, eps = 0.61, 1e-6
+    gf = _f64(g)
+    dq, dk, dv = oracle_mod.attention_backward(q, k, v, g, scale, True)
+
+    def loss(qq, kk, vv):
+        o, _ = oracle_mod.attention(qq, kk, vv, scale, True)
+        return float((o * gf).sum())
+
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        base = [q.clone(), k.clone(), v.clone()]
+        t = base[which]
+        for idx in np.ndindex(*t.shape):
+            plus = [x.clone() for x in base]
+            minus = [x.clone() for x in base]
+            plus[which][idx] += eps
+            minus[which][idx] -= eps
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            assert grad[idx] == pytest.approx(fd, abs=1e-7), (which, idx)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_column_sums(oracle_mod, causal):
+    """Rows of P sum to 1, so the dV rows sum to the dO rows summed over queries; rows of
+    dS sum to 0, so the dK rows sum to zero.  (Causal with Nq <= Nkv: every query sees a
+    key.)  A dropped D term or an unnormalised P breaks one of these."""
+    B, H, Nq, Nkv, d = 2, 3, 21, 33, 8
+    q, k, v, g = _bwd_inputs(B, H, Nq, Nkv, d, 63)
+    dq, dk, dv = oracle_mod.attention_backward(q, k, v, g, 0.3, causal)
+    np.testing.assert_allclose(dv.sum(axis=2), _f64(g).sum(axis=2), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, rtol=0, atol=1e-11)
+
+
+def test_backward_key_shift_invariance(oracle_mod):
+    """Adding one vector c to every key adds q_i . c to a whole row of scores, which the
+    softmax ignores: dQ, dK and dV do not change."""
+    B, H, Nq, Nkv, d = 1, 2, 13, 17, 6
+    q, k, v, g = _bwd_inputs(B, H, Nq, Nkv, d, 71)
+    c = torch.linspace(-1.0, 2.0, d, dtype=torch.float64)
+    a = oracle_mod.attention_backward(q, k, v, g, 0.45, True)
+    b = oracle_mod.attention_backward(q, k + c, v, g, 0.45, True)
+    for x, y in zip(a, b):
+        np.testing.assert_allclose(x, y, rtol=0, atol=1e-11)
+
+
+def test_backward_uniform_attention_closed_form(oracle_mod):
+    """K = 0 makes every score 0 and P = 1/Nkv: then dV_j = sum_i dO_i / Nkv,
+    dQ = 0, and dK_j = scale/Nkv * sum_i (dO_i . (V_j - mean V)) Q_i."""
+    B, H, Nq, Nkv, d = 1, 1, 7, 5, 4
+    q, _, v, g = _bwd_inputs(B, H, Nq, Nkv, d, 83)
+    k = torch.zeros(B, H, Nkv, d, dtype=torch.float64)
+    scale = 0.8
+    dq, dk, dv = oracle_mod.attention_backward(q, k, v, g, scale, False)
+    Q, V, G = _f64(q)[0, 0], _f64(v)[0, 0], _f64(g)[0, 0]
+    np.testing.assert_allclose(dq, 0.0, atol=0)
+    np.testing.assert_allclose(dv[0, 0], np.tile(G.sum(axis=0) / Nkv, (Nkv, 1)), atol=1e-13)
+    vbar = V.mean(axis=0)
+    for j in range(Nkv):
+        ref = sum(scale / Nkv * float(G[i] @ (V[j] - vbar)) * Q[i] for i in range(Nq))
+        np.testing.assert_allclose(dk[0, 0, j], ref, atol=1e-13)
+
+
+def test_backward_single_key_and_masked_rows(oracle_mod):
+    """One key: P = 1, so dV = sum of dO and dS = 0 (dQ = dK = 0).  Causal with Nq > Nkv:
+    the first Nq - Nkv queries see no key and get dQ = 0; the rest equal the gradient of
+    the visible block alone."""
+    q, k, v, g = _bwd_inputs(1, 2, 6, 1, 4, 91)
+    dq, dk, dv = oracle_mod.attention_backward(q, k, v, g, 0.5, False)
+    np.testing.assert_allclose(dv[:, :, 0], _f64(g).sum(axis=2), atol=1e-13)
+    assert np.abs(dq).max() < 1e-13 and np.abs(dk).max() < 1e-13
+    q, k, v, g = _bwd_inputs(1, 2, 9, 5, 4, 97)
+    dq, dk, dv = oracle_mod.attention_backward(q, k, v, g, 0.5, True)
+    assert np.all(dq[:, :, :4] == 0)
+    sub = oracle_mod.attention_backward(q[:, :, 4:], k, v, g[:, :, 4:], 0.5, True)
+    np.testing.assert_allclose(dq[:, :, 4:], sub[0], atol=1e-13)
+    np.testing.assert_allclose(dk, sub[1], atol=1e-13)
+    np.testing.assert_allclose(dv, sub[2], atol=1e-13)
+
+
+def test_backward_heads_subset(oracle_mod):
+    q, k, v, g = _bwd_inputs(2, 2, 5, 7, 3, 101)
+    full = oracle_mod.attention_backward(q, k, v, g, 0.4, True)
+    part = oracle_mod.attention_backward(q, k, v, g, 0.4, True, heads=[2])
+    for x, y in zip(full, part):
+        np.testing.assert_array_equal(x[1, 0], y[1, 0])
+        assert np.all(y[0] == 0) and np.all(y[1, 1] == 0)
