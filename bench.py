@@ -10,6 +10,8 @@ One step = one pass of the hot path over one batch of synthetic input:
     fa_fwd_decode_paged call per step;
   * the "prefill_fp8" object times the headline shape with Q and K in E4M3, one
     fa_fwd_fp8 call per step;
+  * the "backward" object times the gradients (dQ, dK, dV) of the headline shape from its
+    O and LSE and a seeded dO, one fa_bwd call (prep, main and dQ kernels) per step;
   * the "prefill_varlen" object times a packed ragged causal batch (16 sequences,
     seeded log-uniform lengths in [512, 8192], H=32, d=128, bf16), one fa_fwd_varlen
     call per step.
@@ -39,8 +41,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_io_aware_59_b200 import binding  # noqa: E402
-from exact_io_aware_59_b200.inputs import (WORKLOADS, Workload, paged_decode_inputs,  # noqa: E402
-                                           varlen_inputs, varlen_lengths, workload_qkv)
+from exact_io_aware_59_b200.inputs import (WORKLOADS, Workload, make_grad_out,  # noqa: E402
+                                           paged_decode_inputs, varlen_inputs, varlen_lengths,
+                                           workload_qkv)
 
 METRIC = "attention fwd TFLOP/s at 1 B200 (% of dense bf16 peak); decode HBM GB/s"
 PREFILL = "long_prefill_causal"
@@ -68,6 +71,13 @@ def attention_flops(w: Workload) -> int:
     visible lower triangle only."""
     pairs = causal_pairs(w.Nq, w.Nkv) if w.causal else w.Nq * w.Nkv
     return 4 * w.d * w.B * w.H * pairs
+
+
+def backward_flops(w: Workload) -> int:
+    """10 * d per visible (query, key) pair: five products (S, dP, dV, dK, dQ) of 2d each,
+    2.5 times the forward's count."""
+    pairs = causal_pairs(w.Nq, w.Nkv) if w.causal else w.Nq * w.Nkv
+    return 10 * w.d * w.B * w.H * pairs
 
 
 def algorithmic_bytes(w: Workload, o_bytes: int) -> int:
@@ -407,6 +417,42 @@ def arm_ours(args, ws, rank, local):
         del q8, k8, o8, l8
         torch.cuda.empty_cache()
 
+    # backward pass (dQ, dK, dV) of the headline shape, from the forward's O and LSE
+    backward = None
+    if not args.skip_decode:
+        q, k, v, o, lse = tensors
+        g = make_grad_out(wp.B, wp.H, wp.Nq, wp.d, wp.dtype, 1000 * wp.index + 3, device="cuda")
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        nws = binding.fa_bwd_workspace_bytes(wp.B, wp.H, wp.Nq, wp.d)
+        bws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        bargs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                 g.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), bws.data_ptr(), nws,
+                 wp.B, wp.H, wp.Nq, wp.Nkv, wp.d, float(wp.softmax_scale), int(wp.causal),
+                 stream.cuda_stream, binding._dtype_code(wp.dtype))
+
+        def bwd_call():
+            check(binding.fa_bwd(*bargs), "fa_bwd")
+
+        bsteps = max(3, args.steps // 4)
+        with ClockSampler(local) as clk_b, torch.cuda.stream(stream):
+            ms_b = time_steps(bwd_call, bsteps, args.warmup, ws, stream)
+        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+        flops_b = backward_flops(wp)
+        tf_b = flops_b / (ms_b * 1e-3) / 1e12
+        backward = {
+            "workload": workload_config(wp, "bf16")["workload"] + ", backward: dQ, dK, dV "
+                        "from Q, K, V, O, LSE and dO (iid N(0,1))",
+            "value": whole_job_rate(flops_b, ms_b, ws) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms_b, "steps": bsteps, "gpu_launches": 3 * bsteps,
+            "roofline": {"bound": "tensor", "achieved": tf_b, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": tf_b / peak_t, "traffic": None, "peak_source": peak_src,
+                         "flops_per_launch": flops_b,
+                         "note": "achieved over the whole call (prep, main and dQ kernels)"},
+            "clocks": clk_b.summary(),
+        }
+        del g, dq, dk, dv, bws
+        torch.cuda.empty_cache()
+
     # packed variable-length prefill: a ragged causal batch
     prefill_varlen = None
     if not args.skip_decode:
@@ -512,6 +558,7 @@ def arm_ours(args, ws, rank, local):
             "decode_paged": decode_paged,
             "prefill_varlen": prefill_varlen,
             "prefill_fp8": prefill_fp8,
+            "backward": backward,
             "e2e": e2e,
             "cpu_baseline": cpu,
         }

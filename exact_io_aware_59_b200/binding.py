@@ -20,6 +20,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_ARCH = 0, 1, 2, 3
 FA_ERR_CUDA, FA_ERR_NOMEM, FA_ERR_DEVICE_TIMEOUT = 4, 5, 6
 FA_F16, FA_BF16, FA_F32 = 0, 1, 2
 FA_DEV_BAD_INPUT = 16
+FA_DEV_TIMEOUT_BACKWARD = 32
 
 HEADER = os.path.join(_build.INCLUDE, "fa.h")
 
@@ -46,6 +47,9 @@ _SIGNATURES = {
                       _I, _I],
     "fa_fwd_decode_paged": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP,
                             _I, _I, _I],
+    "fa_bwd": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _I, _I, _I, _I,
+               _I, _F, _I, _VP, _I],
+    "fa_bwd_workspace_bytes": [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
     "fa_decode_workspace_bytes": [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
     "fa_device_status": [ctypes.POINTER(_I), _I],
     "fa_selftest_wait_timeout": [_VP],
@@ -130,6 +134,20 @@ def fa_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, H
     return library().fa_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, H,
                                          d, page_size, max_pages_per_seq, num_pages, scale,
                                          stream, in_dtype, o_dtype, num_splits)
+
+
+def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Nq, Nkv, d,
+           scale, causal, stream, in_dtype) -> int:
+    return library().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H,
+                            Nq, Nkv, d, scale, causal, stream, in_dtype)
+
+
+def fa_bwd_workspace_bytes(B, H, Nq, d) -> int:
+    out = ctypes.c_size_t(0)
+    rc = library().fa_bwd_workspace_bytes(B, H, Nq, d, ctypes.byref(out))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_workspace_bytes")
+    return int(out.value)
 
 
 def fa_decode_workspace_bytes(B, H, Nkv, d, num_splits) -> int:
@@ -314,3 +332,43 @@ def fp8_attention(q8, k8, v, q_scale: float, k_scale: float, causal: bool = Fals
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd_fp8")
     return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: Optional[float] = None,
+                       workspace=None, stream=None):
+    """dQ, dK, dV of attention() for the upstream gradient dout.  q, o, dout [B,H,Nq,128],
+    k, v [B,H,Nkv,128] contiguous CUDA tensors of one 16-bit dtype; o and lse are the
+    forward's outputs (o in the inputs' dtype, lse fp32 [B,H,Nq]).  workspace: optional
+    uint8 CUDA tensor of at least fa_bwd_workspace_bytes; allocated when omitted.
+    Returns (dq, dk, dv) in the inputs' dtype."""
+    import torch
+
+    ts = (q, k, v, o, dout)
+    if not all(t.is_cuda and t.is_contiguous() for t in ts) or not (lse.is_cuda and lse.is_contiguous()):
+        raise ValueError("attention_backward() takes contiguous CUDA tensors")
+    if any(t.dtype != q.dtype for t in ts) or q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("q, k, v, o and dout must share one dtype, float16 or bfloat16")
+    if lse.dtype != torch.float32:
+        raise ValueError("lse must be float32")
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    if (tuple(k.shape) != (B, H, Nkv, d) or tuple(v.shape) != (B, H, Nkv, d)
+            or tuple(o.shape) != (B, H, Nq, d) or tuple(dout.shape) != (B, H, Nq, d)
+            or tuple(lse.shape) != (B, H, Nq)):
+        raise ValueError("shapes must be q/o/dout [B,H,Nq,d], k/v [B,H,Nkv,d], lse [B,H,Nq]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    nbytes = fa_bwd_workspace_bytes(B, H, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    s = torch.cuda.current_stream(q.device) if stream is None else stream
+    with torch.cuda.device(q.device):
+        rc = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                    dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                    workspace.data_ptr(), workspace.numel() * workspace.element_size(), B, H, Nq,
+                    Nkv, d, scale, int(bool(causal)), s.cuda_stream, _dtype_code(q.dtype))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd")
+    return dq, dk, dv

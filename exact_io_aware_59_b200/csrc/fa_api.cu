@@ -77,12 +77,13 @@ int get_encoder() {
   return FA_OK;
 }
 
-// 3-D view (d, N, B*H) of a [B,H,N,d] tensor; box (64, 128, 1) with 128-byte swizzle.
-int make_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, bool bf16) {
+// 3-D view (d, N, B*H) of a [B,H,N,d] tensor; box (64, box_rows, 1) with 128-byte swizzle.
+int make_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, bool bf16,
+             unsigned box_rows = 128) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                         3, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -445,6 +446,92 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v, void* o, float* ls
   cudaError_t e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, v_dtype == FA_BF16,
                                      o_dtype == FA_F32, static_cast<int>(grid), ds->status,
                                      static_cast<cudaStream_t>(stream), true);
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+namespace {
+
+// Workspace layout of fa_bwd: -LSE*log2(e) [BH, nq_pad], D [BH, nq_pad], then the fp32
+// dQ accumulator [BH, nq_pad, 128]; nq_pad = Nq rounded up to 64 (each part a multiple of
+// 256 bytes).
+size_t bwd_ws_bytes(size_t BH, int Nq) {
+  const size_t nq_pad = (static_cast<size_t>(Nq) + 63) / 64 * 64;
+  return BH * nq_pad * (4 + 4 + 128 * 4);
+}
+
+}  // namespace
+
+int fa_bwd_workspace_bytes(int B, int H, int Nq, int d, size_t* bytes) {
+  if (!bytes || B < 1 || H < 1 || Nq < 1) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  *bytes = bwd_ws_bytes(static_cast<size_t>(B) * H, Nq);
+  return FA_OK;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, void* workspace,
+           size_t workspace_bytes, int B, int H, int Nq, int Nkv, int d, float scale,
+           int causal, void* stream, int in_dtype) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Nq < 1 || Nkv < 1) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (in_dtype != FA_F16 && in_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  const void* a16[9] = {q, k, v, o, dout, dq, dk, dv, workspace};
+  for (const void* ptr : a16)
+    if (!aligned(ptr, 16)) return FA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  const size_t BH = static_cast<size_t>(B) * H;
+  const size_t ws = bwd_ws_bytes(BH, Nq);
+  if (workspace_bytes < ws) return FA_ERR_INVALID_ARG;
+  const long long n_ktiles = (Nkv + 127) / 128, n_qtiles = (Nq + 63) / 64;
+  if (static_cast<long long>(BH) * n_ktiles > 0x7fffffffLL ||
+      static_cast<long long>(BH) * n_qtiles > 0x7fffffffLL)
+    return FA_ERR_INVALID_ARG;
+  const size_t qb = BH * Nq * d * 2, kb = BH * Nkv * d * 2, lb = BH * Nq * 4;
+  const void* outs[4] = {dq, dk, dv, workspace};
+  const size_t out_bytes[4] = {qb, kb, kb, ws};
+  const void* ins[6] = {q, k, v, o, dout, lse};
+  const size_t in_bytes[6] = {qb, kb, kb, qb, qb, lb};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 6; ++j)
+      if (overlaps(outs[i], out_bytes[i], ins[j], in_bytes[j])) return FA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlaps(outs[i], out_bytes[i], outs[j], out_bytes[j])) return FA_ERR_INVALID_ARG;
+  }
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+  const bool bf16 = in_dtype == FA_BF16;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((rc = make_map(&tq, q, Nq, static_cast<long long>(BH), d, bf16, 64)) != FA_OK) return rc;
+  if ((rc = make_map(&tdo, dout, Nq, static_cast<long long>(BH), d, bf16, 64)) != FA_OK) return rc;
+  if ((rc = make_map(&tk, k, Nkv, static_cast<long long>(BH), d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map(&tv, v, Nkv, static_cast<long long>(BH), d, bf16)) != FA_OK) return rc;
+  fa::BwdParams p{};
+  p.BH = static_cast<int>(BH);
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.off = Nkv - Nq;
+  p.causal = causal;
+  p.n_qtiles = static_cast<int>(n_qtiles);
+  p.nq_pad = p.n_qtiles * 64;
+  p.n_ktiles = static_cast<int>(n_ktiles);
+  p.scale = scale;
+  p.scale_log2 = scale_log2(scale);
+  float* w = static_cast<float*>(workspace);
+  p.nlse2 = w;
+  p.delta = w + BH * p.nq_pad;
+  p.dq_acc = w + 2 * BH * p.nq_pad;
+  p.dk = dk;
+  p.dv = dv;
+  cudaError_t e = fa::launch_backward(tq, tk, tv, tdo, o, dout, lse, dq, p, bf16, ds->sm_count,
+                                      ds->status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 

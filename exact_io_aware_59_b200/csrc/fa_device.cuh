@@ -16,6 +16,7 @@ enum : int {
   kStatusTimeoutSoftmax = 1 << 2,   // a softmax / epilogue wait ran out
   kStatusTimeoutDecode = 1 << 3,    // a split-KV decode wait ran out
   kStatusBadInput = 1 << 4,         // paged decode: table entry or length out of range
+  kStatusTimeoutBwd = 1 << 5,       // a backward-pass wait ran out
 };
 
 // A wait that has not finished after this long is treated as a hang.
@@ -156,6 +157,58 @@ __device__ __forceinline__ void bulk_load_stream(uint32_t dst, const void* src, 
       : "memory");
 }
 
+// Element-wise fp32 add of a contiguous shared-memory block into global memory, done by
+// the bulk-copy engine at L2 (16-byte aligned addresses, size a multiple of 16); tracked
+// by this thread's bulk async-group.
+__device__ __forceinline__ void bulk_reduce_add_f32(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until every committed bulk group of this thread has finished reading its shared
+// memory source.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until every committed bulk group of this thread is complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy reads
+// (TMA, bulk copies, tcgen05.mma operands).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Barrier among `count` threads (a multiple of 32) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// The same barrier, returning the AND of `pred` over the participating threads: a
+// decision every thread of the group then takes alike.
+__device__ __forceinline__ bool named_sync_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+// Contiguous global -> shared copy with the default L2 policy (data other CTAs re-read).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -231,6 +284,12 @@ __host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N, bool bf16, b
          | ((b_mn_major ? 1u : 0u) << 16)          // B major-ness
          | (static_cast<uint32_t>(N >> 3) << 17)   // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);  // M / 16
+}
+
+// As make_idesc_f16, with A MN-major as well when a_mn_major (A read from shared memory).
+__host__ __device__ constexpr uint32_t make_idesc_f16_ab(int M, int N, bool bf16, bool a_mn_major,
+                                                         bool b_mn_major) {
+  return make_idesc_f16(M, N, bf16, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
 }
 
 // Instruction descriptor for kind::f8f6f4 with fp32 accumulation, A and B both E4M3

@@ -27,6 +27,27 @@ struct PrefillParams {
   int total_q, total_k;
 };
 
+// Work description of one backward launch ([B,H,N,d] layout, d = 128).
+struct BwdParams {
+  int BH;
+  int Nq, Nkv;
+  int off;          // Nkv - Nq: causal query i sees keys j <= i + off
+  int causal;
+  int n_qtiles;     // ceil(Nq / 64)
+  int nq_pad;       // n_qtiles * 64: rows of the per-row workspace arrays
+  int n_ktiles;     // ceil(Nkv / 128): one CTA per (key tile, b*h)
+  float scale;
+  float scale_log2; // scale * log2(e)
+  // Workspace (written by the prep kernel): -LSE*log2(e) and D = rowsum(dO * O) per padded
+  // query row, and the fp32 dQ accumulator, one 128 x 64 tile (d-major, 16-byte chunks
+  // swizzled) per (b*h, query tile).
+  float* nlse2;
+  float* delta;
+  float* dq_acc;
+  void* dk;         // [BH, Nkv, 128], the inputs' 16-bit type
+  void* dv;
+};
+
 // Work description of one split-KV decode launch.
 struct DecodeParams {
   int BH;
@@ -61,6 +82,14 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
                           const DecodeParams& p, int d, bool bf16, bool o_f32, float* part_o,
                           float* part_lse, int* status, cudaStream_t stream,
                           const PagedKV* paged = nullptr);
+
+// Backward: prep, main and dQ-conversion kernels on `stream` (fa_backward.cu).  tq / tdo
+// are maps with 64-row boxes, tk / tv with 128-row boxes.
+cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const void* o, const void* dout,
+                            const float* lse, void* dq, const BwdParams& p, bool bf16,
+                            int sm_count, int* status, cudaStream_t stream);
+size_t backward_smem_bytes();
 
 // Diagnostic kernel whose only wait can never finish (see fa_selftest_wait_timeout).
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t stream);

@@ -204,6 +204,31 @@ int fa_fwd_decode_paged(const void* q, const void* k_cache, const void* v_cache,
                         int num_pages, float scale, void* stream, int in_dtype, int o_dtype,
                         int num_splits);
 
+/*
+ * fa_bwd -- gradients of fa_fwd for an upstream gradient dO ("Flash Attention -- Module
+ * 12.3", section "Prefill vs Decode", "Training": the backward pass is IO-aware too).
+ *   For O = softmax(scale * Q K^T [+ causal mask, bottom-right]) V and the forward's lse:
+ *     P = exp(scale * Q K^T - lse) (masked entries 0), D = rowsum(dO * O),
+ *     dV = P^T dO,  dS = P * (dO V^T - D),  dQ = scale * dS K,  dK = scale * dS^T Q.
+ *   P is recomputed on chip tile by tile; nothing of size Nq x Nkv is stored.
+ *   q, o, dout, dq [B,H,Nq,d]; k, v, dk, dv [B,H,Nkv,d]; all in_dtype (FA_F16 or FA_BF16),
+ *   contiguous, 16-byte aligned.  lse [B,H,Nq] fp32 natural log as fa_fwd writes it (a
+ *   row with no visible key has -inf and gets dQ = 0).  d must be 128.
+ *   workspace: caller-owned device memory of at least fa_bwd_workspace_bytes bytes,
+ *   16-byte aligned; overwritten (it holds the fp32 dQ accumulator and per-row D and lse).
+ *   dq, dk, dv and the workspace must not overlap each other or any input.
+ *   Enqueues three kernels on `stream` and returns FA_OK; no allocation, no
+ *   synchronisation.  Errors as for fa_fwd: a failed host check launches nothing; a
+ *   kernel wait that runs out sets FA_DEV_TIMEOUT_BACKWARD (outputs then undefined).
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, void* workspace,
+           size_t workspace_bytes, int B, int H, int Nq, int Nkv, int d, float scale,
+           int causal, void* stream, int in_dtype);
+
+/* Bytes of workspace an fa_bwd call with these sizes needs (B*H*ceil(Nq/64)*64*520). */
+int fa_bwd_workspace_bytes(int B, int H, int Nq, int d, size_t* bytes);
+
 /* Bytes of decode workspace a fa_fwd_decode call with these arguments needs. */
 int fa_decode_workspace_bytes(int B, int H, int Nkv, int d, int num_splits, size_t* bytes);
 
@@ -221,7 +246,8 @@ enum {
   FA_DEV_TIMEOUT_MMA = 2,       /* prefill: the MMA issuer's wait ran out */
   FA_DEV_TIMEOUT_SOFTMAX = 4,   /* prefill: a softmax / epilogue wait ran out */
   FA_DEV_TIMEOUT_DECODE = 8,    /* decode: a split kernel wait ran out */
-  FA_DEV_BAD_INPUT = 16         /* paged decode / varlen: a device-side table or offset out of range */
+  FA_DEV_BAD_INPUT = 16,        /* paged decode / varlen: a device-side table or offset out of range */
+  FA_DEV_TIMEOUT_BACKWARD = 32  /* fa_bwd: a kernel wait ran out */
 };
 
 /*

@@ -187,3 +187,33 @@ def test_fp8_entry_checks():
     assert call(vd=2) == binding.FA_ERR_INVALID_ARG          # V must be 16-bit
     assert call(vd=0, od=1) == binding.FA_ERR_UNSUPPORTED     # 16-bit O must be V's type
     assert call(k8=K + 8) == binding.FA_ERR_INVALID_ARG       # misaligned
+
+
+def test_backward_entry_checks():
+    """fa_bwd refuses bad arguments on the host, before touching any device."""
+    ws_ok = 1 * 1 * 64 * 520
+    args = dict(q=Q, k=K, v=V, o=O, lse=L, do=Q + 4096, dq=O + 4096, dk=O + 8192, dv=O + 12288,
+                ws=O + 65536, wsb=ws_ok, B=1, H=1, Nq=4, Nkv=4, d=128, scale=0.1, causal=0,
+                stream=None, dt=1)
+
+    def call(**kw):
+        a = dict(args)
+        a.update(kw)
+        return binding.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"],
+                              a["dv"], a["ws"], a["wsb"], a["B"], a["H"], a["Nq"], a["Nkv"],
+                              a["d"], a["scale"], a["causal"], a["stream"], a["dt"])
+
+    assert call(d=64) == binding.FA_ERR_UNSUPPORTED
+    assert call(lse=None) == binding.FA_ERR_INVALID_ARG
+    assert call(ws=None) == binding.FA_ERR_INVALID_ARG
+    assert call(wsb=ws_ok - 16) == binding.FA_ERR_INVALID_ARG   # workspace too small
+    assert call(Nq=0) == binding.FA_ERR_INVALID_ARG
+    assert call(causal=2) == binding.FA_ERR_INVALID_ARG
+    assert call(dt=2) == binding.FA_ERR_INVALID_ARG             # fp32 inputs
+    assert call(scale=math.nan) == binding.FA_ERR_INVALID_ARG
+    assert call(dk=O + 8200) == binding.FA_ERR_INVALID_ARG      # misaligned
+    assert call(dq=Q) == binding.FA_ERR_INVALID_ARG             # output overlaps an input
+    assert call(dv=O + 8192) == binding.FA_ERR_INVALID_ARG      # two outputs overlap
+    assert binding.fa_bwd_workspace_bytes(2, 3, 65, 128) == 2 * 3 * 128 * 520
+    with pytest.raises(binding.FaError):
+        binding.fa_bwd_workspace_bytes(1, 1, 64, 64)
