@@ -19,7 +19,7 @@
 //    contribution into the fp32 accumulator with one bulk reduce-add (done at L2);
 //  * fa_bwd_dq: dQ = scale * accumulator, converted to the inputs' 16-bit type.
 //
-// fa_bwd_sm100 roles (384 threads; our design for tcgen05, with keys as the MMA's M so the
+// fa_bwd_sm100 roles (512 threads; our design for tcgen05, with keys as the MMA's M so the
 // per-key sums dK and dV stay in TMEM for the whole walk):
 //  * warp 0 (one lane): TMA loads of K and V once, then Q, dO, -LSE*log2e and D of each
 //    query tile into a 3-stage ring;
@@ -29,17 +29,21 @@
 //        dV  += P^T dO_i  (A = P^T, 16-bit, from TMEM over S[b]; B = dO_i MN-major)
 //        dK  += dS^T Q_i  (A = dS^T, 16-bit, from TMEM over dP[b]; B = Q_i MN-major)
 //        dQ^T = K^T dS^T  (M 128 = d, N 64 queries, K 128 keys; A = K read MN-major,
-//                          B = dS[b] from shared memory)          into S[b], over P
-//    software-pipelined one tile deep: step i issues dP(i+1), dV(i), S(i+1), dK(i),
-//    dQ(i), so the tensor pipe has tile i+1's products to run while warpgroup 1 turns
-//    S(i+1) and dP(i+1) into P and dS, and no product waits on the one before it;
-//  * warpgroup 1 (warps 4-7), one thread per key: P^T from S^T, dS^T from dP^T, each
-//    written back to TMEM as 16-bit, dS also to shared memory; at the end the dK / dV
-//    epilogue;
-//  * warpgroup 2 (warps 8-11), one thread per d-row of dQ^T: TMEM -> registers -> shared
+//                          B = dS[b] from shared memory)          into dP[b], over dS^T
+//    software-pipelined one tile deep: step i issues S(i+1), dP(i+1), dV(i), dK(i), dQ(i);
+//    only dP(i+1) waits for dQ(i-1) to be read out of dP[(i+1) % 2], and S(i+1) runs
+//    meanwhile;
+//  * warpgroups 1 and 2 (warps 4-7 and 8-11) take the even and the odd query tiles, one
+//    thread per key: P^T from S^T and dS^T from dP^T, each written back to TMEM as 16-bit,
+//    dS also to shared memory.  Two of them keep the tensor pipe fed: one warpgroup's
+//    exponentials and products for a tile take longer than the tile's five MMAs.  At the
+//    end warpgroup 1 writes dV and warpgroup 2 writes scale * dK;
+//  * warpgroup 3 (warps 12-15), one thread per d-row of dQ^T: TMEM -> registers -> shared
 //    memory -> bulk reduce-add into the accumulator tile of query tile i.
+// Registers: the launch gives 128 per thread; warps 0-3 and 12-15 drop to kRegsSide and
+// warpgroups 1 and 2 rise to kRegsSoftmax (setmaxnreg).
 // TMEM (512 columns): dV [0,128) dK [128,256) S0 [256,320) S1 [320,384) dP0 [384,448)
-// dP1 [448,512); dQ(i) overwrites S[b] once dV(i) has read P(i) from it.  tcgen05.mma
+// dP1 [448,512); dQ(i) overwrites dP[b] once dK(i) has read dS^T(i) from it.  tcgen05.mma
 // operations run in issue order, so an MMA that overwrites columns an earlier MMA reads
 // as its A operand needs no wait in between.
 #include <cuda_bf16.h>
@@ -55,7 +59,11 @@ constexpr int kD = 128;        // head dimension
 constexpr int kBK = 128;       // keys per CTA (MMA M)
 constexpr int kBQ = 64;        // queries per step (MMA N of S^T, dP^T, dQ^T)
 constexpr int kStages = 3;     // Q / dO ring
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kRegsLaunch = 128;   // 65536 / 512
+constexpr int kRegsSide = 96;      // warps 0-3 and 12-15
+constexpr int kRegsSoftmax = 160;  // warps 4-11
+static_assert(256 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
 
 struct BwdCfg {
   static constexpr int kKOff = 0;                           // K tile, 2 x (128 rows x 128 B)
@@ -81,7 +89,8 @@ struct BwdCfg {
   static constexpr int kBarDQFull = kBarDSFull + 2;  // + buffer
   static constexpr int kBarDQEmpty = kBarDQFull + 2;
   static constexpr int kBarDone = kBarDQEmpty + 1;   // every MMA of the CTA complete
-  static constexpr int kNumBars = kBarDone + 1;
+  static constexpr int kBarFinished = kBarDone + 1;  // warps 4-15 done with TMEM
+  static constexpr int kNumBars = kBarFinished + 1;
   static constexpr int kTmemHolderOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemHolderOff + 4;
   static constexpr int kBytes = kAbortOff + 4;
@@ -200,12 +209,16 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
   }
   for (int i = 0; i < n && ok; ++i) {
     const int b = i & 1, nb = b ^ 1, st = i % kStages;
-    const bool next = i + 1 < n;
     const int st1 = (i + 1) % kStages;
-    // dP(i+1): dP[nb] was last read by dK(i-1) (issued earlier) and by warpgroup 1 before
-    // it signalled dS(i-1).
-    if (next) {
+    if (i + 1 < n) {
       if (!(ok = wait(C::kBarFull + st1, ((i + 1) / kStages) & 1))) break;
+      // S(i+1): S[nb] was last read by dV(i-1), issued earlier, and by warpgroup nb before
+      // it signalled P(i-1).
+      issue_st(kTS + nb * kBQ, k_desc, q_kmaj(st1));
+      tc_commit(bar_addr(bars, C::kBarSFull + nb));
+      // dP(i+1) into dP[nb], once dQ(i-1) has been read out of it.
+      if (i > 0 && !(ok = wait(C::kBarDQEmpty, (i - 1) & 1))) break;
+      tc_fence_after();
       issue_st(kTdP + nb * kBQ, v_desc, do_kmaj(st1));
       tc_commit(bar_addr(bars, C::kBarDPFull + nb));
     }
@@ -215,23 +228,16 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
     for (int kk = 0; kk < kBQ / 16; ++kk)
       mma_ts(tmem + kTdV, tmem + kTS + b * kBQ + kk * 8, do_mn(st) + ((kk * 2048) >> 4), idesc_kv,
              (i > 0 || kk > 0) ? 1u : 0u);
-    // S(i+1) into S[nb], once dQ(i-1) has been read out of it.
-    if (next) {
-      if (i > 0 && !(ok = wait(C::kBarDQEmpty, (i - 1) & 1))) break;
-      tc_fence_after();
-      issue_st(kTS + nb * kBQ, k_desc, q_kmaj(st1));
-      tc_commit(bar_addr(bars, C::kBarSFull + nb));
-    }
     if (!(ok = wait(C::kBarDSFull + b, (i >> 1) & 1))) break;
     tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < kBQ / 16; ++kk)
       mma_ts(tmem + kTdK, tmem + kTdP + b * kBQ + kk * 8, q_mn(st) + ((kk * 2048) >> 4), idesc_kv,
              (i > 0 || kk > 0) ? 1u : 0u);
-    // dQ(i) over S[b]: P(i) there has been read by dV(i), issued above.
+    // dQ(i) over dP[b]: dS^T(i) there has been read by dK(i), issued above.
 #pragma unroll
     for (int kk = 0; kk < kBK / 16; ++kk)
-      mma_ss(tmem + kTS + b * kBQ, kt_desc + ((kk * 2048) >> 4), ds_desc(b) + ((kk * 2048) >> 4),
+      mma_ss(tmem + kTdP + b * kBQ, kt_desc + ((kk * 2048) >> 4), ds_desc(b) + ((kk * 2048) >> 4),
              idesc_q, kk > 0 ? 1u : 0u);
     tc_commit(bar_addr(bars, C::kBarDQFull + b));
     tc_commit(bar_addr(bars, C::kBarEmpty + st));  // Q_i, dO_i, LSE_i, D_i consumed
@@ -240,9 +246,10 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
 }
 
 // ---------------------------------------------------------------- P and dS (one thread per key)
+// Warpgroup `wg` (0 or 1) takes query tiles i = wg, wg + 2, ... and buffers [wg].
 template <bool BF16>
-__device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, uint8_t* sgen,
-                             uint32_t sbase, uint32_t bars, uint32_t tmem, int* status,
+__device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, int wg,
+                             uint8_t* sgen, uint32_t bars, uint32_t tmem, int* status,
                              volatile int* abort_flag) {
   using C = BwdCfg;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -259,8 +266,8 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
     return __all_sync(0xffffffffu, ok);
   };
   bool ok = true;
-  for (int i = 0; i < n; ++i) {
-    const int buf = i & 1, st = i % kStages;
+  for (int i = wg; i < n; i += 2) {
+    const int buf = wg, st = i % kStages;
     const int q0 = (i0 + i) * kBQ;
     if (!(ok = wait(C::kBarFull + st, (i / kStages) & 1))) break;  // LSE_i and D_i visible
     if (!(ok = wait(C::kBarSFull + buf, (i >> 1) & 1))) break;
@@ -348,8 +355,8 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
   if (n > 0 && !have) return;
   if (have) tc_fence_after();
   const size_t orow = (static_cast<size_t>(bh) * p.Nkv + kidx) * kD;
-#pragma unroll 1
-  for (int which = 0; which < 2; ++which) {
+  {
+    const int which = wg;  // warpgroup 1 writes dV, warpgroup 2 writes dK
     uint16_t* dst = static_cast<uint16_t*>(which ? p.dk : p.dv) + orow;
     const float mul = which ? p.scale : 1.f;
 #pragma unroll 1
@@ -386,7 +393,7 @@ __device__ void dq_drain(const BwdParams& p, int bh, int i0, int n, uint8_t* sge
   const int wq = warp & 3;
   const int t = wq * 32 + lane;  // d row of dQ^T = TMEM lane
   const bool leader = (t == 0);
-  const uint32_t tq0 = tmem + (static_cast<uint32_t>(wq * 32) << 16) + kTS;
+  const uint32_t tq0 = tmem + (static_cast<uint32_t>(wq * 32) << 16) + kTdP;
   uint8_t* stg_row = sgen + C::kStgOff + t * (kBQ * 4);
   for (int i = 0; i < n; ++i) {
     if (leader) bulk_wait_read_all();  // the previous tile's reduce has read the staging
@@ -451,15 +458,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_addr(bars, C::kBarSFull + b), 1);
-      mbar_init(bar_addr(bars, C::kBarPFull + b), 4);  // one arrival per warp of warpgroup 1
+      mbar_init(bar_addr(bars, C::kBarPFull + b), 4);  // one arrival per warp of warpgroup b+1
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_addr(bars, C::kBarDPFull + b), 1);
       mbar_init(bar_addr(bars, C::kBarDSFull + b), 4);
       mbar_init(bar_addr(bars, C::kBarDQFull + b), 1);
     }
-    mbar_init(bar_addr(bars, C::kBarDQEmpty), 4);    // one arrival per warp of warpgroup 2
+    mbar_init(bar_addr(bars, C::kBarDQEmpty), 4);    // one arrival per warp of warpgroup 3
     mbar_init(bar_addr(bars, C::kBarDone), 1);
+    mbar_init(bar_addr(bars, C::kBarFinished), 12);  // one per warp of warps 4-15
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -478,25 +486,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
-    if (lane == 0 && n > 0) producer(&tq, &tk, &tv, &tdo, p, bh, k0, i0, n, sbase, bars, status, abort_flag);
+  // Each role runs to the end of the kernel on its own path: warps with different
+  // register budgets never re-join.
+  if (warp < 4 || warp >= 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
+    if (warp == 0) {
+      if (lane == 0 && n > 0) producer(&tq, &tk, &tv, &tdo, p, bh, k0, i0, n, sbase, bars, status, abort_flag);
+    } else if (warp == 1) {
+      if (lane == 0) mma_issuer<BF16>(n, sbase, bars, tmem, status, abort_flag);
+      __syncwarp();
+      // Release TMEM once every MMA is complete and warps 4-15 are done with it.
+      drain_wait(bar_addr(bars, C::kBarFinished), 0);
+      drain_wait(bar_addr(bars, C::kBarDone), 0);
+      __syncwarp();
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    } else if (warp >= 12) {
+      dq_drain(p, bh, i0, n, sgen, sbase, bars, tmem, status, abort_flag);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarFinished));
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    softmax_grad<BF16>(p, bh, k0, i0, n, (warp - 4) >> 2, sgen, bars, tmem, status, abort_flag);
+    tc_fence_before();
     __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) mma_issuer<BF16>(n, sbase, bars, tmem, status, abort_flag);
-    __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    softmax_grad<BF16>(p, bh, k0, i0, n, sgen, sbase, bars, tmem, status, abort_flag);
-  } else if (warp >= 8) {
-    dq_drain(p, bh, i0, n, sgen, sbase, bars, tmem, status, abort_flag);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    // Every MMA must be complete before its columns are released.
-    drain_wait(bar_addr(bars, C::kBarDone), 0);
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarFinished));
   }
 }
 
@@ -585,6 +601,13 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   static cudaError_t config_err = cudaSuccess;
   if (!configured) {
     config_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg::kAlloc);
+    if (config_err == cudaSuccess) {
+      cudaFuncAttributes attr;
+      config_err = cudaFuncGetAttributes(&attr, kern);
+      // setmaxnreg redistributes the registers the block was launched with; a launch
+      // with fewer would make the increase wait forever.
+      if (config_err == cudaSuccess && attr.numRegs < kRegsLaunch) config_err = cudaErrorInvalidConfiguration;
+    }
     configured = true;
   }
   if (config_err != cudaSuccess) return config_err;
