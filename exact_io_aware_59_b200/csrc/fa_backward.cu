@@ -30,9 +30,12 @@
 //        dK  += dS^T Q_i  (A = dS^T, 16-bit, from TMEM over dP[b]; B = Q_i MN-major)
 //        dQ^T = K^T dS^T  (M 128 = d, N 64 queries, K 128 keys; A = K read MN-major,
 //                          B = dS[b] from shared memory)          into dP[b], over dS^T
-//    software-pipelined one tile deep: step i issues S(i+1), dP(i+1), dV(i), dK(i), dQ(i);
-//    only dP(i+1) waits for dQ(i-1) to be read out of dP[(i+1) % 2], and S(i+1) runs
-//    meanwhile;
+//    software-pipelined one tile deep: step i issues S(i+1), dP(i+1), then dV(i), dK(i),
+//    dQ(i) once warpgroup b has delivered P(i) and dS(i); only dP(i+1) waits for dQ(i-1)
+//    to be read out of dP[(i+1) % 2], and S(i+1) runs meanwhile.  The MMA lane is the
+//    critical path (the tensor pipe's issue queue is shallow), so a tile costs it just
+//    three waits and two commits: one commit covers S and dP, one covers the tile's last
+//    product (its dQ is then ready and its Q/dO stage free);
 //  * warpgroups 1 and 2 (warps 4-7 and 8-11) take the even and the odd query tiles, one
 //    thread per key: P^T from S^T and dS^T from dP^T, each written back to TMEM as 16-bit,
 //    dS also to shared memory.  Two of them keep the tensor pipe fed: one warpgroup's
@@ -81,10 +84,7 @@ struct BwdCfg {
   // mbarriers
   static constexpr int kBarKV = 0;
   static constexpr int kBarFull = 1;                 // + stage
-  static constexpr int kBarEmpty = 1 + kStages;      // + stage
-  static constexpr int kBarSFull = 1 + 2 * kStages;  // + buffer
-  static constexpr int kBarPFull = kBarSFull + 2;    // + buffer
-  static constexpr int kBarDPFull = kBarPFull + 2;   // + buffer
+  static constexpr int kBarDPFull = 1 + kStages;     // + buffer: S(i) and dP(i) complete
   static constexpr int kBarDSFull = kBarDPFull + 2;  // + buffer
   static constexpr int kBarDQFull = kBarDSFull + 2;  // + buffer
   static constexpr int kBarDQEmpty = kBarDQFull + 2;
@@ -144,9 +144,10 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
   bool ok = true;
   for (int i = 0; i < n; ++i) {
     const int st = i % kStages;
-    if (i >= kStages &&
-        !mbar_wait(bar_addr(bars, C::kBarEmpty + st), ((i / kStages) & 1) ^ 1, status, abort_flag,
-                   kStatusTimeoutBwd)) {
+    // The stage held tile i - 3, whose products are all complete once its dQ is.
+    const int prev = i - kStages;
+    if (prev >= 0 && !mbar_wait(bar_addr(bars, C::kBarDQFull + (prev & 1)), (prev >> 1) & 1, status,
+                                abort_flag, kStatusTimeoutBwd)) {
       ok = false;
       break;
     }
@@ -202,10 +203,9 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
   };
   bool ok = n > 0 && wait(C::kBarKV, 0);  // with no query tile nothing is loaded
   if (ok && (ok = wait(C::kBarFull + 0, 0))) {
+    issue_st(kTS, k_desc, q_kmaj(0));
     issue_st(kTdP, v_desc, do_kmaj(0));
     tc_commit(bar_addr(bars, C::kBarDPFull + 0));
-    issue_st(kTS, k_desc, q_kmaj(0));
-    tc_commit(bar_addr(bars, C::kBarSFull + 0));
   }
   for (int i = 0; i < n && ok; ++i) {
     const int b = i & 1, nb = b ^ 1, st = i % kStages;
@@ -213,23 +213,21 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
     if (i + 1 < n) {
       if (!(ok = wait(C::kBarFull + st1, ((i + 1) / kStages) & 1))) break;
       // S(i+1): S[nb] was last read by dV(i-1), issued earlier, and by warpgroup nb before
-      // it signalled P(i-1).
+      // it signalled dS(i-1).
       issue_st(kTS + nb * kBQ, k_desc, q_kmaj(st1));
-      tc_commit(bar_addr(bars, C::kBarSFull + nb));
       // dP(i+1) into dP[nb], once dQ(i-1) has been read out of it.
       if (i > 0 && !(ok = wait(C::kBarDQEmpty, (i - 1) & 1))) break;
       tc_fence_after();
       issue_st(kTdP + nb * kBQ, v_desc, do_kmaj(st1));
-      tc_commit(bar_addr(bars, C::kBarDPFull + nb));
+      tc_commit(bar_addr(bars, C::kBarDPFull + nb));  // S(i+1) and dP(i+1)
     }
-    if (!(ok = wait(C::kBarPFull + b, (i >> 1) & 1))) break;
+    // Warpgroup b has stored P(i) over S[b] and dS^T(i) over dP[b], and dS(i) in shared memory.
+    if (!(ok = wait(C::kBarDSFull + b, (i >> 1) & 1))) break;
     tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < kBQ / 16; ++kk)
       mma_ts(tmem + kTdV, tmem + kTS + b * kBQ + kk * 8, do_mn(st) + ((kk * 2048) >> 4), idesc_kv,
              (i > 0 || kk > 0) ? 1u : 0u);
-    if (!(ok = wait(C::kBarDSFull + b, (i >> 1) & 1))) break;
-    tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < kBQ / 16; ++kk)
       mma_ts(tmem + kTdK, tmem + kTdP + b * kBQ + kk * 8, q_mn(st) + ((kk * 2048) >> 4), idesc_kv,
@@ -239,8 +237,8 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
     for (int kk = 0; kk < kBK / 16; ++kk)
       mma_ss(tmem + kTdP + b * kBQ, kt_desc + ((kk * 2048) >> 4), ds_desc(b) + ((kk * 2048) >> 4),
              idesc_q, kk > 0 ? 1u : 0u);
+    // Tile i's products are complete: its dQ can be drained and its stage reloaded.
     tc_commit(bar_addr(bars, C::kBarDQFull + b));
-    tc_commit(bar_addr(bars, C::kBarEmpty + st));  // Q_i, dO_i, LSE_i, D_i consumed
   }
   tc_commit(bar_addr(bars, C::kBarDone));
 }
@@ -270,7 +268,7 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
     const int buf = wg, st = i % kStages;
     const int q0 = (i0 + i) * kBQ;
     if (!(ok = wait(C::kBarFull + st, (i / kStages) & 1))) break;  // LSE_i and D_i visible
-    if (!(ok = wait(C::kBarSFull + buf, (i >> 1) & 1))) break;
+    if (!(ok = wait(C::kBarDPFull + buf, (i >> 1) & 1))) break;  // S(i) and dP(i)
     tc_fence_after();
     const uint32_t tS = lane_base + kTS + buf * kBQ;
     float pr[64];
@@ -305,12 +303,9 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
       tmem_st_32x32b_x32(tS, pk);
     }
     tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarPFull + buf));
-
-    if (!(ok = wait(C::kBarDPFull + buf, (i >> 1) & 1))) break;
-    tc_fence_after();
+    // A block boundary between the P pass and the dS pass (ok is true here): interleaving
+    // the two needs more registers than this warpgroup's 160 and spills.
+    if (!__all_sync(0xffffffffu, ok)) break;
     const float4* dl = reinterpret_cast<const float4*>(sgen + C::kDelOff + st * kBQ * 4);
     uint8_t* ds_row = sgen + C::kdSOff + buf * C::kdSBytes + r * 128;
     const uint32_t tdP = lane_base + kTdP + buf * kBQ;
@@ -452,17 +447,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_addr(bars, C::kBarKV), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar_addr(bars, C::kBarFull + s), 1);
-      mbar_init(bar_addr(bars, C::kBarEmpty + s), 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_addr(bars, C::kBarSFull + b), 1);
-      mbar_init(bar_addr(bars, C::kBarPFull + b), 4);  // one arrival per warp of warpgroup b+1
-    }
+    for (int s = 0; s < kStages; ++s) mbar_init(bar_addr(bars, C::kBarFull + s), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_addr(bars, C::kBarDPFull + b), 1);
-      mbar_init(bar_addr(bars, C::kBarDSFull + b), 4);
+      mbar_init(bar_addr(bars, C::kBarDSFull + b), 4);  // one arrival per warp of warpgroup b+1
       mbar_init(bar_addr(bars, C::kBarDQFull + b), 1);
     }
     mbar_init(bar_addr(bars, C::kBarDQEmpty), 4);    // one arrival per warp of warpgroup 3
