@@ -60,7 +60,7 @@ extern "C" {
 enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, misalignment, overlap, ... */
-  FA_ERR_UNSUPPORTED = 2,     /* valid request this build does not implement (d, dtype pair) */
+  FA_ERR_UNSUPPORTED = 2,     /* valid request the library does not implement (d, dtype pair) */
   FA_ERR_ARCH = 3,            /* current device is not compute capability 10.0 (B200) */
   FA_ERR_CUDA = 4,            /* a CUDA runtime call failed: see fa_last_cuda_error() */
   FA_ERR_NOMEM = 5,           /* a library-owned allocation failed */
