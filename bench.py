@@ -445,7 +445,10 @@ def arm_ours(args, ws, rank, local):
             "value": whole_job_rate(flops_b, ms_b, ws) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": ms_b, "steps": bsteps, "gpu_launches": 3 * bsteps,
             "roofline": {"bound": "tensor", "achieved": tf_b, "peak": peak_t, "unit": "TFLOP/s",
-                         "frac": tf_b / peak_t, "traffic": None, "peak_source": peak_src,
+                         "frac": tf_b / peak_t,
+                         "traffic": BWD_TRAFFIC.get((BWD_REV, wp.name)),
+                         "traffic_kernel": "fa_bwd_sm100 (main kernel, 94.5% of the call)",
+                         "peak_source": peak_src,
                          "flops_per_launch": flops_b,
                          "note": "achieved over the whole call (prep, main and dQ kernels)"},
             "clocks": clk_b.summary(),
@@ -564,6 +567,12 @@ def arm_ours(args, ws, rank, local):
         }
         print(json.dumps(line), flush=True)
 
+
+# Bumped whenever the backward main kernel changes, so stale ncu traffic is not reported.
+BWD_REV = "backward-v4"
+# dram__bytes_read.sum + dram__bytes_write.sum of one fa_bwd_sm100 launch at full size
+# (ncu, 1 pass; profiles/fa_bwd_sm100_long_prefill_causal.md).
+BWD_TRAFFIC = {(BWD_REV, "long_prefill_causal"): 626.3e6}
 
 # Bumped whenever the prefill kernel changes, so stale ncu traffic is not reported.
 KERNEL_REV = "prefill-v21"
