@@ -38,9 +38,10 @@
 //    product (its dQ is then ready and its Q/dO stage free);
 //  * warpgroups 1 and 2 (warps 4-7 and 8-11) take the even and the odd query tiles, one
 //    thread per key: P^T from S^T and dS^T from dP^T, each written back to TMEM as 16-bit,
-//    dS also to shared memory.  Two of them keep the tensor pipe fed: one warpgroup's
-//    exponentials and products for a tile take longer than the tile's five MMAs.  At the
-//    end warpgroup 1 writes dV and warpgroup 2 writes scale * dK;
+//    dS also to shared memory.  With two, each has two tiles' time for one tile's work,
+//    so P(i) and dS(i) are ready before the MMA lane asks for them (one warpgroup alone
+//    measured about as fast, the MMA lane being the critical path).  At the end
+//    warpgroup 1 writes dV and warpgroup 2 writes scale * dK;
 //  * warpgroup 3 (warps 12-15), one thread per d-row of dQ^T: TMEM -> registers -> shared
 //    memory -> bulk reduce-add into the accumulator tile of query tile i.
 // Registers: the launch gives 128 per thread; warps 0-3 and 12-15 drop to kRegsSide and
