@@ -39,3 +39,11 @@ def test_flops_of_the_headline_shape():
 def test_backward_is_two_and_a_half_forwards():
     w = Workload("x", 9, 2, 3, 37, 53, 64, torch.bfloat16, True)
     assert 2 * bench.backward_flops(w) == 5 * bench.attention_flops(w)
+
+
+def test_decode_algorithmic_bytes():
+    """Q, K, V read once and O (16-bit) and LSE written once: the decode roofline's unit."""
+    w = WORKLOADS["decode"]
+    BH = 16 * 32
+    expect = BH * (128 * 2 + 2 * 32768 * 128 * 2 + 128 * 2 + 4)
+    assert bench.algorithmic_bytes(w, 2) == expect == 8590198784
