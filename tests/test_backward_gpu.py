@@ -75,6 +75,7 @@ CASES = [
     (1, 2, 300, 130, True, torch.bfloat16),     # Nq > Nkv: the first rows see no key
     (1, 1, 1, 1, False, torch.bfloat16),        # one query, one key
     (1, 1, 64, 1000, False, torch.float16),     # one query tile, many key tiles
+    (1, 2, 192, 320, True, torch.float16),      # fp16 with the bottom-right diagonal
 ]
 
 
