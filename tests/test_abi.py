@@ -217,3 +217,25 @@ def test_backward_entry_checks():
     assert binding.fa_bwd_workspace_bytes(2, 3, 65, 128) == 2 * 3 * 128 * 520
     with pytest.raises(binding.FaError):
         binding.fa_bwd_workspace_bytes(1, 1, 64, 64)
+
+
+def _declared_param_counts():
+    """Parameter count of every function include/fa.h declares."""
+    import re
+    text = open(binding.HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.M | re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else len(params.split(","))
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature has as many arguments as the C declaration (a binding that
+    drifted from the header would pass garbage silently)."""
+    counts = _declared_param_counts()
+    assert set(counts) == set(binding.declared_functions())
+    for name, argtypes in binding._SIGNATURES.items():
+        assert name in counts, name
+        assert len(argtypes) == counts[name], (name, len(argtypes), counts[name])
