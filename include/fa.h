@@ -1,6 +1,7 @@
 /*
- * fa.h -- C ABI of libfa_b200.so: exact fused scaled-dot-product attention forward on
- * NVIDIA B200 (sm_100a).
+ * fa.h -- C ABI of libfa_b200.so: exact fused scaled-dot-product attention on NVIDIA
+ * B200 (sm_100a): the forward (prefill, decode, paged decode, packed varlen, FP8 Q/K) and
+ * the backward (fa_bwd).
  *
  * What is computed ("Flash Attention -- Module 12.3" (aicurriculum), section
  * "Definition": exact softmax(Q K^T / sqrt(d)) V; "FlashAttention" (fp-ai-systems),
@@ -45,7 +46,9 @@
  * undefined.  Read (and clear) that word with fa_device_status() after synchronising.
  *
  * Determinism: tile sizes, the CTA count and the split partition depend only on the
- * shape and the device, so equal inputs give bitwise-equal outputs.
+ * shape and the device, so equal inputs give bitwise-equal outputs.  The one exception
+ * is fa_bwd's dQ, summed in fp32 across key tiles in arrival order (its dK and dV are
+ * bitwise reproducible).
  */
 #ifndef FA_B200_H_
 #define FA_B200_H_
