@@ -1,23 +1,27 @@
 """Benchmark of the exact attention forward on B200: prefill TFLOP/s and decode HBM GB/s.
 
-One step = one pass of the hot path over one batch of synthetic input:
-  * the headline line times the long causal prefill (B=1, H=32, N=8192, d=128, bf16), one
-    fa_fwd call per step;
-  * the "decode" object times the split-KV decode (B=16, H=32, Nq=1, Nkv=32768, d=128,
-    bf16), one fa_fwd call (split kernel + combine kernel) per step;
-  * the "decode_paged" object times the same decode against a paged KV cache (64-key
-    pages scattered over the pool by a seeded random block table), one
-    fa_fwd_decode_paged call per step;
-  * the "prefill_fp8" object times the headline shape with Q and K in E4M3, one
-    fa_fwd_fp8 call per step;
-  * the "backward" object times the gradients (dQ, dK, dV) of the headline shape from its
-    O and LSE and a seeded dO, one fa_bwd call (prep, main and dQ kernels) per step;
-  * the "prefill_varlen" object times a packed ragged causal batch (16 sequences,
-    seeded log-uniform lengths in [512, 8192], H=32, d=128, bf16), one fa_fwd_varlen
-    call per step.
-Inputs are resident in HBM and larger than L2 (126 MB) when the timed region starts.
+One step = one pass of the hot path over one batch of synthetic input.  The headline
+("value", "roofline") times the long causal prefill (B=1, H=32, N=8192, d=128, bf16, bf16
+O), one fa_fwd call per step.  The "configs" object, last in the line, gives every other
+configuration one compact record (value, unit, ms_per_step, roofline fraction of the
+measured burst peak "frac" and of the sustained peak "frac_sus", median SM clock); each is
+timed for the line's own "steps":
+  mha_d64       B=2 H=8 N=2048 d=64 fp16 causal (fa_fwd)
+  noncausal_8k  B=1 H=32 N=8192 d=128 bf16 non-causal
+  peaky_8k      the headline shape with Q drawn with std 4
+  causal_16k    B=1 H=16 N=16384 d=128 bf16 causal
+  causal_32k    B=1 H=16 N=32768 d=128 bf16 causal
+  decode        B=16 H=32 Nq=1 Nkv=32768 d=128 bf16, split-KV decode (HBM GB/s)
+  decode_paged  the decode shape in a paged cache of 64-key pages (fa_fwd_decode_paged)
+  fp8_8k        the headline shape with E4M3 Q and K (fa_fwd_fp8; peak: 4/3 of bf16)
+  bwd_8k        dQ, dK, dV of the headline shape (fa_bwd; 10*d FLOP per visible pair)
+  varlen        a packed causal batch of 16 sequences, lengths log-uniform in [512, 8192]
+Every configuration is timed for the same --steps.  Inputs are resident in HBM when the
+timed region starts; a configuration whose inputs fit in L2 (126 MB) cycles through enough
+copies of them that consecutive steps never find them there.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--skip-extra] [--detail out.json]
 
 Multi-GPU (N > 1, one process per GPU via torch.distributed.run): every rank runs the
 same independent problem (heads are independent; no collective on the data path);
@@ -223,17 +227,6 @@ def make_call(w: Workload, q, k, v, o, lse, stream):
     return call
 
 
-def run_workload(w: Workload, steps, warmup, ws, stream, out_dtype=None):
-    q, k, v = workload_qkv(w, device="cuda")
-    out_dtype = w.dtype if out_dtype is None else out_dtype
-    o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=out_dtype, device="cuda")
-    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device="cuda")
-    call = make_call(w, q, k, v, o, lse, stream)
-    with torch.cuda.stream(stream):
-        ms = time_steps(call, steps, warmup, ws, stream)
-    return ms, (q, k, v, o, lse)
-
-
 def run_e2e(w: Workload, tensors, steps, warmup, ws, stream):
     """The same call with pinned HOST inputs: per step, copy Q/K/V host->device, run,
     copy O and LSE device->host; all inside the timed region."""
@@ -328,58 +321,144 @@ def arm_reference(args, ws, rank):
 
 
 def workload_config(w: Workload, o_dtype: str):
-    return {"workload": f"{w.name}: B={w.B} H={w.H} Nq={w.Nq} Nkv={w.Nkv} d={w.d} "
-                        f"{str(w.dtype).replace('torch.', '')} causal={w.causal}",
-            "B": w.B, "H": w.H, "Nq": w.Nq, "Nkv": w.Nkv, "d": w.d, "causal": w.causal,
+    return {"workload": w.name, "B": w.B, "H": w.H, "Nq": w.Nq, "Nkv": w.Nkv, "d": w.d,
+            "causal": w.causal, "in_dtype": str(w.dtype).replace("torch.", ""),
             "o_dtype": o_dtype, "parallelism": "independent problem per GPU",
             "l2": "inputs larger than L2 (no flush)"}
+
+
+L2_BYTES = 126 * 1024 * 1024
+
+
+def r4(x):
+    """x to 4 significant digits (keeps the JSON line short)."""
+    if x is None:
+        return None
+    return float(f"{x:.4g}")
+
+
+def timed(calls, steps, warmup, ws, stream, local):
+    """Times `steps` steps that cycle through `calls` (one call per step); returns
+    (ms per step, clock summary).  Every call's kernel waits are checked afterwards."""
+    state = {"i": 0}
+
+    def step():
+        calls[state["i"] % len(calls)]()
+        state["i"] += 1
+
+    with ClockSampler(local) as clk, torch.cuda.stream(stream):
+        ms = time_steps(step, steps, warmup, ws, stream)
+    assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+    return ms, clk.summary()
+
+
+def compact(value, unit, ms, steps, frac, frac_sus, clk):
+    """One record of the per-config object: the rate, its time, its roofline fractions."""
+    del steps  # every configuration is timed for the line's own "steps"
+    d = {"value": r4(value), "unit": unit, "ms_per_step": r4(ms), "frac": r4(frac)}
+    if frac_sus is not None:
+        d["frac_sus"] = r4(frac_sus)
+    if clk:
+        d["sm_mhz"] = int(round(clk["sm_mhz"]))
+        if clk["reasons"]:
+            d["reasons"] = clk["reasons"]
+    return d
+
+
+def input_sets(w: Workload, out_dtype):
+    """Enough copies of the workload's inputs and outputs that one pass over them is larger
+    than L2 (one copy when a single one already is): consecutive steps then never find
+    their operands in L2.  Returns (list of (q, k, v, o, lse), bytes per copy)."""
+    per = (w.B * w.H * (w.Nq + 2 * w.Nkv) * w.d * 2
+           + w.B * w.H * w.Nq * (w.d * torch.empty((), dtype=out_dtype).element_size() + 4))
+    n = 1 if per > L2_BYTES else min(64, -(-2 * L2_BYTES // per))
+    sets = []
+    for _ in range(n):
+        q, k, v = workload_qkv(w, device="cuda")
+        o = torch.empty((w.B, w.H, w.Nq, w.d), dtype=out_dtype, device="cuda")
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device="cuda")
+        sets.append((q, k, v, o, lse))
+    return sets, per
+
+
+def prefill_record(w: Workload, args, ws, stream, local, peaks):
+    """Times one fa_fwd per step on workload w (16-bit O); returns (compact record, ms,
+    TFLOP/s of one GPU, clocks, the first input set)."""
+    sets, _ = input_sets(w, w.dtype)
+    calls = [make_call(w, *t, stream) for t in sets]
+    ms, clk = timed(calls, args.steps, args.warmup, ws, stream, local)
+    flops = attention_flops(w)
+    tf = flops / (ms * 1e-3) / 1e12
+    rec = compact(whole_job_rate(flops, ms, ws) / 1e12, "TFLOP/s", ms, args.steps,
+                  tf / peaks["bf16_tflops"],
+                  tf / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), clk)
+    return rec, ms, tf, clk, sets[0]
 
 
 def arm_ours(args, ws, rank, local):
     torch.cuda.set_device(local)
     stream = torch.cuda.Stream()
     peaks, peak_src = load_peaks()
-    out_dtype = None  # O in the inputs' 16-bit type
-
-    # prefill (headline)
-    wp = WORKLOADS[args.prefill_workload]
-    with ClockSampler(local) as clk:
-        ms_p, tensors = run_workload(wp, args.steps, args.warmup, ws, stream, out_dtype)
-    assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
-    flops = attention_flops(wp)
-    tflops = flops / (ms_p * 1e-3) / 1e12
-    value = whole_job_rate(flops, ms_p, ws) / 1e12
     peak_t = peaks["bf16_tflops"]
+    peak_sus = peaks.get("bf16_tflops_sustained", peak_t)
+    configs = {}
+    detail = {}
+
+    # prefill (headline): long causal, 16-bit O
+    wp = WORKLOADS[args.prefill_workload]
+    _, ms_p, tflops, clk, tensors = prefill_record(wp, args, ws, stream, local, peaks)
+    flops = attention_flops(wp)
+    value = whole_job_rate(flops, ms_p, ws) / 1e12
     traffic = DRAM_TRAFFIC.get((KERNEL_REV, wp.name))
 
-    # decode
-    decode = None
-    if not args.skip_decode:
+    if not args.skip_extra:
+        # the other prefill configurations of the same kernel
+        for key, name in (("mha_d64", "prefill_mha"), ("noncausal_8k", "long_prefill"),
+                          ("peaky_8k", "long_prefill_peaky"), ("causal_16k", "long_ctx_16k"),
+                          ("causal_32k", "long_ctx_32k")):
+            if name == wp.name:
+                continue
+            rec, ms, _, _, first = prefill_record(WORKLOADS[name], args, ws, stream, local,
+                                                  peaks)
+            configs[key] = rec
+            del first
+            torch.cuda.empty_cache()
+
+        # split-KV decode (HBM bound): one fa_fwd (split + combine kernels) per step
         wd = WORKLOADS[args.decode_workload]
-        dsteps = max(3, args.steps // 8)
-        with ClockSampler(local) as clk_d:
-            ms_d, dt_ = run_workload(wd, dsteps, args.warmup, ws, stream, out_dtype)
-        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
-        del dt_
+        sets, _ = input_sets(wd, wd.dtype)
+        ms_d, clk_d = timed([make_call(wd, *t, stream) for t in sets], args.steps, args.warmup,
+                            ws, stream, local)
+        del sets
         bytes_d = algorithmic_bytes(wd, 2)
         gbs = bytes_d / (ms_d * 1e-3) / 1e9
-        decode = {
-            "workload": workload_config(wd, "bf16")["workload"],
-            "value": whole_job_rate(bytes_d, ms_d, ws) / 1e9,
-            "unit": "GB/s", "ms_per_step": ms_d, "steps": dsteps,
-            "gpu_launches": 2 * dsteps,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                         "traffic": DECODE_TRAFFIC.get((DECODE_REV, wd.name)),
-                         "peak_source": peak_src,
-                         "algorithmic_bytes_per_launch": bytes_d},
-            "clocks": clk_d.summary(),
-        }
+        configs["decode"] = compact(whole_job_rate(bytes_d, ms_d, ws) / 1e9, "GB/s", ms_d,
+                                    args.steps, gbs / peaks["hbm_gbs"], None, clk_d)
+        detail["decode"] = {"algorithmic_bytes_per_launch": bytes_d, "gpu_launches": 2 * args.steps,
+                            "traffic": DECODE_TRAFFIC.get((DECODE_REV, wd.name))}
         torch.cuda.empty_cache()
 
-    # prefill with E4M3 queries and keys (the headline shape)
-    prefill_fp8 = None
-    if not args.skip_decode:
+        # decode against a paged KV cache (same shape): 64-key pages, seeded random table
+        ps = 64
+        pq, kc, vc, table, sl = paged_decode_inputs(wd.B, wd.H, wd.Nkv, wd.d, ps, wd.dtype,
+                                                    1000 * wd.index + 500, device="cuda")
+        po = torch.empty((wd.B, wd.H, wd.d), dtype=wd.dtype, device="cuda")
+        pl = torch.empty((wd.B, wd.H), dtype=torch.float32, device="cuda")
+        pargs = (pq.data_ptr(), kc.data_ptr(), vc.data_ptr(), table.data_ptr(), sl.data_ptr(),
+                 po.data_ptr(), pl.data_ptr(), wd.B, wd.H, wd.d, ps, table.shape[1], kc.shape[0],
+                 float(wd.softmax_scale), stream.cuda_stream, binding._dtype_code(wd.dtype),
+                 binding._dtype_code(wd.dtype), 0)
+        ms_pd, clk_pd = timed([lambda: check(binding.fa_fwd_decode_paged(*pargs),
+                                             "fa_fwd_decode_paged")],
+                              args.steps, args.warmup, ws, stream, local)
+        gbs_pd = bytes_d / (ms_pd * 1e-3) / 1e9
+        configs["decode_paged"] = compact(whole_job_rate(bytes_d, ms_pd, ws) / 1e9, "GB/s", ms_pd,
+                                          args.steps, gbs_pd / peaks["hbm_gbs"], None, clk_pd)
+        del pq, kc, vc, table, sl, po, pl
+        torch.cuda.empty_cache()
+
+        # headline shape with E4M3 queries and keys; quantisation (amax, scale, cast) runs in
+        # torch before the timed region: the library takes E4M3 codes as its inputs
         q, k, v = tensors[0], tensors[1], tensors[2]
         q_s = float(q.abs().amax()) / 448.0
         k_s = float(k.abs().amax()) / 448.0
@@ -391,35 +470,17 @@ def arm_ours(args, ws, rank, local):
                  wp.B, wp.H, wp.Nq, wp.Nkv, wp.d, float(wp.softmax_scale), int(wp.causal),
                  stream.cuda_stream, q_s, k_s, binding._dtype_code(wp.dtype),
                  binding._dtype_code(o8.dtype))
-
-        def fp8_call():
-            check(binding.fa_fwd_fp8(*fargs), "fa_fwd_fp8")
-
-        fsteps = max(3, args.steps // 4)
-        with ClockSampler(local) as clk_f, torch.cuda.stream(stream):
-            ms_f = time_steps(fp8_call, fsteps, args.warmup, ws, stream)
-        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+        ms_f, clk_f = timed([lambda: check(binding.fa_fwd_fp8(*fargs), "fa_fwd_fp8")],
+                            args.steps, args.warmup, ws, stream, local)
         tf_f = flops / (ms_f * 1e-3) / 1e12
         # Half the FLOPs (Q K^T) run at the E4M3 rate, nominally twice bf16; half (P V) at bf16.
-        peak_f = peak_t * 4.0 / 3.0
-        prefill_fp8 = {
-            "workload": workload_config(wp, "bf16")["workload"] + ", Q and K in E4M3 "
-                        "(per-tensor scales), V and P bf16",
-            "value": whole_job_rate(flops, ms_f, ws) / 1e12, "unit": "TFLOP/s",
-            "ms_per_step": ms_f, "steps": fsteps, "gpu_launches": fsteps,
-            "roofline": {"bound": "tensor", "achieved": tf_f, "peak": peak_f, "unit": "TFLOP/s",
-                         "frac": tf_f / peak_f, "traffic": None,
-                         "peak_source": "blend of half E4M3 (2x measured bf16, the nominal "
-                                        "ratio) and half measured bf16: 4/3 x " + peak_src,
-                         "frac_of_bf16_peak": tf_f / peak_t, "flops_per_launch": flops},
-            "clocks": clk_f.summary(),
-        }
+        configs["fp8_8k"] = compact(whole_job_rate(flops, ms_f, ws) / 1e12, "TFLOP/s", ms_f,
+                                    args.steps, tf_f / (peak_t * 4 / 3), tf_f / (peak_sus * 4 / 3),
+                                    clk_f)
         del q8, k8, o8, l8
         torch.cuda.empty_cache()
 
-    # backward pass (dQ, dK, dV) of the headline shape, from the forward's O and LSE
-    backward = None
-    if not args.skip_decode:
+        # backward (dQ, dK, dV) of the headline shape from its O and LSE and a seeded dO
         q, k, v, o, lse = tensors
         g = make_grad_out(wp.B, wp.H, wp.Nq, wp.d, wp.dtype, 1000 * wp.index + 3, device="cuda")
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -429,118 +490,49 @@ def arm_ours(args, ws, rank, local):
                  g.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), bws.data_ptr(), nws,
                  wp.B, wp.H, wp.Nq, wp.Nkv, wp.d, float(wp.softmax_scale), int(wp.causal),
                  stream.cuda_stream, binding._dtype_code(wp.dtype))
-
-        def bwd_call():
-            check(binding.fa_bwd(*bargs), "fa_bwd")
-
-        bsteps = max(3, args.steps // 4)
-        with ClockSampler(local) as clk_b, torch.cuda.stream(stream):
-            ms_b = time_steps(bwd_call, bsteps, args.warmup, ws, stream)
-        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
+        ms_b, clk_b = timed([lambda: check(binding.fa_bwd(*bargs), "fa_bwd")], args.steps,
+                            args.warmup, ws, stream, local)
         flops_b = backward_flops(wp)
         tf_b = flops_b / (ms_b * 1e-3) / 1e12
-        backward = {
-            "workload": workload_config(wp, "bf16")["workload"] + ", backward: dQ, dK, dV "
-                        "from Q, K, V, O, LSE and dO (iid N(0,1))",
-            "value": whole_job_rate(flops_b, ms_b, ws) / 1e12, "unit": "TFLOP/s",
-            "ms_per_step": ms_b, "steps": bsteps, "gpu_launches": 3 * bsteps,
-            "roofline": {"bound": "tensor", "achieved": tf_b, "peak": peak_t, "unit": "TFLOP/s",
-                         "frac": tf_b / peak_t,
-                         "traffic": BWD_TRAFFIC.get((BWD_REV, wp.name)),
-                         "traffic_kernel": "fa_bwd_sm100 (main kernel, 94.5% of the call)",
-                         "peak_source": peak_src,
-                         "flops_per_launch": flops_b,
-                         "note": "achieved over the whole call (prep, main and dQ kernels)"},
-            "clocks": clk_b.summary(),
-        }
+        configs["bwd_8k"] = compact(whole_job_rate(flops_b, ms_b, ws) / 1e12, "TFLOP/s", ms_b,
+                                    args.steps, tf_b / peak_t, tf_b / peak_sus, clk_b)
+        detail["bwd_8k"] = {"traffic": BWD_TRAFFIC.get((BWD_REV, wp.name)),
+                            "gpu_launches": 3 * args.steps, "flops_per_launch": flops_b}
         del g, dq, dk, dv, bws
         torch.cuda.empty_cache()
 
-    # packed variable-length prefill: a ragged causal batch
-    prefill_varlen = None
-    if not args.skip_decode:
+        # packed variable-length prefill: a ragged causal batch
         lens = varlen_lengths(16, 512, 8192, 4242)
-        Hv, dv = 32, 128
-        vq, vk, vv, vcu = varlen_inputs(lens, Hv, dv, torch.bfloat16, 8000, device="cuda")
+        Hv, dv_ = 32, 128
+        vq, vk, vv, vcu = varlen_inputs(lens, Hv, dv_, torch.bfloat16, 8000, device="cuda")
         vo = torch.empty_like(vq)
         vlse = torch.empty((vq.shape[0], Hv), dtype=torch.float32, device="cuda")
         vargs = (vq.data_ptr(), vk.data_ptr(), vv.data_ptr(), vo.data_ptr(), vlse.data_ptr(),
                  vcu.data_ptr(), vcu.data_ptr(), len(lens), Hv, vq.shape[0], vk.shape[0],
-                 max(lens), max(lens), dv, float(dv ** -0.5), 1, stream.cuda_stream,
+                 max(lens), max(lens), dv_, float(dv_ ** -0.5), 1, stream.cuda_stream,
                  binding.FA_BF16, binding.FA_BF16)
-
-        def varlen_call():
-            check(binding.fa_fwd_varlen(*vargs), "fa_fwd_varlen")
-
-        vsteps = max(3, args.steps // 4)
-        with ClockSampler(local) as clk_v, torch.cuda.stream(stream):
-            ms_v = time_steps(varlen_call, vsteps, args.warmup, ws, stream)
-        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
-        flops_v = sum(4 * dv * Hv * causal_pairs(n, n) for n in lens)
+        ms_v, clk_v = timed([lambda: check(binding.fa_fwd_varlen(*vargs), "fa_fwd_varlen")],
+                            args.steps, args.warmup, ws, stream, local)
+        flops_v = sum(4 * dv_ * Hv * causal_pairs(n, n) for n in lens)
         tf_v = flops_v / (ms_v * 1e-3) / 1e12
-        prefill_varlen = {
-            "workload": f"packed causal batch of {len(lens)} sequences, {sum(lens)} tokens "
-                        f"(lengths log-uniform in [512, 8192], seeded), H={Hv} d={dv} bf16",
-            "value": whole_job_rate(flops_v, ms_v, ws) / 1e12, "unit": "TFLOP/s",
-            "ms_per_step": ms_v, "steps": vsteps, "gpu_launches": vsteps,
-            "roofline": {"bound": "tensor", "achieved": tf_v, "peak": peak_t, "unit": "TFLOP/s",
-                         "frac": tf_v / peak_t, "traffic": None, "peak_source": peak_src,
-                         "flops_per_launch": flops_v},
-            "clocks": clk_v.summary(),
-        }
+        configs["varlen"] = compact(whole_job_rate(flops_v, ms_v, ws) / 1e12, "TFLOP/s", ms_v,
+                                    args.steps, tf_v / peak_t, tf_v / peak_sus, clk_v)
         del vq, vk, vv, vcu, vo, vlse
-        torch.cuda.empty_cache()
-
-    # decode against a paged KV cache (same shape as the decode workload)
-    decode_paged = None
-    if not args.skip_decode:
-        wd = WORKLOADS[args.decode_workload]
-        ps = 64
-        pq, kc, vc, table, sl = paged_decode_inputs(wd.B, wd.H, wd.Nkv, wd.d, ps, wd.dtype,
-                                                    1000 * wd.index + 500, device="cuda")
-        po = torch.empty((wd.B, wd.H, wd.d), dtype=wd.dtype, device="cuda")
-        pl = torch.empty((wd.B, wd.H), dtype=torch.float32, device="cuda")
-        pargs = (pq.data_ptr(), kc.data_ptr(), vc.data_ptr(), table.data_ptr(), sl.data_ptr(),
-                 po.data_ptr(), pl.data_ptr(), wd.B, wd.H, wd.d, ps, table.shape[1], kc.shape[0],
-                 float(wd.softmax_scale), stream.cuda_stream, binding._dtype_code(wd.dtype),
-                 binding._dtype_code(wd.dtype), 0)
-
-        def paged_call():
-            check(binding.fa_fwd_decode_paged(*pargs), "fa_fwd_decode_paged")
-
-        psteps = max(3, args.steps // 8)
-        with ClockSampler(local) as clk_p, torch.cuda.stream(stream):
-            ms_pd = time_steps(paged_call, psteps, args.warmup, ws, stream)
-        assert binding.fa_device_status(clear=True) == 0, "a kernel wait timed out"
-        bytes_pd = algorithmic_bytes(wd, 2)
-        gbs_pd = bytes_pd / (ms_pd * 1e-3) / 1e9
-        decode_paged = {
-            "workload": f"{wd.name} in a paged cache: {ps}-key pages, block table a seeded "
-                        f"random permutation of {kc.shape[0]} pages",
-            "value": whole_job_rate(bytes_pd, ms_pd, ws) / 1e9, "unit": "GB/s",
-            "ms_per_step": ms_pd, "steps": psteps, "gpu_launches": 2 * psteps,
-            "roofline": {"bound": "hbm", "achieved": gbs_pd, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": gbs_pd / peaks["hbm_gbs"], "traffic": None,
-                         "peak_source": peak_src, "algorithmic_bytes_per_launch": bytes_pd},
-            "clocks": clk_p.summary(),
-        }
-        del pq, kc, vc, table, sl, po, pl
         torch.cuda.empty_cache()
 
     # end to end through the C ABI with host buffers
     e2e = None
     if not args.skip_e2e:
-        esteps = max(3, min(args.steps, 20))
-        ms_e, h2d, d2h = run_e2e(wp, tensors, esteps, 3, ws, stream)
-        e2e = {"value": whole_job_rate(flops, ms_e, ws) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e,
-               "steps": esteps}
+        ms_e, h2d, d2h = run_e2e(wp, tensors, args.steps, args.warmup, ws, stream)
+        e2e = {"value": r4(whole_job_rate(flops, ms_e, ws) / 1e12), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": r4(ms_e),
+               "steps": args.steps}
     del tensors
 
     cpu = None
     if rank == 0 and ws == 1 and not args.skip_cpu:
         v, threads, desc, _ = cpu_baseline(wp, args.cpu_seconds)
-        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+        cpu = {"value": r4(v), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": desc}
 
     if rank == 0:
@@ -551,21 +543,20 @@ def arm_ours(args, ws, rank, local):
             "dtype": "bf16", "data": "synthetic",
             "config": workload_config(wp, "bf16"),
             "gpu_launches": args.steps,
-            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_t,
-                         "unit": "TFLOP/s", "frac": tflops / peak_t, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16 burst (kernel timed back to back)",
-                         "flops_per_launch": flops,
-                         "frac_of_sustained": tflops / peaks.get("bf16_tflops_sustained", peak_t)},
-            "clocks": clk.summary(),
-            "decode": decode,
-            "decode_paged": decode_paged,
-            "prefill_varlen": prefill_varlen,
-            "prefill_fp8": prefill_fp8,
-            "backward": backward,
+            "roofline": {"bound": "tensor", "achieved": r4(tflops), "peak": peak_t,
+                         "unit": "TFLOP/s", "frac": r4(tflops / peak_t), "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst",
+                         "flops_per_launch": flops, "frac_sus": r4(tflops / peak_sus)},
+            "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            # every other configuration, last, so that the end of the line holds all of it
+            "configs": configs,
         }
-        print(json.dumps(line), flush=True)
+        if args.detail:
+            with open(args.detail, "w") as f:
+                json.dump({"line": line, "detail": detail, "peaks": peaks}, f, indent=1)
+        print(json.dumps(line, separators=(",", ":")), flush=True)
 
 
 # Bumped whenever the backward main kernel changes, so stale ncu traffic is not reported.
@@ -593,7 +584,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--prefill-workload", default=PREFILL, choices=sorted(WORKLOADS))
     ap.add_argument("--decode-workload", default=DECODE, choices=sorted(WORKLOADS))
-    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-extra", action="store_true",
+                    help="time the headline prefill only")
+    ap.add_argument("--detail", default=None, help="also write a detailed JSON record here")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -54,6 +54,7 @@ _SIGNATURES = {
     "fa_device_status": [ctypes.POINTER(_I), _I],
     "fa_selftest_wait_timeout": [_VP],
     "fa_release_workspace": [],
+    "fa_get_last_cuda_error": [ctypes.POINTER(_I)],
     "fa_last_cuda_error": [],
     "fa_status_string": [_I],
     "fa_version": [],
@@ -169,6 +170,15 @@ def fa_device_status(clear: bool = True) -> int:
 
 def fa_selftest_wait_timeout(stream=None) -> int:
     return library().fa_selftest_wait_timeout(stream)
+
+
+def fa_get_last_cuda_error() -> int:
+    """The cudaError_t behind this thread's last FA_ERR_CUDA (0 if none); clears it."""
+    err = ctypes.c_int(0)
+    rc = library().fa_get_last_cuda_error(ctypes.byref(err))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_get_last_cuda_error")
+    return int(err.value)
 
 
 def fa_release_workspace() -> None:

@@ -14,13 +14,24 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// The device status word the kernels OR their wait-timeout and bad-input bits into: one
+// word per device (each device's copy of this array), zero when the module loads, so no
+// allocation is needed for it.
+__device__ __align__(256) int g_status_word[64];
+
+struct KernelConfig {
+  const void* fn;
+  cudaError_t err;
+};
+
 struct DeviceState {
   bool probed = false;
   bool arch_ok = false;
   int sm_count = 0;
-  int* status = nullptr;   // device status word (256 bytes allocated)
-  float* ws = nullptr;     // decode partials
-  size_t ws_bytes = 0;
+  int* status = nullptr;               // device address of this device's g_status_word
+  cudaMemPool_t pool = nullptr;        // workspace pool (decode partials, varlen unit list)
+  KernelConfig kernels[64] = {};       // kernels already configured on this device
+  int n_kernels = 0;
 };
 
 std::mutex g_mu;
@@ -33,8 +44,10 @@ int cuda_fail(cudaError_t e) {
   return FA_ERR_CUDA;
 }
 
-// Looks up (and on first use initialises) the current device's state.
-int device_state(DeviceState** out) {
+// Looks up (and on first use initialises) the current device's state: architecture, SM
+// count and the status word's address.  Nothing here allocates device memory or
+// synchronises.
+int device_state_core(DeviceState** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -53,16 +66,55 @@ int device_state(DeviceState** out) {
   }
   if (!s.arch_ok) return FA_ERR_ARCH;
   if (!s.status) {
+    // In host code g_status_word names a host-side stand-in: kernels get the address of
+    // this device's copy.
     void* p = nullptr;
-    if ((e = cudaMalloc(&p, 256)) != cudaSuccess) return e == cudaErrorMemoryAllocation ? FA_ERR_NOMEM : cuda_fail(e);
-    if ((e = cudaMemset(p, 0, 256)) != cudaSuccess || (e = cudaDeviceSynchronize()) != cudaSuccess) {
-      cudaFree(p);
-      return cuda_fail(e);
-    }
+    if ((e = cudaGetSymbolAddress(&p, g_status_word)) != cudaSuccess)
+      return e == cudaErrorMemoryAllocation ? FA_ERR_NOMEM : cuda_fail(e);
     s.status = static_cast<int*>(p);
   }
   *out = &s;
   return FA_OK;
+}
+
+// device_state_core, plus the device's workspace pool (created on the first call of any
+// entry point that may need workspace; creating a pool reserves no memory).  The pool
+// keeps freed memory mapped (release threshold: all of it), so after the first calls an
+// allocation from it is a bookkeeping step in stream order.
+int device_state(DeviceState** out) {
+  DeviceState* s = nullptr;
+  int rc = device_state_core(&s);
+  if (rc != FA_OK) return rc;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!s->pool) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if ((e = cudaMemPoolCreate(&pool, &props)) != cudaSuccess) return cuda_fail(e);
+    uint64_t keep = ~0ull;
+    if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return cuda_fail(e);
+    }
+    s->pool = pool;
+  }
+  *out = s;
+  return FA_OK;
+}
+
+// Stream-ordered workspace from the device's pool.  Under stream capture the allocation
+// and the matching cudaFreeAsync become graph memory nodes.
+int workspace_alloc(DeviceState* ds, size_t bytes, cudaStream_t stream, void** ptr) {
+  const cudaError_t e = cudaMallocFromPoolAsync(ptr, bytes, ds->pool, stream);
+  if (e == cudaErrorMemoryAllocation) return FA_ERR_NOMEM;
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
 int get_encoder() {
@@ -292,28 +344,17 @@ int run_decode(const void* q, const void* k, const void* v, void* o, float* lse,
   int rc = device_state(&ds);
   if (rc != FA_OK) return rc;
   const fa::DecodeParams p = decode_params(B, H, Nkv, scale, num_splits, ds->sm_count);
-  const size_t need = decode_ws_bytes(p, d);
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (ds->ws_bytes < need) {
-      if (ds->ws) {
-        cudaError_t e = cudaFree(ds->ws);  // synchronises: no kernel still reads it
-        ds->ws = nullptr;
-        ds->ws_bytes = 0;
-        if (e != cudaSuccess) return cuda_fail(e);
-      }
-      void* ptr = nullptr;
-      cudaError_t e = cudaMalloc(&ptr, need);
-      if (e != cudaSuccess) return e == cudaErrorMemoryAllocation ? FA_ERR_NOMEM : cuda_fail(e);
-      ds->ws = static_cast<float*>(ptr);
-      ds->ws_bytes = need;
-    }
-  }
-  float* part_o = ds->ws;
-  float* part_lse = ds->ws + static_cast<size_t>(p.grid) * p.max_seg * 8 * d;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The split partials live for this call only: allocated and freed in stream order, so
+  // calls on different streams never share them and no call waits for the device.
+  void* ws = nullptr;
+  if ((rc = workspace_alloc(ds, decode_ws_bytes(p, d), st, &ws)) != FA_OK) return rc;
+  float* part_o = static_cast<float*>(ws);
+  float* part_lse = part_o + static_cast<size_t>(p.grid) * p.max_seg * 8 * d;
   cudaError_t e = fa::launch_decode(q, k, v, o, lse, p, d, in_dtype == FA_BF16, o_dtype == FA_F32,
-                                    part_o, part_lse, ds->status, static_cast<cudaStream_t>(stream),
-                                    paged);
+                                    part_o, part_lse, ds->status, st, paged);
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e == cudaSuccess) e = ef;
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
@@ -359,6 +400,39 @@ DecodeParams plan_decode(int B, int H, int Nkv, float scale, int num_splits, int
   return decode_params(B, H, Nkv, scale, num_splits, sm_count);
 }
 size_t decode_workspace_bytes(const DecodeParams& p, int d) { return decode_ws_bytes(p, d); }
+
+int cuda_failure(cudaError_t e) { return cuda_fail(e); }
+
+int current_device(int* sm_count, int** status) {
+  DeviceState* ds = nullptr;
+  const int rc = device_state_core(&ds);
+  if (rc != FA_OK) return rc;
+  *sm_count = ds->sm_count;
+  *status = ds->status;
+  return FA_OK;
+}
+
+cudaError_t configure_kernel(const void* kernel, int smem_bytes, int min_regs) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  for (int i = 0; i < s.n_kernels; ++i)
+    if (s.kernels[i].fn == kernel) return s.kernels[i].err;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e == cudaSuccess && min_regs > 0) {
+    cudaFuncAttributes attr;
+    e = cudaFuncGetAttributes(&attr, kernel);
+    // setmaxnreg redistributes the registers the block was launched with; a launch with
+    // fewer would make the increase wait forever.
+    if (e == cudaSuccess && attr.numRegs < min_regs) e = cudaErrorInvalidConfiguration;
+  }
+  if (s.n_kernels < static_cast<int>(sizeof(s.kernels) / sizeof(s.kernels[0])))
+    s.kernels[s.n_kernels++] = KernelConfig{kernel, e};
+  return e;
+}
 }  // namespace fa
 
 extern "C" {
@@ -611,12 +685,18 @@ int fa_release_workspace(void) {
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& s = g_dev[dev];
-  if (s.ws) {
-    e = cudaFree(s.ws);
-    s.ws = nullptr;
-    s.ws_bytes = 0;
-    if (e != cudaSuccess) return cuda_fail(e);
+  if (s.pool) {
+    // Every free the kernels' calls enqueued has completed once the device is idle.
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemPoolTrimTo(s.pool, 0)) != cudaSuccess) return cuda_fail(e);
   }
+  return FA_OK;
+}
+
+int fa_get_last_cuda_error(int* cuda_err) {
+  if (!cuda_err) return FA_ERR_INVALID_ARG;
+  *cuda_err = g_last_cuda_error;
+  g_last_cuda_error = 0;
   return FA_OK;
 }
 

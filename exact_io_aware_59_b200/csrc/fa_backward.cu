@@ -586,19 +586,8 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      const CUtensorMap& tdo, const void* o, const void* dout, const float* lse,
                      void* dq, const BwdParams& p, int sm_count, int* status, cudaStream_t stream) {
   auto kern = fa_bwd_sm100<BF16>;
-  static bool configured = false;  // per template instance
-  static cudaError_t config_err = cudaSuccess;
-  if (!configured) {
-    config_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg::kAlloc);
-    if (config_err == cudaSuccess) {
-      cudaFuncAttributes attr;
-      config_err = cudaFuncGetAttributes(&attr, kern);
-      // setmaxnreg redistributes the registers the block was launched with; a launch
-      // with fewer would make the increase wait forever.
-      if (config_err == cudaSuccess && attr.numRegs < kRegsLaunch) config_err = cudaErrorInvalidConfiguration;
-    }
-    configured = true;
-  }
+  const cudaError_t config_err =
+      configure_kernel(reinterpret_cast<const void*>(kern), BwdCfg::kAlloc, kRegsLaunch);
   if (config_err != cudaSuccess) return config_err;
   const long long rows = static_cast<long long>(p.BH) * p.nq_pad;
   long long prep_blocks = (rows + 15) / 16;  // 16 rows per 256-thread block

@@ -380,8 +380,7 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, void* o, float
                      const DecodeParams& p, bool o_f32, float* part_o, float* part_lse,
                      int* status, cudaStream_t stream, const PagedKV* paged) {
   auto kern = paged ? fa_decode_split_sm100<D, BF16, true> : fa_decode_split_sm100<D, BF16, false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       DecodeCfg<D>::kBytes);
+  cudaError_t e = configure_kernel(reinterpret_cast<const void*>(kern), DecodeCfg<D>::kBytes, 0);
   if (e != cudaSuccess) return e;
   const PagedKV pk = paged ? *paged : PagedKV{nullptr, nullptr, 1, 0, 0, 0};
   kern<<<p.grid, kThreads, DecodeCfg<D>::kBytes, stream>>>(

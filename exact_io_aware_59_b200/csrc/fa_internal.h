@@ -100,6 +100,20 @@ int check_decode_call(const void* q, const void* k, const void* v, void* o, floa
 DecodeParams plan_decode(int B, int H, int Nkv, float scale, int num_splits, int sm_count);
 size_t decode_workspace_bytes(const DecodeParams& p, int d);
 
+// Records `e` as this host thread's last CUDA error (what fa_get_last_cuda_error reports)
+// and returns FA_ERR_CUDA (fa_api.cu).
+int cuda_failure(cudaError_t e);
+
+// The current device's SM count and status-word address, set up on first use (checks the
+// architecture; allocates nothing).  Returns an FA_* status (fa_api.cu).
+int current_device(int* sm_count, int** status);
+
+// One-time, thread-safe set-up of a kernel on the CURRENT device: opts it into
+// `smem_bytes` of dynamic shared memory and, when min_regs > 0, checks that it was built
+// with at least that many registers per thread (setmaxnreg redistributes them).  Later
+// calls on the same device return the first call's result (fa_api.cu).
+cudaError_t configure_kernel(const void* kernel, int smem_bytes, int min_regs);
+
 // Bytes of dynamic shared memory each kernel needs.
 size_t prefill_smem_bytes(int d);
 size_t decode_smem_bytes(int d);

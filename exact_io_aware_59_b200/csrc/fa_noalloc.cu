@@ -1,12 +1,12 @@
 // fa_noalloc.cu -- split-KV decode that allocates no device memory.
 //
-// fa_fwd_decode keeps its split partials in a workspace it allocates with cudaMalloc on
-// first use.  Some callers cannot allow that: a runtime that has already handed all
-// device memory to its own pool, a plug-in inside a host program that forbids device
-// allocations after start-up, or latency-critical code that cannot pay for the device
-// synchronisation cudaMalloc and cudaFree imply.  fa_fwd_decode_noalloc runs the same
-// two kernels with the partials (and the kernels' status word) in the fixed array below
-// instead.  Every GPU that loads this library holds the array until the process exits.
+// fa_fwd_decode takes its split partials from a stream-ordered memory pool that the
+// library creates and grows on demand.  Some callers cannot allow any device allocation
+// by a library: a runtime that has already handed all device memory to its own pool, a
+// plug-in inside a host program that forbids device allocations after start-up, or code
+// that must not depend on an allocator's state for its latency.  fa_fwd_decode_noalloc
+// runs the same two kernels with the partials in the fixed array below instead.  Every
+// GPU that loads this file's module holds the array until the process exits.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -16,46 +16,33 @@
 
 namespace {
 
-// Static scratch: [0, 256) status word, then the decode partials (O_s, then lse_s).
+// Static scratch for the decode partials (O_s, then lse_s).
 static __device__ __align__(256) unsigned char g_decode_scratch[FA_NOALLOC_SCRATCH_BYTES];
-constexpr size_t kStatusBytes = 256;
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-bool g_ready[kMaxDevices] = {};
 unsigned char* g_scratch_ptr[kMaxDevices] = {};  // device address of g_decode_scratch
-int g_sm_count[kMaxDevices] = {};
-thread_local int g_noalloc_cuda_error = 0;
 
-// Once per device, with that device current: checks the architecture and looks up the
-// device address of the static array.  In host code `g_decode_scratch` names only a host
-// stand-in, never the device memory, so kernels must be given this address.
-int setup_device(int* dev_out) {
+// Once per device, with that device current: looks up the device address of the static
+// array.  In host code `g_decode_scratch` names only a host stand-in, never the device
+// memory, so kernels must be given this address.  With CUDA's lazy module loading this
+// lookup is what loads the module, and so what commits the array's memory on the device:
+// an allocation failure there is reported as FA_ERR_NOMEM.
+int setup_scratch(unsigned char** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) { g_noalloc_cuda_error = e; return FA_ERR_CUDA; }
+  if (e != cudaSuccess) return fa::cuda_failure(e);
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_ready[dev]) {
-    int major = 0, minor = 0, sms = 0;
-    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
-        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) {
-      g_noalloc_cuda_error = e;
-      return FA_ERR_CUDA;
-    }
-    if (major != 10 || minor != 0) return FA_ERR_ARCH;
+  if (!g_scratch_ptr[dev]) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-    if (e != cudaSuccess || ptr == nullptr) {
-      g_noalloc_cuda_error = (e != cudaSuccess) ? e : cudaErrorInvalidSymbol;
-      return FA_ERR_CUDA;
-    }
+    if (e == cudaErrorMemoryAllocation) return FA_ERR_NOMEM;
+    if (e != cudaSuccess) return fa::cuda_failure(e);
+    if (ptr == nullptr) return fa::cuda_failure(cudaErrorInvalidSymbol);
     g_scratch_ptr[dev] = static_cast<unsigned char*>(ptr);
-    g_sm_count[dev] = sms;
-    g_ready[dev] = true;
   }
-  *dev_out = dev;
+  *out = g_scratch_ptr[dev];
   return FA_OK;
 }
 
@@ -67,21 +54,24 @@ extern "C" int fa_fwd_decode_noalloc(const void* q, const void* k, const void* v
   int rc = fa::check_decode_call(q, k, v, o, lse, B, H, Nkv, d, scale, in_dtype, o_dtype);
   if (rc != FA_OK) return rc;
   if (num_splits < 0) return FA_ERR_INVALID_ARG;
-  int dev = 0;
-  if ((rc = setup_device(&dev)) != FA_OK) return rc;
-  const fa::DecodeParams p = fa::plan_decode(B, H, Nkv, scale, num_splits, g_sm_count[dev]);
+  // The architecture check, the SM count and the status word (a static device variable,
+  // shared with the other entry points) come from the library's per-device state, which
+  // allocates nothing.
+  int sm_count = 0;
+  int* status = nullptr;
+  if ((rc = fa::current_device(&sm_count, &status)) != FA_OK) return rc;
+  const fa::DecodeParams p = fa::plan_decode(B, H, Nkv, scale, num_splits, sm_count);
   // Too large for the fixed array: refuse before anything is enqueued.
-  if (kStatusBytes + fa::decode_workspace_bytes(p, d) > FA_NOALLOC_SCRATCH_BYTES)
-    return FA_ERR_UNSUPPORTED;
+  if (fa::decode_workspace_bytes(p, d) > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  unsigned char* base = nullptr;
+  if ((rc = setup_scratch(&base)) != FA_OK) return rc;
   // The partials need no clearing: every record the combine kernel reads is written by the
-  // split kernel of the same call.  The status word is only ever OR-ed into.
-  unsigned char* base = g_scratch_ptr[dev];
-  int* status = reinterpret_cast<int*>(base);
-  float* part_o = reinterpret_cast<float*>(base + kStatusBytes);
+  // split kernel of the same call, unless a split kernel's wait runs out, which the status
+  // word reports (fa_device_status); the outputs of such a call are undefined.
+  float* part_o = reinterpret_cast<float*>(base);
   float* part_lse = part_o + static_cast<size_t>(p.grid) * p.max_seg * 8 * d;
-  cudaError_t e = fa::launch_decode(q, k, v, o, lse, p, d, in_dtype == FA_BF16,
-                                    o_dtype == FA_F32, part_o, part_lse, status,
-                                    static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) { g_noalloc_cuda_error = e; return FA_ERR_CUDA; }
-  return FA_OK;
+  const cudaError_t e = fa::launch_decode(q, k, v, o, lse, p, d, in_dtype == FA_BF16,
+                                          o_dtype == FA_F32, part_o, part_lse, status,
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : fa::cuda_failure(e);
 }

@@ -696,20 +696,8 @@ cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
                      float* lse, const PrefillParams& p, int grid, int* status,
                      cudaStream_t stream) {
   auto kern = fa_prefill_sm100<D, BF16, OF32, VARLEN, QK8>;
-  static bool configured = false;  // per template instance
-  static cudaError_t config_err = cudaSuccess;
-  if (!configured) {
-    config_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      PrefillCfg<D>::kAlloc);
-    if (config_err == cudaSuccess) {
-      cudaFuncAttributes attr;
-      config_err = cudaFuncGetAttributes(&attr, kern);
-      // setmaxnreg redistributes the registers the block was launched with; a launch
-      // with fewer would make the increase wait forever.
-      if (config_err == cudaSuccess && attr.numRegs < kRegsLaunch) config_err = cudaErrorInvalidConfiguration;
-    }
-    configured = true;
-  }
+  const cudaError_t config_err =
+      configure_kernel(reinterpret_cast<const void*>(kern), PrefillCfg<D>::kAlloc, kRegsLaunch);
   if (config_err != cudaSuccess) return config_err;
   kern<<<grid, kThreads, PrefillCfg<D>::kAlloc, stream>>>(tq, tk, tv, o, lse, p, status);
   return cudaGetLastError();

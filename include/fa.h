@@ -31,16 +31,18 @@
  * Ownership and ordering: the caller owns every buffer.  Calls only enqueue work on
  * `stream` (a cudaStream_t; NULL = the legacy default stream) and never synchronise
  * it; the buffers must stay valid until that work has finished.  The library keeps no
- * pointer to caller memory after a call returns.  It owns two per-device allocations:
- * a 256-byte device status word (allocated on the first call on a device) and, for
- * decode, a grow-only workspace for the split partials (allocated with cudaMalloc on the
- * first decode call that needs more; do that first call outside stream capture).
- * Decode calls on one device share that workspace, so decode calls that can run
- * concurrently (different streams without ordering between them) race on it.
+ * pointer to caller memory after a call returns.  Per device it owns a status word (a
+ * static device variable: nothing is allocated for it) and a stream-ordered memory pool
+ * for call-local workspace (the decode split partials, the varlen unit list): a call
+ * that needs workspace allocates it from the pool on `stream` (cudaMallocFromPoolAsync)
+ * and frees it on `stream` after its last kernel (cudaFreeAsync), so calls on different
+ * streams never share workspace, no call synchronises, and under stream capture the pair
+ * becomes graph memory nodes.  The pool is created on the first call that needs it and
+ * keeps freed memory mapped for reuse until fa_release_workspace().
  *
  * Errors: argument checks run on the host before anything is enqueued; a failed check
  * returns its code and launches nothing.  FA_ERR_CUDA means a CUDA runtime call failed;
- * fa_last_cuda_error() returns the cudaError_t.  Device-side faults are never raised on
+ * fa_get_last_cuda_error() returns the cudaError_t.  Device-side faults are never raised on
  * purpose: every wait inside the kernels is bounded (about 1 s); a wait that runs out
  * sets bits in the device status word and the kernel returns early, leaving the outputs
  * undefined.  Read (and clear) that word with fa_device_status() after synchronising.
@@ -65,8 +67,8 @@ enum {
   FA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, misalignment, overlap, ... */
   FA_ERR_UNSUPPORTED = 2,     /* valid request the library does not implement (d, dtype pair) */
   FA_ERR_ARCH = 3,            /* current device is not compute capability 10.0 (B200) */
-  FA_ERR_CUDA = 4,            /* a CUDA runtime call failed: see fa_last_cuda_error() */
-  FA_ERR_NOMEM = 5,           /* a library-owned allocation failed */
+  FA_ERR_CUDA = 4,            /* a CUDA runtime call failed: see fa_get_last_cuda_error() */
+  FA_ERR_NOMEM = 5,           /* device memory for workspace (or a static array) ran out */
   FA_ERR_DEVICE_TIMEOUT = 6   /* fa_device_status(): a kernel's bounded wait ran out */
 };
 
@@ -110,29 +112,31 @@ int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* l
 /*
  * fa_fwd_decode_noalloc -- fa_fwd_decode for callers that cannot allocate device memory.
  * The pages have no counterpart: this is a deployment variant, not part of the method.
- *   Who needs it: fa_fwd_decode allocates its split workspace with cudaMalloc on first
- *   use, and some callers cannot allow that -- a runtime that has handed all device
- *   memory to its own pool, a plug-in whose host program forbids device allocations after
- *   start-up, or latency-critical code that cannot pay for the device synchronisation
- *   that cudaMalloc / cudaFree imply.
+ *   Who needs it: fa_fwd_decode takes its split partials from a memory pool the library
+ *   creates and grows on demand, and some callers cannot allow a library to allocate --
+ *   a runtime that has handed all device memory to its own pool, a plug-in whose host
+ *   program forbids device allocations after start-up, or code whose latency must not
+ *   depend on an allocator's state.
  *   What it does: the same split-KV decode and combine kernels, same arguments, layouts
  *   and results as fa_fwd_decode, with the split partials kept in one fixed static device
- *   array of FA_NOALLOC_SCRATCH_BYTES bytes that every GPU loading this library holds
- *   until the process exits.  The caller still passes q, k, v, o and lse.  No cudaMalloc,
- *   cudaFree or other allocating routine is called.
+ *   array of FA_NOALLOC_SCRATCH_BYTES bytes.  The caller still passes q, k, v, o and lse.
+ *   No cudaMalloc, cudaFree or other allocating routine is called.
  *   Limit: a call whose partials need more than the array (G * max_seg * 8 * (d+1) * 4
- *   bytes plus 256, see fa_decode_workspace_bytes) is refused with FA_ERR_UNSUPPORTED
- *   before anything is enqueued.  With the default split count (one CTA per SM, 148 on
- *   B200) that holds for B*H up to about 1,700 heads at d = 128 and 3,800 at d = 64, for
- *   any Nkv (B=16, H=32, d=128 needs 3.1 MB).
- *   First call: the first call on each device (made with that device current) checks the
- *   device and looks up the array's device address; make that first call before any
- *   stream capture.
+ *   bytes, the figure fa_decode_workspace_bytes returns) is refused with
+ *   FA_ERR_UNSUPPORTED before anything is enqueued.  With the default split count (one
+ *   CTA per SM, 148 on B200) that holds for B*H up to about 1,700 heads at d = 128 and
+ *   3,800 at d = 64, for any Nkv (B=16, H=32, d=128 needs 3.1 MB).
+ *   First call: the first call on each device (made with that device current) looks up
+ *   the array's device address.  Under CUDA's default lazy module loading that lookup is
+ *   what loads the array's module, so it is the moment the 8 MiB are committed on that
+ *   device (FA_ERR_NOMEM if they cannot be); make that first call before the caller's own
+ *   pool claims the device's memory.  Every GPU where that happened holds the array until
+ *   the process exits.
  *   Sharing: every call on a device uses the same array, which keeps the last call's
  *   contents.  Nothing in it needs clearing between calls.  Calls whose kernels can
  *   overlap on the GPU (different streams without ordering between them) race on the
- *   array.  A kernel wait that runs out is recorded in a status word inside the array,
- *   which this entry point does not report (use fa_fwd_decode when that is needed).
+ *   array.  A kernel wait that runs out is recorded in the same device status word as for
+ *   the other entry points (fa_device_status); the outputs of that call are undefined.
  */
 #define FA_NOALLOC_SCRATCH_BYTES (8u << 20)
 int fa_fwd_decode_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -261,10 +265,22 @@ enum {
  */
 int fa_selftest_wait_timeout(void* stream);
 
-/* Frees the current device's decode workspace (synchronises the device). */
+/*
+ * fa_release_workspace -- returns the memory the current device's workspace pool keeps
+ * mapped for reuse.  Synchronises the device first (so every enqueued free has
+ * completed); do not call it during stream capture.  Later calls that need workspace
+ * allocate it again.
+ */
 int fa_release_workspace(void);
 
-/* The cudaError_t behind the last FA_ERR_CUDA returned on this host thread. */
+/*
+ * fa_get_last_cuda_error -- writes the cudaError_t behind the last FA_ERR_CUDA returned on
+ * this host thread (0 if none since the last read) to *cuda_err and clears it, like
+ * cudaGetLastError.  Returns FA_OK, or FA_ERR_INVALID_ARG when cuda_err is NULL.
+ */
+int fa_get_last_cuda_error(int* cuda_err);
+
+/* The same value as fa_get_last_cuda_error, without clearing it. */
 int fa_last_cuda_error(void);
 
 /* A static, human-readable name for a status code. */

@@ -107,6 +107,70 @@ def test_valid_call_without_device_reports_cuda_error():
     assert binding.library().fa_last_cuda_error() != 0
 
 
+# Every entry point that reaches the device, called with valid arguments in a process that
+# sees no CUDA device: each must return FA_ERR_CUDA and leave the CUDA error code for
+# fa_get_last_cuda_error, which clears it.  No device is visible, so nothing can launch.
+_NO_DEVICE_SCRIPT = r"""
+import ctypes, json, sys
+sys.path.insert(0, sys.argv[1])
+from exact_io_aware_59_b200 import binding as b
+A = 1 << 20
+Q, K, V, O, L = A, 2 * A, 3 * A, 4 * A, 5 * A
+lib = b.library()
+calls = {
+    "fa_fwd": lambda: b.fa_fwd(Q, K, V, O, L, 1, 2, 16, 16, 64, 0.125, 0, None, 0, 2),
+    "fa_fwd_prefill": lambda: b.fa_fwd_prefill(Q, K, V, O, L, 1, 2, 16, 16, 64, 0.125, 1, None,
+                                               0, 2, 0),
+    "fa_fwd_decode": lambda: b.fa_fwd_decode(Q, K, V, O, L, 1, 2, 16, 64, 0.125, None, 0, 2, 0),
+    "fa_fwd_decode_noalloc": lambda: b.fa_fwd_decode_noalloc(Q, K, V, O, L, 1, 2, 16, 64, 0.125,
+                                                             None, 0, 2, 0),
+    "fa_fwd_fp8": lambda: b.fa_fwd_fp8(Q, K, V, O, L, 1, 1, 4, 4, 128, 0.1, 0, None, 1.0, 1.0, 1,
+                                       2),
+    "fa_fwd_varlen": lambda: b.fa_fwd_varlen(Q, K, V, O, L, L + 4096, L + 8192, 2, 2, 100, 100,
+                                             60, 60, 64, 0.1, 1, None, 0, 2),
+    "fa_fwd_decode_paged": lambda: b.fa_fwd_decode_paged(Q, K, V, L + 64, L + 128, O, L, 1, 1,
+                                                         64, 16, 4, 8, 0.1, None, 0, 2, 0),
+    "fa_bwd": lambda: b.fa_bwd(Q, K, V, O, L, Q + 4096, O + 4096, O + 8192, O + 12288,
+                               O + 65536, 64 * 520, 1, 1, 4, 4, 128, 0.1, 0, None, 1),
+    "fa_device_status": lambda: lib.fa_device_status(ctypes.byref(ctypes.c_int(0)), 0),
+    "fa_selftest_wait_timeout": lambda: lib.fa_selftest_wait_timeout(None),
+    "fa_release_workspace": lambda: lib.fa_release_workspace(),
+    "fa_decode_workspace_bytes": lambda: lib.fa_decode_workspace_bytes(
+        1, 1, 64, 64, 0, ctypes.byref(ctypes.c_size_t(0))),
+}
+out = {}
+for name, fn in calls.items():
+    rc = int(fn())
+    err = b.fa_get_last_cuda_error()
+    out[name] = [rc, err, b.fa_get_last_cuda_error()]
+print(json.dumps(out))
+"""
+
+
+def test_every_entry_point_reports_its_cuda_error():
+    import json
+    import os
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-c", _NO_DEVICE_SCRIPT, root], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    out = json.loads(r.stdout.strip().splitlines()[-1])
+    codes = set()
+    for name, (rc, err, err_after) in out.items():
+        assert rc == binding.FA_ERR_CUDA, (name, rc)
+        assert err != 0, name                # the cudaError_t behind FA_ERR_CUDA
+        assert err_after == 0, name          # reading it cleared it
+        codes.add(err)
+    assert len(codes) == 1                   # the same "no device" error everywhere
+
+
+def test_get_last_cuda_error_checks_its_pointer():
+    assert binding.library().fa_get_last_cuda_error(None) == binding.FA_ERR_INVALID_ARG
+
+
 def test_binding_rejects_host_tensors():
     q = torch.zeros(1, 1, 4, 64, dtype=torch.float16)
     with pytest.raises(ValueError):

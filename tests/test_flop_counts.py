@@ -47,3 +47,19 @@ def test_decode_algorithmic_bytes():
     BH = 16 * 32
     expect = BH * (128 * 2 + 2 * 32768 * 128 * 2 + 128 * 2 + 4)
     assert bench.algorithmic_bytes(w, 2) == expect == 8590198784
+
+
+def test_bench_line_keeps_every_config_in_its_last_1500_characters():
+    """The per-config records go last in the printed line and stay short enough that the
+    end of the line (what a log tail keeps) holds every one of them."""
+    import json
+
+    clk = {"sm_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    names = ["mha_d64", "noncausal_8k", "peaky_8k", "causal_16k", "causal_32k", "decode",
+             "decode_paged", "fp8_8k", "bwd_8k", "varlen"]
+    configs = {n: bench.compact(1234.56789, "TFLOP/s", 0.123456789, 2000, 0.6789012,
+                                0.7890123, clk) for n in names}
+    line = {"metric": bench.METRIC, "value": 1.0, "configs": configs}
+    tail = json.dumps(line, separators=(",", ":"))[-1500:]
+    for n in names:
+        assert f'"{n}":' in tail, n
