@@ -13,7 +13,8 @@ timed for the line's own "steps":
   causal_32k    B=1 H=16 N=32768 d=128 bf16 causal
   decode        B=16 H=32 Nq=1 Nkv=32768 d=128 bf16, split-KV decode (HBM GB/s)
   decode_paged  the decode shape in a paged cache of 64-key pages (fa_fwd_decode_paged)
-  fp8_8k        the headline shape with E4M3 Q and K (fa_fwd_fp8; peak: 4/3 of bf16)
+  fp8_8k        the headline shape with E4M3 Q and K given (fa_fwd_fp8; peak: 4/3 of bf16)
+  fp8q_8k       the same, Q and K quantised on the fly inside the step (fa_fwd_fp8_quant)
   bwd_8k        dQ, dK, dV of the headline shape (fa_bwd; 10*d FLOP per visible pair)
   varlen        a packed causal batch of 16 sequences, lengths log-uniform in [512, 8192]
 Every configuration is timed for the same --steps.  Inputs are resident in HBM when the
@@ -360,8 +361,11 @@ def compact(value, unit, ms, steps, frac, frac_sus, clk):
         d["frac_sus"] = r4(frac_sus)
     if clk:
         d["sm_mhz"] = int(round(clk["sm_mhz"]))
-        if clk["reasons"]:
-            d["reasons"] = clk["reasons"]
+        # sw_power_cap is the normal state of a long dense run on a 1 kW part; any other
+        # throttle reason is named
+        other = [r for r in clk["reasons"] if r != "sw_power_cap"]
+        if other:
+            d["reasons"] = other
     return d
 
 
@@ -411,26 +415,31 @@ def arm_ours(args, ws, rank, local):
     value = whole_job_rate(flops, ms_p, ws) / 1e12
     traffic = DRAM_TRAFFIC.get((KERNEL_REV, wp.name))
 
-    if not args.skip_extra:
-        # the other prefill configurations of the same kernel
-        for key, name in (("mha_d64", "prefill_mha"), ("noncausal_8k", "long_prefill"),
-                          ("peaky_8k", "long_prefill_peaky"), ("causal_16k", "long_ctx_16k"),
-                          ("causal_32k", "long_ctx_32k")):
-            if name == wp.name:
-                continue
-            rec, ms, _, _, first = prefill_record(WORKLOADS[name], args, ws, stream, local,
-                                                  peaks)
-            configs[key] = rec
-            del first
-            torch.cuda.empty_cache()
+    only = set(args.only.split(",")) if args.only else None
 
-        # split-KV decode (HBM bound): one fa_fwd (split + combine kernels) per step
-        wd = WORKLOADS[args.decode_workload]
+    def want(key):
+        return not args.skip_extra and (only is None or key in only)
+
+    # the other prefill configurations of the same kernel
+    for key, name in (("mha_d64", "prefill_mha"), ("noncausal_8k", "long_prefill"),
+                      ("peaky_8k", "long_prefill_peaky"), ("causal_16k", "long_ctx_16k"),
+                      ("causal_32k", "long_ctx_32k")):
+        if name == wp.name or not want(key):
+            continue
+        rec, ms, _, _, first = prefill_record(WORKLOADS[name], args, ws, stream, local,
+                                              peaks)
+        configs[key] = rec
+        del first
+        torch.cuda.empty_cache()
+
+    # split-KV decode (HBM bound): one fa_fwd (split + combine kernels) per step
+    wd = WORKLOADS[args.decode_workload]
+    bytes_d = algorithmic_bytes(wd, 2)
+    if want("decode"):
         sets, _ = input_sets(wd, wd.dtype)
         ms_d, clk_d = timed([make_call(wd, *t, stream) for t in sets], args.steps, args.warmup,
                             ws, stream, local)
         del sets
-        bytes_d = algorithmic_bytes(wd, 2)
         gbs = bytes_d / (ms_d * 1e-3) / 1e9
         configs["decode"] = compact(whole_job_rate(bytes_d, ms_d, ws) / 1e9, "GB/s", ms_d,
                                     args.steps, gbs / peaks["hbm_gbs"], None, clk_d)
@@ -438,6 +447,7 @@ def arm_ours(args, ws, rank, local):
                             "traffic": DECODE_TRAFFIC.get((DECODE_REV, wd.name))}
         torch.cuda.empty_cache()
 
+    if want("decode_paged"):
         # decode against a paged KV cache (same shape): 64-key pages, seeded random table
         ps = 64
         pq, kc, vc, table, sl = paged_decode_inputs(wd.B, wd.H, wd.Nkv, wd.d, ps, wd.dtype,
@@ -457,9 +467,10 @@ def arm_ours(args, ws, rank, local):
         del pq, kc, vc, table, sl, po, pl
         torch.cuda.empty_cache()
 
-        # headline shape with E4M3 queries and keys; quantisation (amax, scale, cast) runs in
-        # torch before the timed region: the library takes E4M3 codes as its inputs
-        q, k, v = tensors[0], tensors[1], tensors[2]
+    q, k, v = tensors[0], tensors[1], tensors[2]
+    if want("fp8_8k"):
+        # headline shape with E4M3 queries and keys given as codes (quantised by torch with
+        # per-tensor scales before the timed region); fp8q_8k below times the on-the-fly path
         q_s = float(q.abs().amax()) / 448.0
         k_s = float(k.abs().amax()) / 448.0
         q8 = (q.float() / q_s).to(torch.float8_e4m3fn).view(torch.uint8)
@@ -480,6 +491,24 @@ def arm_ours(args, ws, rank, local):
         del q8, k8, o8, l8
         torch.cuda.empty_cache()
 
+    if want("fp8q_8k"):
+        # the same with the quantisation inside the timed region: fa_fwd_fp8_quant takes the
+        # bf16 Q and K and quantises them on the fly (one scale per 128-row tile)
+        o8 = torch.empty_like(tensors[3])
+        l8 = torch.empty_like(tensors[4])
+        qargs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o8.data_ptr(), l8.data_ptr(), wp.B,
+                 wp.H, wp.Nq, wp.Nkv, wp.d, float(wp.softmax_scale), int(wp.causal),
+                 stream.cuda_stream, binding._dtype_code(wp.dtype), binding._dtype_code(o8.dtype))
+        ms_fq, clk_fq = timed([lambda: check(binding.fa_fwd_fp8_quant(*qargs), "fa_fwd_fp8_quant")],
+                              args.steps, args.warmup, ws, stream, local)
+        tf_fq = flops / (ms_fq * 1e-3) / 1e12
+        configs["fp8q_8k"] = compact(whole_job_rate(flops, ms_fq, ws) / 1e12, "TFLOP/s", ms_fq,
+                                     args.steps, tf_fq / (peak_t * 4 / 3),
+                                     tf_fq / (peak_sus * 4 / 3), clk_fq)
+        del o8, l8
+        torch.cuda.empty_cache()
+
+    if want("bwd_8k"):
         # backward (dQ, dK, dV) of the headline shape from its O and LSE and a seeded dO
         q, k, v, o, lse = tensors
         g = make_grad_out(wp.B, wp.H, wp.Nq, wp.d, wp.dtype, 1000 * wp.index + 3, device="cuda")
@@ -501,6 +530,7 @@ def arm_ours(args, ws, rank, local):
         del g, dq, dk, dv, bws
         torch.cuda.empty_cache()
 
+    if want("varlen"):
         # packed variable-length prefill: a ragged causal batch
         lens = varlen_lengths(16, 512, 8192, 4242)
         Hv, dv_ = 32, 128
@@ -587,6 +617,8 @@ def main():
     ap.add_argument("--skip-extra", action="store_true",
                     help="time the headline prefill only")
     ap.add_argument("--detail", default=None, help="also write a detailed JSON record here")
+    ap.add_argument("--only", default=None,
+                    help="comma-separated configs to time besides the headline (default: all)")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

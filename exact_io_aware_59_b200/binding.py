@@ -47,6 +47,8 @@ _SIGNATURES = {
                       _I, _I],
     "fa_fwd_decode_paged": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP,
                             _I, _I, _I],
+    "fa_quantize_e4m3": [_VP, _I, _I, _I, _I, _VP, _VP, _VP],
+    "fa_fwd_fp8_quant": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I],
     "fa_bwd": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _I, _I, _I, _I,
                _I, _F, _I, _VP, _I],
     "fa_bwd_workspace_bytes": [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
@@ -135,6 +137,59 @@ def fa_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, H
     return library().fa_fwd_decode_paged(q, k_cache, v_cache, block_table, seq_lens, o, lse, B, H,
                                          d, page_size, max_pages_per_seq, num_pages, scale,
                                          stream, in_dtype, o_dtype, num_splits)
+
+
+def fa_quantize_e4m3(x, in_dtype, BH, N, d, codes, scales, stream) -> int:
+    return library().fa_quantize_e4m3(x, in_dtype, BH, N, d, codes, scales, stream)
+
+
+def fa_fwd_fp8_quant(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype,
+                     o_dtype) -> int:
+    return library().fa_fwd_fp8_quant(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream,
+                                      in_dtype, o_dtype)
+
+
+def fp8_quant_attention(q, k, v, causal: bool = False, scale: Optional[float] = None,
+                        out_dtype=None, stream=None):
+    """attention() with Q and K quantised to E4M3 on the fly (one scale per 128-row tile):
+    q [B,H,Nq,128], k/v [B,H,Nkv,128] contiguous fp16/bf16 CUDA tensors.  Returns (o, lse)."""
+    import torch
+
+    if not all(t.is_cuda and t.is_contiguous() for t in (q, k, v)):
+        raise ValueError("fp8_quant_attention() takes contiguous CUDA tensors")
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    out_dtype = torch.float32 if out_dtype is None else out_dtype
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((B, H, Nq, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    s = torch.cuda.current_stream(q.device) if stream is None else stream
+    with torch.cuda.device(q.device):
+        rc = fa_fwd_fp8_quant(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              lse.data_ptr(), B, H, Nq, Nkv, d, scale, int(bool(causal)),
+                              s.cuda_stream, _dtype_code(q.dtype), _dtype_code(o.dtype))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_fp8_quant")
+    return o, lse
+
+
+def quantize_e4m3(x, stream=None):
+    """E4M3 codes (uint8, x's shape) and per-128-row-tile scales (fp32 [B*H, ceil(N/128)])
+    of a contiguous CUDA tensor x [B, H, N, 128] (fp16/bf16)."""
+    import torch
+
+    if not (x.is_cuda and x.is_contiguous()) or x.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("quantize_e4m3() takes a contiguous fp16/bf16 CUDA tensor")
+    B, H, N, d = x.shape
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.empty((B * H, (N + 127) // 128), dtype=torch.float32, device=x.device)
+    s = torch.cuda.current_stream(x.device) if stream is None else stream
+    with torch.cuda.device(x.device):
+        rc = fa_quantize_e4m3(x.data_ptr(), _dtype_code(x.dtype), B * H, N, d, codes.data_ptr(),
+                              scales.data_ptr(), s.cuda_stream)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_quantize_e4m3")
+    return codes, scales
 
 
 def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, Nq, Nkv, d,
@@ -346,8 +401,8 @@ def fp8_attention(q8, k8, v, q_scale: float, k_scale: float, causal: bool = Fals
 
 def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: Optional[float] = None,
                        workspace=None, stream=None):
-    """dQ, dK, dV of attention() for the upstream gradient dout.  q, o, dout [B,H,Nq,128],
-    k, v [B,H,Nkv,128] contiguous CUDA tensors of one 16-bit dtype; o and lse are the
+    """dQ, dK, dV of attention() for the upstream gradient dout.  q, o, dout [B,H,Nq,d],
+    k, v [B,H,Nkv,d] (d 64 or 128) contiguous CUDA tensors of one 16-bit dtype; o and lse are the
     forward's outputs (o in the inputs' dtype, lse fp32 [B,H,Nq]).  workspace: optional
     uint8 CUDA tensor of at least fa_bwd_workspace_bytes; allocated when omitted.
     Returns (dq, dk, dv) in the inputs' dtype."""

@@ -16,7 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OBJDIR = os.path.join(ROOT, "_build")
 LIB_PATH = os.path.join(PKG, "libfa_b200.so")
-SOURCES = ["fa_api.cu", "fa_prefill.cu", "fa_decode.cu", "fa_noalloc.cu", "fa_backward.cu"]
+SOURCES = ["fa_api.cu", "fa_prefill.cu", "fa_decode.cu", "fa_noalloc.cu", "fa_backward.cu",
+           "fa_quant.cu"]
 HEADERS = ["fa_device.cuh", "fa_internal.h"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]

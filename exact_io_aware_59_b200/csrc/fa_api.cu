@@ -289,21 +289,32 @@ int run_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   p.n_qtiles = (max_q + 127) / 128;
   p.n_pairs = (p.n_qtiles + 1) / 2;
   p.n_kvtiles = (max_k + 127) / 128;
-  const long long units = static_cast<long long>(p.BH) * p.n_pairs;
+  // At most one item per (sequence, Q-tile pair) and H units per item.
+  const long long items = static_cast<long long>(B) * p.n_pairs;
+  const long long units = items * H;
   if (units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-  p.n_units = static_cast<int>(units);
+  p.n_units = static_cast<int>(units);  // an upper bound: the plan kernel counts the real ones
   p.scale_log2 = scale_log2(scale);
   p.cu_q = cu_q;
   p.cu_k = cu_k;
   p.H = H;
   p.total_q = total_q;
   p.total_k = total_k;
+  // Call-local workspace for the plan: item count (16 bytes), B sequence records, items.
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  const size_t ws_bytes = 16 + static_cast<size_t>(B) * sizeof(int4) + static_cast<size_t>(items) * 4;
+  if ((rc = workspace_alloc(ds, ws_bytes, st, &ws)) != FA_OK) return rc;
+  p.vl_count = static_cast<int*>(ws);
+  p.vl_seqs = reinterpret_cast<int4*>(static_cast<char*>(ws) + 16);
+  p.vl_items = reinterpret_cast<int*>(static_cast<char*>(ws) + 16 + static_cast<size_t>(B) * sizeof(int4));
   long long grid = ds->sm_count;
   if (grid > units) grid = units;
   if (grid < 1) grid = 1;
   cudaError_t e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, bf16, o_dtype == FA_F32,
-                                     static_cast<int>(grid), ds->status,
-                                     static_cast<cudaStream_t>(stream));
+                                     static_cast<int>(grid), ds->status, st);
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e == cudaSuccess) e = ef;
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
@@ -526,11 +537,11 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v, void* o, float* ls
 namespace {
 
 // Workspace layout of fa_bwd: -LSE*log2(e) [BH, nq_pad], D [BH, nq_pad], then the fp32
-// dQ accumulator [BH, nq_pad, 128]; nq_pad = Nq rounded up to 64 (each part a multiple of
-// 256 bytes).
-size_t bwd_ws_bytes(size_t BH, int Nq) {
-  const size_t nq_pad = (static_cast<size_t>(Nq) + 63) / 64 * 64;
-  return BH * nq_pad * (4 + 4 + 128 * 4);
+// dQ accumulator [BH, nq_pad, d]; nq_pad = Nq rounded up to 128 (each part a multiple of
+// 512 bytes).
+size_t bwd_ws_bytes(size_t BH, int Nq, int d) {
+  const size_t nq_pad = (static_cast<size_t>(Nq) + 127) / 128 * 128;
+  return BH * nq_pad * (4 + 4 + static_cast<size_t>(d) * 4);
 }
 
 }  // namespace
@@ -538,8 +549,8 @@ size_t bwd_ws_bytes(size_t BH, int Nq) {
 int fa_bwd_workspace_bytes(int B, int H, int Nq, int d, size_t* bytes) {
   if (!bytes || B < 1 || H < 1 || Nq < 1) return FA_ERR_INVALID_ARG;
   if (static_cast<long long>(B) * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
-  *bytes = bwd_ws_bytes(static_cast<size_t>(B) * H, Nq);
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  *bytes = bwd_ws_bytes(static_cast<size_t>(B) * H, Nq, d);
   return FA_OK;
 }
 
@@ -554,15 +565,15 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (in_dtype != FA_F16 && in_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   const void* a16[9] = {q, k, v, o, dout, dq, dk, dv, workspace};
   for (const void* ptr : a16)
     if (!aligned(ptr, 16)) return FA_ERR_INVALID_ARG;
   if (!aligned(lse, 4)) return FA_ERR_INVALID_ARG;
   const size_t BH = static_cast<size_t>(B) * H;
-  const size_t ws = bwd_ws_bytes(BH, Nq);
+  const size_t ws = bwd_ws_bytes(BH, Nq, d);
   if (workspace_bytes < ws) return FA_ERR_INVALID_ARG;
-  const long long n_ktiles = (Nkv + 127) / 128, n_qtiles = (Nq + 63) / 64;
+  const long long n_ktiles = (Nkv + 127) / 128, n_qtiles = (Nq + 127) / 128;
   if (static_cast<long long>(BH) * n_ktiles > 0x7fffffffLL ||
       static_cast<long long>(BH) * n_qtiles > 0x7fffffffLL)
     return FA_ERR_INVALID_ARG;
@@ -583,8 +594,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if ((rc = get_encoder()) != FA_OK) return rc;
   const bool bf16 = in_dtype == FA_BF16;
   CUtensorMap tq, tk, tv, tdo;
-  if ((rc = make_map(&tq, q, Nq, static_cast<long long>(BH), d, bf16, 64)) != FA_OK) return rc;
-  if ((rc = make_map(&tdo, dout, Nq, static_cast<long long>(BH), d, bf16, 64)) != FA_OK) return rc;
+  if ((rc = make_map(&tq, q, Nq, static_cast<long long>(BH), d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map(&tdo, dout, Nq, static_cast<long long>(BH), d, bf16)) != FA_OK) return rc;
   if ((rc = make_map(&tk, k, Nkv, static_cast<long long>(BH), d, bf16)) != FA_OK) return rc;
   if ((rc = make_map(&tv, v, Nkv, static_cast<long long>(BH), d, bf16)) != FA_OK) return rc;
   fa::BwdParams p{};
@@ -594,7 +605,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   p.off = Nkv - Nq;
   p.causal = causal;
   p.n_qtiles = static_cast<int>(n_qtiles);
-  p.nq_pad = p.n_qtiles * 64;
+  p.nq_pad = p.n_qtiles * 128;
   p.n_ktiles = static_cast<int>(n_ktiles);
   p.scale = scale;
   p.scale_log2 = scale_log2(scale);
@@ -604,8 +615,88 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   p.dq_acc = w + 2 * BH * p.nq_pad;
   p.dk = dk;
   p.dv = dv;
-  cudaError_t e = fa::launch_backward(tq, tk, tv, tdo, o, dout, lse, dq, p, bf16, ds->sm_count,
-                                      ds->status, static_cast<cudaStream_t>(stream));
+  cudaError_t e = fa::launch_backward(tq, tk, tv, tdo, o, dout, lse, dq, p, d, bf16,
+                                      ds->sm_count, ds->status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_fwd_fp8_quant(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
+                     int in_dtype, int o_dtype) {
+  int rc = check_args(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, in_dtype, o_dtype);
+  if (rc != FA_OK) return rc;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  DeviceState* ds = nullptr;
+  if ((rc = device_state(&ds)) != FA_OK) return rc;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+  const size_t BH = static_cast<size_t>(B) * H;
+  const int nqt = (Nq + 127) / 128, nkt = (Nkv + 127) / 128;
+  auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  // Call-local workspace: Q codes, K codes, Q tile scales, K tile scales.
+  const size_t qb = up256(BH * Nq * d), kb = up256(BH * Nkv * d);
+  const size_t qsb = up256(BH * nqt * 4), ksb = up256(BH * nkt * 4);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  if ((rc = workspace_alloc(ds, qb + kb + qsb + ksb, st, &ws)) != FA_OK) return rc;
+  char* w = static_cast<char*>(ws);
+  void* q8 = w;
+  void* k8 = w + qb;
+  float* qs = reinterpret_cast<float*>(w + qb + kb);
+  float* ks = reinterpret_cast<float*>(w + qb + kb + qsb);
+  const bool bf16 = in_dtype == FA_BF16;
+  cudaError_t e = fa::launch_quantize_e4m3(q, bf16, static_cast<long long>(BH), Nq, q8, qs, st);
+  if (e == cudaSuccess)
+    e = fa::launch_quantize_e4m3(k, bf16, static_cast<long long>(BH), Nkv, k8, ks, st);
+  CUtensorMap tq, tk, tv;
+  if (e == cudaSuccess) {
+    if ((rc = make_map_u8(&tq, q8, Nq, static_cast<long long>(BH), d)) != FA_OK ||
+        (rc = make_map_u8(&tk, k8, Nkv, static_cast<long long>(BH), d)) != FA_OK ||
+        (rc = make_map(&tv, v, Nkv, static_cast<long long>(BH), d, bf16)) != FA_OK) {
+      cudaFreeAsync(ws, st);
+      return rc;
+    }
+    fa::PrefillParams p{};
+    p.BH = static_cast<int>(BH);
+    p.Nq = Nq;
+    p.Nkv = Nkv;
+    p.off = Nkv - Nq;
+    p.causal = causal;
+    p.n_qtiles = nqt;
+    p.n_pairs = (nqt + 1) / 2;
+    p.n_kvtiles = nkt;
+    const long long units = static_cast<long long>(BH) * p.n_pairs;
+    p.n_units = static_cast<int>(units);
+    p.scale_log2 = scale_log2(scale);
+    p.H = H;
+    p.q_tscale = qs;
+    p.k_tscale = ks;
+    long long grid = ds->sm_count;
+    if (grid > units) grid = units;
+    if (grid < 1) grid = 1;
+    e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, bf16, o_dtype == FA_F32,
+                           static_cast<int>(grid), ds->status, st, true);
+  }
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (e == cudaSuccess) e = ef;
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_quantize_e4m3(const void* x, int in_dtype, int BH, int N, int d, void* codes,
+                     float* scales, void* stream) {
+  if (!x || !codes || !scales) return FA_ERR_INVALID_ARG;
+  if (BH < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (in_dtype != FA_F16 && in_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return FA_ERR_INVALID_ARG;
+  const size_t n = static_cast<size_t>(BH) * N * d;
+  const size_t sb = static_cast<size_t>(BH) * ((N + 127) / 128) * 4;
+  if (overlaps(codes, n, x, 2 * n) || overlaps(scales, sb, x, 2 * n) || overlaps(scales, sb, codes, n))
+    return FA_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  const int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  const cudaError_t e = fa::launch_quantize_e4m3(x, in_dtype == FA_BF16, BH, N, codes, scales,
+                                                 static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 

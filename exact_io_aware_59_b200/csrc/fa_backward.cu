@@ -13,43 +13,38 @@
 //
 // Three kernels, in stream order:
 //  * fa_bwd_prep: D and -LSE * log2(e) per query row (into a workspace padded to whole
-//    query tiles), and zeroes the fp32 dQ accumulator;
-//  * fa_bwd_sm100: one CTA per (key tile of 128, b*h).  It walks the query tiles of 64 that
-//    see its keys, keeps dK and dV for its keys in TMEM, and adds each step's dQ
-//    contribution into the fp32 accumulator with one bulk reduce-add (done at L2);
+//    128-row query tiles), and zeroes the fp32 dQ accumulator;
+//  * fa_bwd_sm100: one CTA per (key tile of 128, b*h).  It walks the query tiles of 128
+//    that see its keys, keeps dK and dV for its keys in TMEM, and adds each step's dQ
+//    contribution into the fp32 accumulator (coalesced reductions at L2);
 //  * fa_bwd_dq: dQ = scale * accumulator, converted to the inputs' 16-bit type.
 //
 // fa_bwd_sm100 roles (512 threads; our design for tcgen05, with keys as the MMA's M so the
-// per-key sums dK and dV stay in TMEM for the whole walk):
-//  * warp 0 (one lane): TMA loads of K and V once, then Q, dO, -LSE*log2e and D of each
-//    query tile into a 3-stage ring;
-//  * warp 1 (one lane): tcgen05.mma issue, per query tile i (b = i % 2):
-//        S^T  = K Q_i^T   (M 128 keys, N 64 queries, K = d)      into S[b]
-//        dP^T = V dO_i^T  (same shape)                            into dP[b]
-//        dV  += P^T dO_i  (A = P^T, 16-bit, from TMEM over S[b]; B = dO_i MN-major)
-//        dK  += dS^T Q_i  (A = dS^T, 16-bit, from TMEM over dP[b]; B = Q_i MN-major)
-//        dQ^T = K^T dS^T  (M 128 = d, N 64 queries, K 128 keys; A = K read MN-major,
-//                          B = dS[b] from shared memory)          into dP[b], over dS^T
-//    software-pipelined one tile deep: step i issues S(i+1), dP(i+1), then dV(i), dK(i),
-//    dQ(i) once warpgroup b has delivered P(i) and dS(i); only dP(i+1) waits for dQ(i-1)
-//    to be read out of dP[(i+1) % 2], and S(i+1) runs meanwhile.  The MMA lane is the
-//    critical path (the tensor pipe's issue queue is shallow), so a tile costs it just
-//    three waits and two commits: one commit covers S and dP, one covers the tile's last
-//    product (its dQ is then ready and its Q/dO stage free);
-//  * warpgroups 1 and 2 (warps 4-7 and 8-11) take the even and the odd query tiles, one
-//    thread per key: P^T from S^T and dS^T from dP^T, each written back to TMEM as 16-bit,
-//    dS also to shared memory.  With two, each has two tiles' time for one tile's work,
-//    so P(i) and dS(i) are ready before the MMA lane asks for them (one warpgroup alone
-//    measured about as fast, the MMA lane being the critical path).  At the end
-//    warpgroup 1 writes dV and warpgroup 2 writes scale * dK;
-//  * warpgroup 3 (warps 12-15), one thread per d-row of dQ^T: TMEM -> registers -> shared
-//    memory -> bulk reduce-add into the accumulator tile of query tile i.
-// Registers: the launch gives 128 per thread; warps 0-3 and 12-15 drop to kRegsSide and
-// warpgroups 1 and 2 rise to kRegsSoftmax (setmaxnreg).
-// TMEM (512 columns): dV [0,128) dK [128,256) S0 [256,320) S1 [320,384) dP0 [384,448)
-// dP1 [448,512); dQ(i) overwrites dP[b] once dK(i) has read dS^T(i) from it.  tcgen05.mma
-// operations run in issue order, so an MMA that overwrites columns an earlier MMA reads
-// as its A operand needs no wait in between.
+// per-key sums dK and dV stay in TMEM for the whole walk, and every product 128 x 128 --
+// the tensor core's full rate):
+//  * warp 0 (one lane): TMA loads of K and V once; per query tile i, Q_i with -LSE*log2e
+//    and D into a 2-stage ring, and dO_i into one buffer that is reloaded as soon as dV(i)
+//    has read it;
+//  * warp 1 (one lane): tcgen05.mma issue, per query tile i:
+//        dV  += P^T dO_i   (A = P^T, 16-bit, from TMEM over S; B = dO_i MN-major)
+//        dK  += dS^T Q_i   (A = dS^T, 16-bit, from TMEM over dP; B = Q_i MN-major)
+//        S^T  = K Q_{i+1}^T  (M 128 keys, N 128 queries, K = d) into S, once dV(i) is issued
+//        dQ^T = K^T dS^T   (M 128 = d, N 128 queries, K 128 keys; A = K read MN-major, B = dS
+//                           from shared memory) into dP, over dS^T once dK(i) is issued
+//        dP^T = V dO_{i+1}^T into dP, once the drain has read dQ^T(i) out of it
+//    tcgen05.mma operations run in issue order, so an MMA that overwrites columns an
+//    earlier MMA reads as its A operand needs no wait in between;
+//  * warpgroups 1 and 2 (warps 4-7 and 8-11) both work on every query tile, one thread per
+//    key, warpgroup w on queries 64w .. 64w+63: P^T from S^T as soon as S is ready, then
+//    dS^T = P^T (dP^T - D) once dP is; each stored back as 16-bit over the warpgroup's
+//    own S / dP columns (64w .. 64w+31), dS also to shared memory for the dQ product.  At
+//    the end warpgroup 1 writes dV and warpgroup 2 writes scale * dK;
+//  * warpgroup 3 (warps 12-15), one thread per d-row of dQ^T: TMEM -> registers (the
+//    columns are then free for dP(i+1)) -> fp32 reductions into row-major dQ accumulator
+//    rows, each warp instruction adding 32 consecutive floats of one query row.
+// Registers: the launch gives 128 per thread; warpgroup 0 drops to kRegsSide, the softmax
+// warpgroups rise to kRegsSoftmax and the drain warpgroup to kRegsDrain (setmaxnreg).
+// TMEM (512 columns): dV [0,128) dK [128,256) S [256,384) dP [384,512).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -59,36 +54,46 @@
 namespace fa {
 namespace {
 
-constexpr int kD = 128;        // head dimension
 constexpr int kBK = 128;       // keys per CTA (MMA M)
-constexpr int kBQ = 64;        // queries per step (MMA N of S^T, dP^T, dQ^T)
-constexpr int kStages = 3;     // Q / dO ring
+constexpr int kBQ = 128;       // queries per step (MMA N of S^T, dP^T, dQ^T; K of dV, dK)
+constexpr int kHalfQ = 64;     // queries per softmax warpgroup
+constexpr int kStages = 2;     // Q ring
 constexpr int kThreads = 512;
 constexpr int kRegsLaunch = 128;   // 65536 / 512
-constexpr int kRegsSide = 96;      // warps 0-3 and 12-15
-constexpr int kRegsSoftmax = 160;  // warps 4-11
-static_assert(256 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+constexpr int kRegsSide = 64;      // warps 0-3
+constexpr int kRegsSoftmax = 152;  // warps 4-11
+constexpr int kRegsDrain = 144;    // warps 12-15
+static_assert(128 * kRegsSide + 256 * kRegsSoftmax + 128 * kRegsDrain <= kThreads * kRegsLaunch,
+              "register split");
 
+// D: head dimension, 64 or 128.  A tile of 128 rows is D / 64 blocks of 128 rows x 128 B.
+template <int D>
 struct BwdCfg {
-  static constexpr int kKOff = 0;                           // K tile, 2 x (128 rows x 128 B)
-  static constexpr int kVOff = kKOff + kBK * kD * 2;        // V tile
-  static constexpr int kQOff = kVOff + kBK * kD * 2;        // Q stages, 2 x (64 x 128 B)
-  static constexpr int kQBytes = kBQ * kD * 2;
-  static constexpr int kdOOff = kQOff + kStages * kQBytes;  // dO stages
-  static constexpr int kdSOff = kdOOff + kStages * kQBytes; // dS x2, 128 keys x 64 queries
-  static constexpr int kdSBytes = kBK * kBQ * 2;
-  static constexpr int kStgOff = kdSOff + 2 * kdSBytes;     // dQ^T staging, fp32 128 x 64
-  static constexpr int kStgBytes = kD * kBQ * 4;
-  static constexpr int kLseOff = kStgOff + kStgBytes;       // -LSE*log2e per stage
+  static constexpr int kTileBytes = 128 * D * 2;           // 128 rows of D 16-bit values
+  static constexpr int kKOff = 0;                           // K tile
+  // The dQ product reads K as an MN-major A operand of M = 128 rows of d: for d = 64 the
+  // second 64-row block (one LBO, 16 KB, after K) is a block of zeros, so rows 64-127 of
+  // dQ^T come out 0 and are not drained.
+  static constexpr int kZeroOff = kKOff + kTileBytes;
+  static constexpr int kVOff = (D == 64) ? kZeroOff + 16384 : kKOff + kTileBytes;  // V tile
+  static constexpr int kQOff = kVOff + kTileBytes;          // Q stages
+  static constexpr int kdOOff = kQOff + kStages * kTileBytes;  // dO (one buffer)
+  static constexpr int kdSOff = kdOOff + kTileBytes;        // dS, 128 keys x 128 queries,
+                                                            // two 64-query blocks
+  static constexpr int kLseOff = kdSOff + kTileBytes;       // -LSE*log2e per stage
   static constexpr int kDelOff = kLseOff + kStages * kBQ * 4;  // D per stage
   static constexpr int kBarOff = kDelOff + kStages * kBQ * 4;
   // mbarriers
   static constexpr int kBarKV = 0;
-  static constexpr int kBarFull = 1;                 // + stage
-  static constexpr int kBarDPFull = 1 + kStages;     // + buffer: S(i) and dP(i) complete
-  static constexpr int kBarDSFull = kBarDPFull + 2;  // + buffer
-  static constexpr int kBarDQFull = kBarDSFull + 2;  // + buffer
-  static constexpr int kBarDQEmpty = kBarDQFull + 2;
+  static constexpr int kBarQFull = 1;                // + stage: Q, -LSE*log2e and D landed
+  static constexpr int kBarDOFull = kBarQFull + kStages;
+  static constexpr int kBarDOFree = kBarDOFull + 1;  // dV(i) done: the dO buffer may be reloaded
+  static constexpr int kBarSFull = kBarDOFree + 1;   // S(i) complete
+  static constexpr int kBarDPFull = kBarSFull + 1;   // dP(i) complete
+  static constexpr int kBarPReady = kBarDPFull + 1;  // P^T(i) stored (8 softmax warps)
+  static constexpr int kBarDSReady = kBarPReady + 1; // dS^T(i) and dS(i) stored (8 warps)
+  static constexpr int kBarDQFull = kBarDSReady + 1; // dQ^T(i) complete (and all before it)
+  static constexpr int kBarDQEmpty = kBarDQFull + 1; // dQ^T(i) read out of TMEM (4 warps)
   static constexpr int kBarDone = kBarDQEmpty + 1;   // every MMA of the CTA complete
   static constexpr int kBarFinished = kBarDone + 1;  // warps 4-15 done with TMEM
   static constexpr int kNumBars = kBarFinished + 1;
@@ -97,11 +102,17 @@ struct BwdCfg {
   static constexpr int kBytes = kAbortOff + 4;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
   static_assert(kAlloc <= 232448, "shared memory budget");
-  static_assert(kdSOff % 1024 == 0 && kQOff % 1024 == 0 && kdOOff % 1024 == 0, "swizzle atoms");
+  static_assert(kdSOff % 1024 == 0 && kQOff % 1024 == 0 && kdOOff % 1024 == 0 &&
+                kVOff % 1024 == 0, "swizzle atoms");
+  static_assert(D == 64 || D == 128, "head dimension");
 };
 
 // TMEM columns.
 constexpr uint32_t kTdV = 0, kTdK = 128, kTS = 256, kTdP = 384;
+
+// Column of the 16-bit A operand (P^T or dS^T, 8 columns per 16 queries) for K-step kk:
+// warpgroup w stores its queries 64w .. 64w+63 over its own columns 64w .. 64w+31.
+__device__ __forceinline__ uint32_t a16_col(int kk) { return (kk < 4) ? 8u * kk : 64u + 8u * (kk - 4); }
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t bars, int i) { return bars + 8u * i; }
 
@@ -129,128 +140,158 @@ __device__ __forceinline__ uint64_t kmajor_step(int kk, int rows) {
 }
 
 // ---------------------------------------------------------------- producer (TMA)
+template <int D>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                          const CUtensorMap* tdo, const BwdParams& p, int bh, int k0, int i0,
                          int n, uint32_t sbase, uint32_t bars, int* status,
                          volatile int* abort_flag) {
-  using C = BwdCfg;
+  using C = BwdCfg<D>;
   const uint32_t kv = bar_addr(bars, C::kBarKV);
-  mbar_arrive_expect_tx(kv, 4 * kBK * 64 * 2);
+  mbar_arrive_expect_tx(kv, 2 * C::kTileBytes);
 #pragma unroll
-  for (int sub = 0; sub < 2; ++sub) {
+  for (int sub = 0; sub < D / 64; ++sub) {
     tma_load_3d(sbase + C::kKOff + sub * kBK * 128, tk, kv, sub * 64, k0, bh);
     tma_load_3d(sbase + C::kVOff + sub * kBK * 128, tv, kv, sub * 64, k0, bh);
   }
-  int issued = 0;
+  int q_issued = 0, do_issued = 0;
   bool ok = true;
+  auto wait = [&](int b, uint32_t parity) {
+    return mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutBwd);
+  };
   for (int i = 0; i < n; ++i) {
     const int st = i % kStages;
-    // The stage held tile i - 3, whose products are all complete once its dQ is.
-    const int prev = i - kStages;
-    if (prev >= 0 && !mbar_wait(bar_addr(bars, C::kBarDQFull + (prev & 1)), (prev >> 1) & 1, status,
-                                abort_flag, kStatusTimeoutBwd)) {
-      ok = false;
-      break;
-    }
-    const uint32_t fb = bar_addr(bars, C::kBarFull + st);
-    mbar_arrive_expect_tx(fb, 2 * C::kQBytes + 2 * kBQ * 4);
     const int q0 = (i0 + i) * kBQ;
+    // Q stage st held tile i - 2, whose products are all complete once its dQ is (dQ(i-1)
+    // cannot complete before Q(i) is loaded, so the barrier is at most one phase ahead).
+    if (i >= kStages && !(ok = wait(C::kBarDQFull, (i - kStages) & 1))) break;
+    const uint32_t qf = bar_addr(bars, C::kBarQFull + st);
+    mbar_arrive_expect_tx(qf, C::kTileBytes + 2 * kBQ * 4);
 #pragma unroll
-    for (int sub = 0; sub < 2; ++sub) {
-      tma_load_3d(sbase + C::kQOff + st * C::kQBytes + sub * kBQ * 128, tq, fb, sub * 64, q0, bh);
-      tma_load_3d(sbase + C::kdOOff + st * C::kQBytes + sub * kBQ * 128, tdo, fb, sub * 64, q0, bh);
-    }
+    for (int sub = 0; sub < D / 64; ++sub)
+      tma_load_3d(sbase + C::kQOff + st * C::kTileBytes + sub * kBQ * 128, tq, qf, sub * 64, q0, bh);
     const size_t row = static_cast<size_t>(bh) * p.nq_pad + q0;
-    bulk_load(sbase + C::kLseOff + st * kBQ * 4, p.nlse2 + row, kBQ * 4, fb);
-    bulk_load(sbase + C::kDelOff + st * kBQ * 4, p.delta + row, kBQ * 4, fb);
-    ++issued;
+    bulk_load(sbase + C::kLseOff + st * kBQ * 4, p.nlse2 + row, kBQ * 4, qf);
+    bulk_load(sbase + C::kDelOff + st * kBQ * 4, p.delta + row, kBQ * 4, qf);
+    ++q_issued;
+    // dO: one buffer, free once dV(i-1) has read it.
+    if (i >= 1 && !(ok = wait(C::kBarDOFree, (i - 1) & 1))) break;
+    const uint32_t df = bar_addr(bars, C::kBarDOFull);
+    mbar_arrive_expect_tx(df, C::kTileBytes);
+#pragma unroll
+    for (int sub = 0; sub < D / 64; ++sub)
+      tma_load_3d(sbase + C::kdOOff + sub * kBQ * 128, tdo, df, sub * 64, q0, bh);
+    ++do_issued;
   }
   if (!ok) {
     // Let every copy still in flight land before the CTA's shared memory goes away.
-    for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-      drain_wait(bar_addr(bars, C::kBarFull + i % kStages), (i / kStages) & 1);
+    for (int i = (q_issued > kStages ? q_issued - kStages : 0); i < q_issued; ++i)
+      drain_wait(bar_addr(bars, C::kBarQFull + i % kStages), (i / kStages) & 1);
+    if (do_issued) drain_wait(bar_addr(bars, C::kBarDOFull), (do_issued - 1) & 1);
     drain_wait(kv, 0);
   }
 }
 
 // ---------------------------------------------------------------- MMA issuer
-template <bool BF16>
+template <int D, bool BF16>
 __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, int* status,
                            volatile int* abort_flag) {
-  using C = BwdCfg;
-  constexpr uint32_t idesc_s = make_idesc_f16(kBK, kBQ, BF16, false);       // S^T, dP^T
-  constexpr uint32_t idesc_kv = make_idesc_f16(kBK, kD, BF16, true);        // dV, dK
-  constexpr uint32_t idesc_q = make_idesc_f16_ab(kD, kBQ, BF16, true, true);  // dQ^T
-  const uint64_t k_desc = make_sdesc_sw128(sbase + C::kKOff, 16, 1024);
-  const uint64_t v_desc = make_sdesc_sw128(sbase + C::kVOff, 16, 1024);
+  using C = BwdCfg<D>;
+  constexpr uint32_t idesc_s = make_idesc_f16(kBK, kBQ, BF16, false);          // S^T, dP^T
+  constexpr uint32_t idesc_kv = make_idesc_f16(kBK, D, BF16, true);            // dV, dK
+  constexpr uint32_t idesc_q = make_idesc_f16_ab(128, kBQ, BF16, true, true);  // dQ^T (M = 128
+                                                                               // rows of d)
+  // Descriptors are rebuilt from these two bases where they are used (the bases pass
+  // through an opaque move each step), so the compiler does not keep all forty per-MMA
+  // descriptors of a step live at once.
+  uint64_t kmaj0 = make_sdesc_sw128(sbase, 16, 1024);           // K-major operands
+  uint64_t mn0 = make_sdesc_sw128(sbase, kBK * 128, 1024);      // MN-major operands
+  auto at = [](uint64_t base, uint32_t off) { return base + (off >> 4); };
+  auto k_desc = [&]() { return at(kmaj0, C::kKOff); };
+  auto v_desc = [&]() { return at(kmaj0, C::kVOff); };
   // K as the MN-major A of dQ^T: 64-row d blocks 128 x 128 B = 16 KB apart (LBO), 8-key
-  // groups 1024 B apart (SBO); 16 keys per step.
-  const uint64_t kt_desc = make_sdesc_sw128(sbase + C::kKOff, kBK * 128, 1024);
-  // dS as the MN-major B of dQ^T: one 128-byte row of 64 queries per key.
-  auto ds_desc = [&](int b) { return make_sdesc_sw128(sbase + C::kdSOff + b * C::kdSBytes, kBQ * 128, 1024); };
-  auto q_kmaj = [&](int st) { return make_sdesc_sw128(sbase + C::kQOff + st * C::kQBytes, 16, 1024); };
-  auto do_kmaj = [&](int st) { return make_sdesc_sw128(sbase + C::kdOOff + st * C::kQBytes, 16, 1024); };
-  // Q and dO as MN-major B (d contiguous): d blocks 64 x 128 B = 8 KB apart, 16 queries
+  // groups 1024 B apart (SBO); 16 keys (2048 B) per step.
+  auto kt_desc = [&]() { return at(mn0, C::kKOff); };
+  // dS as the MN-major B of dQ^T: two 64-query blocks 128 keys x 128 B = 16 KB apart.
+  auto ds_desc = [&]() { return at(mn0, C::kdSOff); };
+  auto q_kmaj = [&](int st) { return at(kmaj0, C::kQOff + st * C::kTileBytes); };
+  auto do_kmaj = [&]() { return at(kmaj0, C::kdOOff); };
+  // Q and dO as MN-major B (d contiguous): d blocks 128 x 128 B = 16 KB apart, 16 queries
   // (2048 B) per step.
-  auto q_mn = [&](int st) { return make_sdesc_sw128(sbase + C::kQOff + st * C::kQBytes, kBQ * 128, 1024); };
-  auto do_mn = [&](int st) { return make_sdesc_sw128(sbase + C::kdOOff + st * C::kQBytes, kBQ * 128, 1024); };
+  auto q_mn = [&](int st) { return at(mn0, C::kQOff + st * C::kTileBytes); };
+  auto do_mn = [&]() { return at(mn0, C::kdOOff); };
+  auto refresh = [&]() {
+    asm volatile("" : "+l"(kmaj0), "+l"(mn0));
+  };
   auto wait = [&](int b, uint32_t parity) {
     return mbar_wait_spin(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutBwd);
   };
   auto issue_st = [&](uint32_t d_col, uint64_t a, uint64_t b) {  // S^T or dP^T
 #pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk)
+    for (int kk = 0; kk < D / 16; ++kk)
       mma_ss(tmem + d_col, a + kmajor_step(kk, kBK), b + kmajor_step(kk, kBQ), idesc_s, kk > 0 ? 1u : 0u);
   };
   bool ok = n > 0 && wait(C::kBarKV, 0);  // with no query tile nothing is loaded
-  if (ok && (ok = wait(C::kBarFull + 0, 0))) {
-    issue_st(kTS, k_desc, q_kmaj(0));
-    issue_st(kTdP, v_desc, do_kmaj(0));
-    tc_commit(bar_addr(bars, C::kBarDPFull + 0));
+  if (ok && (ok = wait(C::kBarQFull + 0, 0))) {
+    tc_fence_after();
+    issue_st(kTS, k_desc(), q_kmaj(0));
+    tc_commit(bar_addr(bars, C::kBarSFull));
+    if ((ok = wait(C::kBarDOFull, 0))) {
+      tc_fence_after();
+      issue_st(kTdP, v_desc(), do_kmaj());
+      tc_commit(bar_addr(bars, C::kBarDPFull));
+    }
   }
   for (int i = 0; i < n && ok; ++i) {
-    const int b = i & 1, nb = b ^ 1, st = i % kStages;
-    const int st1 = (i + 1) % kStages;
-    if (i + 1 < n) {
-      if (!(ok = wait(C::kBarFull + st1, ((i + 1) / kStages) & 1))) break;
-      // S(i+1): S[nb] was last read by dV(i-1), issued earlier, and by warpgroup nb before
-      // it signalled dS(i-1).
-      issue_st(kTS + nb * kBQ, k_desc, q_kmaj(st1));
-      // dP(i+1) into dP[nb], once dQ(i-1) has been read out of it.
-      if (i > 0 && !(ok = wait(C::kBarDQEmpty, (i - 1) & 1))) break;
-      tc_fence_after();
-      issue_st(kTdP + nb * kBQ, v_desc, do_kmaj(st1));
-      tc_commit(bar_addr(bars, C::kBarDPFull + nb));  // S(i+1) and dP(i+1)
-    }
-    // Warpgroup b has stored P(i) over S[b] and dS^T(i) over dP[b], and dS(i) in shared memory.
-    if (!(ok = wait(C::kBarDSFull + b, (i >> 1) & 1))) break;
+    const int st = i % kStages, st1 = (i + 1) % kStages;
+    refresh();
+    // P^T(i) is stored over S: dV(i), then release the dO buffer.
+    if (!(ok = wait(C::kBarPReady, i & 1))) break;
     tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < kBQ / 16; ++kk)
-      mma_ts(tmem + kTdV, tmem + kTS + b * kBQ + kk * 8, do_mn(st) + ((kk * 2048) >> 4), idesc_kv,
+      mma_ts(tmem + kTdV, tmem + kTS + a16_col(kk), do_mn() + ((kk * 2048) >> 4), idesc_kv,
              (i > 0 || kk > 0) ? 1u : 0u);
+    tc_commit(bar_addr(bars, C::kBarDOFree));
+    // dS^T(i) is stored over dP and dS(i) in shared memory: dK(i).
+    if (!(ok = wait(C::kBarDSReady, i & 1))) break;
+    tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < kBQ / 16; ++kk)
-      mma_ts(tmem + kTdK, tmem + kTdP + b * kBQ + kk * 8, q_mn(st) + ((kk * 2048) >> 4), idesc_kv,
+      mma_ts(tmem + kTdK, tmem + kTdP + a16_col(kk), q_mn(st) + ((kk * 2048) >> 4), idesc_kv,
              (i > 0 || kk > 0) ? 1u : 0u);
-    // dQ(i) over dP[b]: dS^T(i) there has been read by dK(i), issued above.
+    // S(i+1) over S: P^T(i) there has been read by dV(i), issued above.
+    if (i + 1 < n) {
+      if (!(ok = wait(C::kBarQFull + st1, ((i + 1) / kStages) & 1))) break;
+      tc_fence_after();
+      issue_st(kTS, k_desc(), q_kmaj(st1));
+      tc_commit(bar_addr(bars, C::kBarSFull));
+    }
+    // dQ^T(i) over dP: dS^T(i) there has been read by dK(i), issued above.
 #pragma unroll
     for (int kk = 0; kk < kBK / 16; ++kk)
-      mma_ss(tmem + kTdP + b * kBQ, kt_desc + ((kk * 2048) >> 4), ds_desc(b) + ((kk * 2048) >> 4),
-             idesc_q, kk > 0 ? 1u : 0u);
-    // Tile i's products are complete: its dQ can be drained and its stage reloaded.
-    tc_commit(bar_addr(bars, C::kBarDQFull + b));
+      mma_ss(tmem + kTdP, kt_desc() + ((kk * 2048) >> 4), ds_desc() + ((kk * 2048) >> 4), idesc_q,
+             kk > 0 ? 1u : 0u);
+    // Tile i's products are complete: its dQ can be drained, its Q stage and dS reused.
+    tc_commit(bar_addr(bars, C::kBarDQFull));
+    if (i + 1 < n) {
+      // dP(i+1) over dP, once the drain has read dQ^T(i) and dO(i+1) has landed.
+      if (!(ok = wait(C::kBarDQEmpty, i & 1))) break;
+      if (!(ok = wait(C::kBarDOFull, (i + 1) & 1))) break;
+      tc_fence_after();
+      issue_st(kTdP, v_desc(), do_kmaj());
+      tc_commit(bar_addr(bars, C::kBarDPFull));
+    }
   }
   tc_commit(bar_addr(bars, C::kBarDone));
 }
 
 // ---------------------------------------------------------------- P and dS (one thread per key)
-// Warpgroup `wg` (0 or 1) takes query tiles i = wg, wg + 2, ... and buffers [wg].
-template <bool BF16>
+// Warpgroup `wg` (0 or 1) takes queries 64 wg .. 64 wg + 63 of every query tile.
+template <int D, bool BF16>
 __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, int wg,
                              uint8_t* sgen, uint32_t bars, uint32_t tmem, int* status,
                              volatile int* abort_flag) {
-  using C = BwdCfg;
+  using C = BwdCfg<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wq = warp & 3;
   const int r = wq * 32 + lane;  // key row of the tile = TMEM lane
@@ -260,26 +301,32 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
   const long long qvis = kidx >= p.Nkv ? (1ll << 40) : (p.causal ? static_cast<long long>(kidx) - p.off : -(1ll << 40));
   const bool key_tail = k0 + kBK > p.Nkv;
   const float sl2 = p.scale_log2;
+  const int c0 = wg * kHalfQ;  // this warpgroup's first query (and S / dP column) of the tile
   auto wait = [&](int b, uint32_t parity) {
     const bool ok = mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutBwd);
     return __all_sync(0xffffffffu, ok);
   };
+  auto arrive = [&](int b) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_addr(bars, b));
+  };
   bool ok = true;
-  for (int i = wg; i < n; i += 2) {
-    const int buf = wg, st = i % kStages;
+  for (int i = 0; i < n; ++i) {
+    const int st = i % kStages;
     const int q0 = (i0 + i) * kBQ;
-    if (!(ok = wait(C::kBarFull + st, (i / kStages) & 1))) break;  // LSE_i and D_i visible
-    if (!(ok = wait(C::kBarDPFull + buf, (i >> 1) & 1))) break;  // S(i) and dP(i)
+    if (!(ok = wait(C::kBarQFull + st, (i / kStages) & 1))) break;  // LSE_i and D_i visible
+    if (!(ok = wait(C::kBarSFull, i & 1))) break;                   // S(i)
     tc_fence_after();
-    const uint32_t tS = lane_base + kTS + buf * kBQ;
-    float pr[64];
+    const uint32_t tS = lane_base + kTS + c0;
+    float pr[kHalfQ];
     {
       uint32_t a[32], b[32];
       tmem_ld_32x32b_x32(tS, a);
       tmem_ld_32x32b_x32(tS + 32, b);
       tmem_ld_wait(a);
       reg_fence(b);
-      const float4* nl = reinterpret_cast<const float4*>(sgen + C::kLseOff + st * kBQ * 4);
+      const float4* nl = reinterpret_cast<const float4*>(sgen + C::kLseOff + st * kBQ * 4 + c0 * 4);
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
         const float4 l = nl[c4];
@@ -292,24 +339,27 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
     }
     // Causal diagonal or key tail: column c is visible iff q0 + c >= qvis.
     if (key_tail || (p.causal && k0 + kBK - 1 - p.off > q0)) {
-      const long long cm = qvis - q0;
-      const int cmin = cm < 0 ? 0 : (cm > kBQ ? kBQ : static_cast<int>(cm));
+      const long long cm = qvis - q0 - c0;
+      const int cmin = cm < 0 ? 0 : (cm > kHalfQ ? kHalfQ : static_cast<int>(cm));
 #pragma unroll
-      for (int c = 0; c < 64; ++c) pr[c] = (c >= cmin) ? pr[c] : 0.f;
+      for (int c = 0; c < kHalfQ; ++c) pr[c] = (c >= cmin) ? pr[c] : 0.f;
     }
     {
       uint32_t pk[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) pk[j] = pack2<BF16>(pr[2 * j], pr[2 * j + 1]);
-      tmem_st_32x32b_x32(tS, pk);
+      tmem_st_32x32b_x32(tS, pk);  // P^T over this warpgroup's first 32 S columns (read above)
     }
     tmem_st_wait();
-    // A block boundary between the P pass and the dS pass (ok is true here): interleaving
-    // the two needs more registers than this warpgroup's 160 and spills.
-    if (!__all_sync(0xffffffffu, ok)) break;
-    const float4* dl = reinterpret_cast<const float4*>(sgen + C::kDelOff + st * kBQ * 4);
-    uint8_t* ds_row = sgen + C::kdSOff + buf * C::kdSBytes + r * 128;
-    const uint32_t tdP = lane_base + kTdP + buf * kBQ;
+    arrive(C::kBarPReady);
+    // dS = P (dP - D) once dP(i) is complete (dQ(i-1), issued before dP(i), is complete
+    // too, so the shared-memory dS buffer is free).
+    if (!(ok = wait(C::kBarDPFull, i & 1))) break;
+    tc_fence_after();
+    const float4* dl = reinterpret_cast<const float4*>(sgen + C::kDelOff + st * kBQ * 4 + c0 * 4);
+    // dS row r (this key) of the 64-query block wg: 16-byte chunk cc at position cc ^ (r & 7).
+    uint8_t* ds_row = sgen + C::kdSOff + wg * (kBK * 128) + r * 128;
+    const uint32_t tdP = lane_base + kTdP + c0;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t dp[32];
@@ -327,10 +377,8 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
         pk[2 * c4] = pack2<BF16>(d0, d1);
         pk[2 * c4 + 1] = pack2<BF16>(d2, d3);
       }
-      // dS^T over the first 32 dP columns (16-bit pairs), already read.
+      // dS^T over this warpgroup's first 32 dP columns (16-bit pairs), already read.
       tmem_st_32x32b_x16(tdP + 16 * h, pk);
-      // dS for the dQ product: key row r, 16-byte chunk cc (queries 8cc..8cc+7) at chunk
-      // position cc ^ (r & 7) (128-byte swizzle).
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int cc = 4 * h + j;
@@ -340,9 +388,7 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
     }
     tmem_st_wait();
     fence_proxy_async_smem();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarDSFull + buf));
+    arrive(C::kBarDSReady);
   }
 
   // Epilogue: dV and scale * dK rows of this thread's key.
@@ -350,13 +396,13 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
   if (have) have = ok && wait(C::kBarDone, 0);
   if (n > 0 && !have) return;
   if (have) tc_fence_after();
-  const size_t orow = (static_cast<size_t>(bh) * p.Nkv + kidx) * kD;
+  const size_t orow = (static_cast<size_t>(bh) * p.Nkv + kidx) * D;
   {
     const int which = wg;  // warpgroup 1 writes dV, warpgroup 2 writes dK
     uint16_t* dst = static_cast<uint16_t*>(which ? p.dk : p.dv) + orow;
     const float mul = which ? p.scale : 1.f;
 #pragma unroll 1
-    for (int cc = 0; cc < kD / 32; ++cc) {
+    for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t v[32];
       if (have) {
         tmem_ld_32x32b_x32(lane_base + (which ? kTdK : kTdV) + 32 * cc, v);
@@ -382,54 +428,65 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
 }
 
 // ---------------------------------------------------------------- dQ drain (one thread per d)
-__device__ void dq_drain(const BwdParams& p, int bh, int i0, int n, uint8_t* sgen, uint32_t sbase,
-                         uint32_t bars, uint32_t tmem, int* status, volatile int* abort_flag) {
-  using C = BwdCfg;
+// *addr += v in global memory, done at L2 (no value returned).
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+template <int D>
+__device__ void dq_drain(const BwdParams& p, int bh, int i0, int n, uint32_t bars, uint32_t tmem,
+                         int* status, volatile int* abort_flag) {
+  using C = BwdCfg<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wq = warp & 3;
   const int t = wq * 32 + lane;  // d row of dQ^T = TMEM lane
-  const bool leader = (t == 0);
-  const uint32_t tq0 = tmem + (static_cast<uint32_t>(wq * 32) << 16) + kTdP;
-  uint8_t* stg_row = sgen + C::kStgOff + t * (kBQ * 4);
+  const bool live = t < D;       // warp-uniform: rows past d (zero padding for d = 64) are skipped
+  const uint32_t tq = tmem + (static_cast<uint32_t>(wq * 32) << 16) + kTdP;
   for (int i = 0; i < n; ++i) {
-    if (leader) bulk_wait_read_all();  // the previous tile's reduce has read the staging
-    const bool got = mbar_wait(bar_addr(bars, C::kBarDQFull + (i & 1)), (i >> 1) & 1, status, abort_flag,
+    const bool got = mbar_wait(bar_addr(bars, C::kBarDQFull), i & 1, status, abort_flag,
                                kStatusTimeoutBwd);
-    // One decision for the whole warpgroup, so no thread is left alone at a named barrier.
-    if (!named_sync_and(1, 128, got)) break;
+    if (!__all_sync(0xffffffffu, got)) break;
     tc_fence_after();
-    const uint32_t tq = tq0 + (i & 1) * kBQ;
-    uint32_t a[32], b[32];
-    tmem_ld_32x32b_x32(tq, a);
-    tmem_ld_32x32b_x32(tq + 32, b);
-    tmem_ld_wait(a);
-    reg_fence(b);
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarDQEmpty));
-    // Row t of the fp32 tile, 16-byte chunk c (queries 4c..4c+3) at position c ^ (t & 15).
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const uint32_t* s = c < 8 ? &a[4 * c] : &b[4 * (c - 8)];
-      *reinterpret_cast<uint4*>(stg_row + ((c ^ (t & 15)) << 4)) = make_uint4(s[0], s[1], s[2], s[3]);
+    if (!live) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarDQEmpty));
+      continue;
     }
-    fence_proxy_async_smem();
-    named_sync(1, 128);
-    if (leader) {
-      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.n_qtiles + i0 + i) * (kD * kBQ);
-      bulk_reduce_add_f32(dst, sbase + C::kStgOff, C::kStgBytes);
-      bulk_commit_group();
+    // Accumulator row q (query q0 + q) is D contiguous floats: a warp adds 32 consecutive
+    // ones per instruction.
+    float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.nq_pad + static_cast<size_t>(i0 + i) * kBQ) * D + t;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // queries 64h .. 64h+63
+      uint32_t a[2][32];
+      tmem_ld_32x32b_x32(tq + 64 * h, a[0]);
+      tmem_ld_32x32b_x32(tq + 64 * h + 32, a[1]);
+      tmem_ld_wait_only();
+      reg_fence(a[0]);
+      reg_fence(a[1]);
+      if (h == 1) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarDQEmpty));  // dP(i+1) may overwrite it
+      }
+      float* row = acc + static_cast<size_t>(64 * h) * D;
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          red_add_f32(row, __uint_as_float(a[c][q]));
+          row += D;
+        }
     }
   }
-  if (leader) bulk_wait_all();
 }
 
-template <bool BF16>
+template <int D, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_sm100(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                  const BwdParams p, int* __restrict__ status) {
-  using C = BwdCfg;
+  using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -448,17 +505,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_addr(bars, C::kBarKV), 1);
-    for (int s = 0; s < kStages; ++s) mbar_init(bar_addr(bars, C::kBarFull + s), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_addr(bars, C::kBarDPFull + b), 1);
-      mbar_init(bar_addr(bars, C::kBarDSFull + b), 4);  // one arrival per warp of warpgroup b+1
-      mbar_init(bar_addr(bars, C::kBarDQFull + b), 1);
-    }
-    mbar_init(bar_addr(bars, C::kBarDQEmpty), 4);    // one arrival per warp of warpgroup 3
+    for (int s = 0; s < kStages; ++s) mbar_init(bar_addr(bars, C::kBarQFull + s), 1);
+    mbar_init(bar_addr(bars, C::kBarDOFull), 1);
+    mbar_init(bar_addr(bars, C::kBarDOFree), 1);
+    mbar_init(bar_addr(bars, C::kBarSFull), 1);
+    mbar_init(bar_addr(bars, C::kBarDPFull), 1);
+    mbar_init(bar_addr(bars, C::kBarPReady), 8);     // one arrival per softmax warp
+    mbar_init(bar_addr(bars, C::kBarDSReady), 8);
+    mbar_init(bar_addr(bars, C::kBarDQFull), 1);
+    mbar_init(bar_addr(bars, C::kBarDQEmpty), 4);    // one arrival per drain warp
     mbar_init(bar_addr(bars, C::kBarDone), 1);
     mbar_init(bar_addr(bars, C::kBarFinished), 12);  // one per warp of warps 4-15
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if constexpr (D == 64) {
+    // The zero block of the padded K^T (16 KB, 32 bytes per thread), made visible to the
+    // tensor core before any MMA can read it.
+    uint4* z = reinterpret_cast<uint4*>(sgen + C::kZeroOff) + 2 * threadIdx.x;
+    z[0] = make_uint4(0u, 0u, 0u, 0u);
+    z[1] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tq);
@@ -477,12 +544,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // Each role runs to the end of the kernel on its own path: warps with different
   // register budgets never re-join.
-  if (warp < 4 || warp >= 12) {
+  if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
     if (warp == 0) {
-      if (lane == 0 && n > 0) producer(&tq, &tk, &tv, &tdo, p, bh, k0, i0, n, sbase, bars, status, abort_flag);
+      if (lane == 0 && n > 0) producer<D>(&tq, &tk, &tv, &tdo, p, bh, k0, i0, n, sbase, bars, status, abort_flag);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<BF16>(n, sbase, bars, tmem, status, abort_flag);
+      if (lane == 0) mma_issuer<D, BF16>(n, sbase, bars, tmem, status, abort_flag);
       __syncwarp();
       // Release TMEM once every MMA is complete and warps 4-15 are done with it.
       drain_wait(bar_addr(bars, C::kBarFinished), 0);
@@ -490,15 +557,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tc_fence_after();
       tmem_dealloc(tmem, 512);
-    } else if (warp >= 12) {
-      dq_drain(p, bh, i0, n, sgen, sbase, bars, tmem, status, abort_flag);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarFinished));
     }
+  } else if (warp >= 12) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
+    dq_drain<D>(p, bh, i0, n, bars, tmem, status, abort_flag);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarFinished));
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    softmax_grad<BF16>(p, bh, k0, i0, n, (warp - 4) >> 2, sgen, bars, tmem, status, abort_flag);
+    softmax_grad<D, BF16>(p, bh, k0, i0, n, (warp - 4) >> 2, sgen, bars, tmem, status, abort_flag);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarFinished));
@@ -506,25 +574,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- prep and dQ conversion
-// Per query row (16 threads, 16 bytes of O and dO each): D = dO . O, -LSE * log2(e), and
-// the row's 128 floats of the dQ accumulator zeroed.  Rows past Nq (padding of the last
+// Per query row (D/8 threads, 16 bytes of O and dO each): D = dO . O, -LSE * log2(e), and
+// the row's D floats of the dQ accumulator zeroed.  Rows past Nq (padding of the last
 // query tile) get D = 0 and -inf, so their P is 0.
-template <bool BF16>
+template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
     fa_bwd_prep(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                 const float* __restrict__ lse, const BwdParams p) {
+  constexpr int kTpr = D / 8;          // threads per row
+  constexpr int kRpw = 32 / kTpr;      // rows per warp
   const long long rows = static_cast<long long>(p.BH) * p.nq_pad;
-  const int sub = threadIdx.x & 15;
+  const int sub = threadIdx.x & (kTpr - 1);
   const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-  for (long long base = 2 * gw; base < rows; base += 2 * nw) {  // two rows per warp
-    const long long row = base + ((threadIdx.x >> 4) & 1);
+  for (long long base = kRpw * gw; base < rows; base += kRpw * nw) {
+    const long long row = base + ((threadIdx.x & 31) / kTpr);
     const bool in = row < rows;
     const int bh = in ? static_cast<int>(row / p.nq_pad) : 0;
     const int q = in ? static_cast<int>(row % p.nq_pad) : 0;
     float acc = 0.f;
     if (in && q < p.Nq) {
-      const size_t e = (static_cast<size_t>(bh) * p.Nq + q) * kD + sub * 8;
+      const size_t e = (static_cast<size_t>(bh) * p.Nq + q) * D + sub * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(o + e);
       const uint4 b = *reinterpret_cast<const uint4*>(dout + e);
       const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -538,84 +608,82 @@ __global__ void __launch_bounds__(256)
       }
     }
 #pragma unroll
-    for (int m = 8; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+    for (int m = kTpr / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
     if (!in) continue;
     if (sub == 0) {
       p.delta[row] = acc;
       p.nlse2[row] = q < p.Nq ? -lse[static_cast<size_t>(bh) * p.Nq + q] * 1.4426950408889634f : -INFINITY;
     }
-    float4* z = reinterpret_cast<float4*>(p.dq_acc + row * kD) + sub * 2;
+    float4* z = reinterpret_cast<float4*>(p.dq_acc + row * D) + sub * 2;
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
     z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
-// One block per (b*h, query tile): un-swizzles the tile's fp32 dQ^T accumulator through
-// shared memory and writes scale * dQ rows in the 16-bit type.
-template <bool BF16>
+// dQ = scale * accumulator in the 16-bit type: 8 values (one 16-byte store) per thread per
+// step, grid-stride over the B*H*Nq rows (padding rows of the accumulator are skipped).
+template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
     fa_bwd_dq(uint16_t* __restrict__ dq, const BwdParams p) {
-  __shared__ float t[kBQ][kD + 1];
-  const long long tile = blockIdx.x;
-  const int bh = static_cast<int>(tile / p.n_qtiles), qt = static_cast<int>(tile % p.n_qtiles);
-  const float4* src = reinterpret_cast<const float4*>(p.dq_acc + tile * (kD * kBQ));
-  for (int f = threadIdx.x; f < kD * kBQ / 4; f += blockDim.x) {
-    const float4 v = src[f];
-    const int dd = f >> 4, qq = ((f & 15) ^ (dd & 15)) << 2;
-    t[qq][dd] = v.x;
-    t[qq + 1][dd] = v.y;
-    t[qq + 2][dd] = v.z;
-    t[qq + 3][dd] = v.w;
-  }
-  __syncthreads();
-  for (int it = threadIdx.x; it < kBQ * kD / 8; it += blockDim.x) {
-    const int qq = it >> 4, g = it & 15;
-    const int q = qt * kBQ + qq;
-    if (q >= p.Nq) continue;
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      w[e] = pack2<BF16>(t[qq][8 * g + 2 * e] * p.scale, t[qq][8 * g + 2 * e + 1] * p.scale);
-    *reinterpret_cast<uint4*>(dq + (static_cast<size_t>(bh) * p.Nq + q) * kD + 8 * g) =
-        make_uint4(w[0], w[1], w[2], w[3]);
+  const long long total = static_cast<long long>(p.BH) * p.Nq * (D / 8);
+  for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long row = g / (D / 8);  // bh * Nq + q
+    const int c8 = static_cast<int>(g - row * (D / 8));
+    const long long bh = row / p.Nq, q = row - bh * p.Nq;
+    const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.nq_pad + q) * D + 8 * c8);
+    const float4 a = src[0], b = src[1];
+    uint4 w;
+    w.x = pack2<BF16>(a.x * p.scale, a.y * p.scale);
+    w.y = pack2<BF16>(a.z * p.scale, a.w * p.scale);
+    w.z = pack2<BF16>(b.x * p.scale, b.y * p.scale);
+    w.w = pack2<BF16>(b.z * p.scale, b.w * p.scale);
+    reinterpret_cast<uint4*>(dq)[g] = w;
   }
 }
 
-template <bool BF16>
+template <int D, bool BF16>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& tdo, const void* o, const void* dout, const float* lse,
                      void* dq, const BwdParams& p, int sm_count, int* status, cudaStream_t stream) {
-  auto kern = fa_bwd_sm100<BF16>;
+  auto kern = fa_bwd_sm100<D, BF16>;
   const cudaError_t config_err =
-      configure_kernel(reinterpret_cast<const void*>(kern), BwdCfg::kAlloc, kRegsLaunch);
+      configure_kernel(reinterpret_cast<const void*>(kern), BwdCfg<D>::kAlloc, kRegsLaunch);
   if (config_err != cudaSuccess) return config_err;
   const long long rows = static_cast<long long>(p.BH) * p.nq_pad;
-  long long prep_blocks = (rows + 15) / 16;  // 16 rows per 256-thread block
+  long long prep_blocks = (rows + 15) / 16;  // at least 16 rows per 256-thread block
   const long long cap = static_cast<long long>(sm_count) * 16;
   if (prep_blocks > cap) prep_blocks = cap;
   if (prep_blocks < 1) prep_blocks = 1;
-  fa_bwd_prep<BF16><<<static_cast<int>(prep_blocks), 256, 0, stream>>>(
+  fa_bwd_prep<D, BF16><<<static_cast<int>(prep_blocks), 256, 0, stream>>>(
       static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long grid = static_cast<long long>(p.BH) * p.n_ktiles;
-  kern<<<static_cast<int>(grid), kThreads, BwdCfg::kAlloc, stream>>>(tq, tk, tv, tdo, p, status);
+  kern<<<static_cast<int>(grid), kThreads, BwdCfg<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const long long tiles = static_cast<long long>(p.BH) * p.n_qtiles;
-  fa_bwd_dq<BF16><<<static_cast<int>(tiles), 256, 0, stream>>>(static_cast<uint16_t*>(dq), p);
+  const long long chunks = static_cast<long long>(p.BH) * p.Nq * (D / 8);
+  long long dq_blocks = (chunks + 255) / 256;
+  if (dq_blocks > cap) dq_blocks = cap;
+  fa_bwd_dq<D, BF16><<<static_cast<int>(dq_blocks), 256, 0, stream>>>(static_cast<uint16_t*>(dq), p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t backward_smem_bytes() { return BwdCfg::kAlloc; }
+size_t backward_smem_bytes(int d) { return d == 64 ? BwdCfg<64>::kAlloc : BwdCfg<128>::kAlloc; }
 
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const void* o, const void* dout,
-                            const float* lse, void* dq, const BwdParams& p, bool bf16,
+                            const float* lse, void* dq, const BwdParams& p, int d, bool bf16,
                             int sm_count, int* status, cudaStream_t stream) {
-  return bf16 ? launch_t<true>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream)
-              : launch_t<false>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream);
+  if (d == 128)
+    return bf16 ? launch_t<128, true>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream)
+                : launch_t<128, false>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream);
+  if (d == 64)
+    return bf16 ? launch_t<64, true>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream)
+                : launch_t<64, false>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace fa

@@ -72,6 +72,17 @@ __device__ __forceinline__ void chunk_info(const DecodeParams& p, const PagedKV&
   nk = min(kDecodeChunk, len - key0);
 }
 
+// Waits (bounded, ignoring the abort flag) for the copies of the last S stages issued, so
+// that none is still in flight when the CTA's shared memory goes away (error path only).
+template <int S>
+__device__ __forceinline__ void drain_ring(uint32_t bars, uint32_t ld) {
+  for (uint32_t i = (ld > static_cast<uint32_t>(S) ? ld - S : 0); i < ld; ++i) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bars + 8 * (i % S), (i / S) & 1))
+      if (global_timer_ns() - t0 > kWaitLimitNs) break;
+  }
+}
+
 template <int D, bool BF16>
 __device__ __forceinline__ void load_slice(const uint8_t* row, int lane, float (&x)[D / 32]) {
   constexpr int E = D / 32;  // elements per lane
@@ -115,58 +126,110 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t policy = l2_policy_evict_first();
-      uint32_t ld = 0;
-      bool ok = true;
-      for (long long c = c_begin; c < c_end; ++c) {
-        int h, key0, nk;
-        chunk_info<PAGED>(p, pk, c, h, key0, nk, status, true);
-        if (nk <= 0) continue;  // empty slot: no stage, the consumers skip it too
-        const uint32_t bytes = static_cast<uint32_t>(nk) * D * 2;
-        const uint32_t slot = ld % S;
-        if (!mbar_wait(bars + 8 * (S + slot), ((ld / S) & 1) ^ 1, status, abort_flag,
-                       kStatusTimeoutDecode)) {
-          ok = false;
-          break;
+    if constexpr (!PAGED) {
+      if (lane == 0) {
+        const uint64_t policy = l2_policy_evict_first();
+        uint32_t ld = 0;
+        bool ok = true;
+        for (long long c = c_begin; c < c_end; ++c) {
+          int h, key0, nk;
+          chunk_info<PAGED>(p, pk, c, h, key0, nk, status, true);
+          if (nk <= 0) continue;
+          const uint32_t bytes = static_cast<uint32_t>(nk) * D * 2;
+          const uint32_t slot = ld % S;
+          if (!mbar_wait(bars + 8 * (S + slot), ((ld / S) & 1) ^ 1, status, abort_flag,
+                         kStatusTimeoutDecode)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bars + 8 * slot;
+          mbar_arrive_expect_tx(fb, 2 * bytes);
+          const uint32_t dst = sbase + slot * C::kStageBytes;
+          const size_t off = (static_cast<size_t>(h) * p.Nkv + key0) * D;
+          bulk_load_stream(dst, k + off, bytes, fb, policy);
+          bulk_load_stream(dst + C::kChunkBytes, v + off, bytes, fb, policy);
+          ++ld;
         }
-        const uint32_t fb = bars + 8 * slot;
-        mbar_arrive_expect_tx(fb, 2 * bytes);
-        const uint32_t dst = sbase + slot * C::kStageBytes;
-        if constexpr (PAGED) {
-          // One copy per page the chunk touches: [key, key + seg) lies in logical page
-          // key >> page_shift of sequence b, at slot key & (page_size - 1).
-          const int b = h / pk.H, hh = h % pk.H;
-          const int ps = 1 << pk.page_shift;
-          for (int key = key0; key < key0 + nk;) {
-            const int in_page = key & (ps - 1);
-            const int seg = min(key0 + nk - key, ps - in_page);
+        if (!ok) drain_ring<S>(bars, ld);
+      }
+    } else {
+      // Paged cache: the whole warp.  Lane L looks up, 32 chunks ahead, the length and the
+      // block-table entries of chunk base + L, so the table reads (dependent global loads)
+      // are off the copy-issue path; then a chunk's K and V segments (one per page it
+      // touches: 1, 2 or 4) are issued by one lane each, in parallel.
+      const uint64_t policy = l2_policy_evict_first();
+      const int ps = 1 << pk.page_shift;
+      const int per_chunk = ps >= kDecodeChunk ? 1 : kDecodeChunk / ps;  // pages per chunk
+      auto lookup = [&](long long c, int& nk, int (&pg)[4]) {
+        nk = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pg[e] = 0;
+        if (c >= c_end) return;
+        int h, key0;
+        chunk_info<PAGED>(p, pk, c, h, key0, nk, status, true);
+        const int b = h / pk.H;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = key0 + e * ps;
+          if (e < per_chunk && key < key0 + nk) {
             int page = pk.block_table[static_cast<size_t>(b) * pk.max_pages + (key >> pk.page_shift)];
             if (page < 0 || page >= pk.num_pages) {
               atomicOr(status, kStatusBadInput);
               page = 0;
             }
-            const size_t off = ((static_cast<size_t>(page) * pk.H + hh) * ps + in_page) * D;
-            const uint32_t sb = static_cast<uint32_t>(seg) * D * 2;
-            const uint32_t so = static_cast<uint32_t>(key - key0) * D * 2;
-            bulk_load_stream(dst + so, k + off, sb, fb, policy);
-            bulk_load_stream(dst + C::kChunkBytes + so, v + off, sb, fb, policy);
-            key += seg;
+            pg[e] = page;
           }
-        } else {
-          const size_t off = (static_cast<size_t>(h) * p.Nkv + key0) * D;
-          bulk_load_stream(dst, k + off, bytes, fb, policy);
-          bulk_load_stream(dst + C::kChunkBytes, v + off, bytes, fb, policy);
         }
-        ++ld;
-      }
-      if (!ok) {
-        for (uint32_t i = (ld > (uint32_t)S ? ld - S : 0); i < ld; ++i) {
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(bars + 8 * (i % S), (i / S) & 1))
-            if (global_timer_ns() - t0 > kWaitLimitNs) break;
+      };
+      int cur_nk, cur_pg[4], nxt_nk, nxt_pg[4];
+      lookup(c_begin + lane, cur_nk, cur_pg);
+      uint32_t ld = 0;
+      bool ok = true;
+      for (long long base = c_begin; base < c_end && ok; base += 32) {
+        lookup(base + 32 + lane, nxt_nk, nxt_pg);  // in flight while this batch is issued
+        const int batch = static_cast<int>(min(32ll, c_end - base));
+        for (int i = 0; i < batch; ++i) {
+          const int nk = __shfl_sync(0xffffffffu, cur_nk, i);
+          if (nk <= 0) continue;  // empty slot: no stage, the consumers skip it too
+          const long long c = base + i;
+          const int h = static_cast<int>(c / p.n_chunks);
+          const int key0 = static_cast<int>(c % p.n_chunks) * kDecodeChunk;
+          const int hh = h % pk.H;
+          const uint32_t slot = ld % S;
+          const bool got = mbar_wait(bars + 8 * (S + slot), ((ld / S) & 1) ^ 1, status,
+                                     abort_flag, kStatusTimeoutDecode);
+          if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bars + 8 * slot;
+          if (lane == 0) mbar_arrive_expect_tx(fb, 2u * static_cast<uint32_t>(nk) * D * 2);
+          __syncwarp();
+          // Lane 2e copies the K segment in page e of the chunk, lane 2e + 1 its V segment.
+          const int e = lane >> 1;
+          int page = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int pj = __shfl_sync(0xffffffffu, cur_pg[j], i);
+            if (j == e) page = pj;
+          }
+          const int key = key0 + e * ps;
+          if (lane < 2 * per_chunk && key < key0 + nk) {
+            const int in_page = key & (ps - 1);
+            const int seg = min(key0 + nk - key, ps - in_page);
+            const size_t off = ((static_cast<size_t>(page) * pk.H + hh) * ps + in_page) * D;
+            const uint32_t so = static_cast<uint32_t>(key - key0) * D * 2;
+            const uint32_t dst = sbase + slot * C::kStageBytes + (lane & 1) * C::kChunkBytes + so;
+            bulk_load_stream(dst, ((lane & 1) ? v : k) + off, static_cast<uint32_t>(seg) * D * 2,
+                             fb, policy);
+          }
+          ++ld;
         }
+        cur_nk = nxt_nk;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cur_pg[e] = nxt_pg[e];
       }
+      if (!ok && lane == 0) drain_ring<S>(bars, ld);
     }
   } else {
     // ------------------------------------------------------------ consumers

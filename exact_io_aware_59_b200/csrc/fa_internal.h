@@ -25,26 +25,37 @@ struct PrefillParams {
   const int* cu_k;
   int H;            // heads per sequence (bh = b * H + h)
   int total_q, total_k;
+  // The packed batch's work list, built on the device by the plan kernel that runs before
+  // the prefill kernel (call-local workspace): the number of (sequence, Q-tile pair) items
+  // that hold query rows, each sequence's (q0, Lq, k0, Lk) after the bounds checks, and the
+  // items heaviest first, each as b * n_pairs + pair.  Work unit u is head u % H of item
+  // u / H.
+  const int* vl_count;
+  const int4* vl_seqs;
+  const int* vl_items;
+  // E4M3 queries and keys with one scale per 128-row tile (null: per-tensor scales folded
+  // into scale_log2): [BH, n_qtiles] and [BH, n_kvtiles].
+  const float* q_tscale;
+  const float* k_tscale;
 };
 
-// Work description of one backward launch ([B,H,N,d] layout, d = 128).
+// Work description of one backward launch ([B,H,N,d] layout, d = 64 or 128).
 struct BwdParams {
   int BH;
   int Nq, Nkv;
   int off;          // Nkv - Nq: causal query i sees keys j <= i + off
   int causal;
-  int n_qtiles;     // ceil(Nq / 64)
-  int nq_pad;       // n_qtiles * 64: rows of the per-row workspace arrays
+  int n_qtiles;     // ceil(Nq / 128)
+  int nq_pad;       // n_qtiles * 128: rows of the per-row workspace arrays
   int n_ktiles;     // ceil(Nkv / 128): one CTA per (key tile, b*h)
   float scale;
   float scale_log2; // scale * log2(e)
   // Workspace (written by the prep kernel): -LSE*log2(e) and D = rowsum(dO * O) per padded
-  // query row, and the fp32 dQ accumulator, one 128 x 64 tile (d-major, 16-byte chunks
-  // swizzled) per (b*h, query tile).
+  // query row, and the fp32 dQ accumulator, [BH, nq_pad, d] row-major.
   float* nlse2;
   float* delta;
   float* dq_acc;
-  void* dk;         // [BH, Nkv, 128], the inputs' 16-bit type
+  void* dk;         // [BH, Nkv, d], the inputs' 16-bit type
   void* dv;
 };
 
@@ -83,13 +94,18 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, 
                           float* part_lse, int* status, cudaStream_t stream,
                           const PagedKV* paged = nullptr);
 
-// Backward: prep, main and dQ-conversion kernels on `stream` (fa_backward.cu).  tq / tdo
-// are maps with 64-row boxes, tk / tv with 128-row boxes.
+// Backward: prep, main and dQ-conversion kernels on `stream` (fa_backward.cu).  All four
+// maps have 128-row boxes.
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const void* o, const void* dout,
-                            const float* lse, void* dq, const BwdParams& p, bool bf16,
+                            const float* lse, void* dq, const BwdParams& p, int d, bool bf16,
                             int sm_count, int* status, cudaStream_t stream);
-size_t backward_smem_bytes();
+size_t backward_smem_bytes(int d);
+
+// E4M3 codes of x [BH, N, 128] (16-bit) with one scale per 128-row tile of one head
+// (fa_quant.cu): codes [BH, N, 128] bytes, scales [BH, ceil(N / 128)] fp32.
+cudaError_t launch_quantize_e4m3(const void* x, bool bf16, long long BH, int N, void* codes,
+                                 float* scales, cudaStream_t stream);
 
 // Diagnostic kernel whose only wait can never finish (see fa_selftest_wait_timeout).
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t stream);

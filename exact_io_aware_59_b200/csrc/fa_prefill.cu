@@ -62,8 +62,9 @@ struct PrefillCfg {
   static constexpr int kBarFull = 2;                 // + slot
   static constexpr int kBarEmpty = 2 + kStages;      // + slot
   static constexpr int kBarSFull = 2 + 2 * kStages;  // + tile
-  static constexpr int kBarPFull = kBarSFull + 2;    // + tile
-  static constexpr int kBarODone = kBarPFull + 2;    // + tile
+  static constexpr int kBarPFull = kBarSFull + 2;    // + 2 * tile + half (keys 0-63, 64-127)
+  static constexpr int kBarOHalf = kBarPFull + 4;    // + tile: P V over the first 64 keys done
+  static constexpr int kBarODone = kBarOHalf + 2;    // + tile
   static constexpr int kBarDrain = kBarODone + 2;
   static constexpr int kBarDone = kBarDrain + 1;     // softmax warps finished with TMEM
   static constexpr int kNumBars = kBarDone + 1;
@@ -92,10 +93,7 @@ __device__ __forceinline__ int unit_of_round(int r) {
   return r * G + ((r & 1) ? (G - 1 - c) : c);
 }
 
-// One work unit: its (b*H + h, Q-tile pair) and the sequence it belongs to.  For a packed
-// variable-length batch the sequence's token ranges come from cu_q / cu_k, which live
-// on the device: a range outside [0, total] or longer than the longest sequence the
-// caller declared is clamped and, when `flag`, reported in the status word.
+// One work unit: its (b*H + h, Q-tile pair) and the sequence it belongs to.
 struct Unit {
   int bh, pair;
   int Lq, Lk;  // queries and keys of the sequence
@@ -103,34 +101,38 @@ struct Unit {
   int h;       // head within the sequence (packed layout)
 };
 
+// Work units of the launch.  A packed batch's count was written on the device by the plan
+// kernel (fa_varlen_plan) that ran before this kernel on the same stream.
 template <bool VARLEN>
-__device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u, int* status, bool flag) {
+__device__ __forceinline__ int unit_count(const PrefillParams& p) {
+  if constexpr (VARLEN) return *p.vl_count * p.H;
+  return p.n_units;
+}
+
+template <bool VARLEN>
+__device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u) {
   Unit x;
-  unit_coords(p, u, x.bh, x.pair);
   if constexpr (!VARLEN) {
+    unit_coords(p, u, x.bh, x.pair);
     x.Lq = p.Nq;
     x.Lk = p.Nkv;
     x.q0 = x.k0 = x.h = 0;
-    return x;
   } else {
-    const int b = x.bh / p.H;
-    x.h = x.bh % p.H;
-    int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
-    const bool bad = q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
-                     k1 > p.total_k || k1 - k0 > p.Nkv;
-    if (bad) {
-      if (flag) atomicOr(status, kStatusBadInput);
-      q0 = min(max(q0, 0), p.total_q);
-      q1 = min(max(q1, q0), min(p.total_q, q0 + p.Nq));
-      k0 = min(max(k0, 0), p.total_k);
-      k1 = min(max(k1, k0), min(p.total_k, k0 + p.Nkv));
-    }
-    x.q0 = q0;
-    x.Lq = q1 - q0;
-    x.k0 = k0;
-    x.Lk = k1 - k0;
-    return x;
+    // Head u % H of item u / H of the plan's list; the sequence's ranges were
+    // bounds-checked by the plan kernel.
+    const int it = u / p.H;
+    x.h = u - it * p.H;
+    const int item = p.vl_items[it];
+    const int b = item / p.n_pairs;
+    x.pair = item - b * p.n_pairs;
+    x.bh = b * p.H + x.h;
+    const int4 sq = p.vl_seqs[b];
+    x.q0 = sq.x;
+    x.Lq = sq.y;
+    x.k0 = sq.z;
+    x.Lk = sq.w;
   }
+  return x;
 }
 
 // Number of K/V tiles Q tile `qtile` of unit x must visit (0 when every row is fully
@@ -179,8 +181,9 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
   constexpr int S = C::kStages;
   uint32_t ld = 0, q_issued = 0;
   bool ok = true;
-  for (int rnd = 0, u = unit_of_round(0); u < p.n_units && ok; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of<VARLEN>(p, u, status, true);
+  const int n_units = unit_count<VARLEN>(p);
+  for (int rnd = 0, u = unit_of_round(0); u < n_units && ok; u = unit_of_round(++rnd)) {
+    const Unit x = unit_of<VARLEN>(p, u);
     const int pair = x.pair;
     const int n0 = kv_tiles_for(p, x, 2 * pair), n1 = kv_tiles_for(p, x, 2 * pair + 1);
     const int nmax = max(n0, n1);
@@ -264,11 +267,12 @@ __device__ __forceinline__ void issue_s(uint32_t d_tmem, uint64_t q_desc, uint64
   }
 }
 
+// O += P V over keys 64*half .. 64*half+63 of the tile (four K=16 steps).
 template <int D>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
-                                         uint32_t idesc, bool accumulate) {
+                                         uint32_t idesc, bool accumulate, int half) {
 #pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk) {
+  for (int kk = half * 4; kk < half * 4 + 4; ++kk) {
     // V is MN-major (d contiguous): 16 keys per step = two 1024-byte swizzle atoms;
     // the second 64-column block of d lies BN*128 bytes further (the descriptor's LBO).
     mma_ts(d_tmem, p_tmem + kk * 8, v_desc + ((kk * 16 * 128) >> 4), idesc,
@@ -294,8 +298,9 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
   auto wait = [&](int b, uint32_t parity) {
     return mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutMma);
   };
-  for (int rnd = 0, u = unit_of_round(0); u < p.n_units && ok; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of<VARLEN>(p, u, status, false);
+  const int n_units = unit_count<VARLEN>(p);
+  for (int rnd = 0, u = unit_of_round(0); u < n_units && ok; u = unit_of_round(++rnd)) {
+    const Unit x = unit_of<VARLEN>(p, u);
     const int n[2] = {kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)};
     const int nmax = max(n[0], n[1]);
     if (nmax == 0) continue;
@@ -325,11 +330,18 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (j >= n[t]) continue;
-        if (!mbar_wait_spin(bar_addr(bars, C::kBarPFull + t), pcount[t] & 1, status, abort_flag,
-                            kStatusTimeoutMma)) { ok = false; break; }
+        // P arrives in two halves (keys 0-63, then 64-127): the first half's products run
+        // while the softmax is still exponentiating the second.
+        if (!mbar_wait_spin(bar_addr(bars, C::kBarPFull + 2 * t), pcount[t] & 1, status,
+                            abort_flag, kStatusTimeoutMma)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, j > 0, 0);
+        tc_commit(bar_addr(bars, C::kBarOHalf + t));
+        if (!mbar_wait_spin(bar_addr(bars, C::kBarPFull + 2 * t + 1), pcount[t] & 1, status,
+                            abort_flag, kStatusTimeoutMma)) { ok = false; break; }
         ++pcount[t];
         tc_fence_after();
-        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, j > 0);
+        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, true, 1);
         tc_commit(bar_addr(bars, C::kBarODone + t));
         if (j + 1 < n[t]) {
           if (knext < 0) {
@@ -406,18 +418,46 @@ __device__ __forceinline__ void exp_pack32(const uint32_t (&s)[32], uint64_t sc2
   }
 }
 
-template <bool BF16, bool FULL>
-__device__ __forceinline__ void exp_pack_store32(const uint32_t (&s)[32], uint64_t sc2, uint64_t nm2,
-                                                 int col0, int lim_c, uint32_t tP,
-                                                 uint64_t (&acc)[4]) {
-  uint32_t pk[16];
-  float unused[2];
-  exp_pack32<BF16, FULL>(s, sc2, nm2, col0, lim_c, pk, acc, unused);
-  tmem_st_32x32b_x16(tP, pk);
+// P = 2^(s * scale_log2 - m_eff) for score chunks 2H and 2H+1 (keys 64H .. 64H+63 of the
+// tile), stored as 16-bit pairs over S columns 32H .. 32H+31.  Returns the sum of the
+// unrounded p and sets xh to the largest exponent s * scale_log2 - m_eff of those keys
+// (-inf when none is visible).  all_visible: every column visible (else columns past lim_c
+// get p = 0; their scores must already hold the masking sentinel).
+template <bool BF16, int H>
+__device__ __forceinline__ float exp_half(const uint32_t (&s)[4][32], uint64_t sc2, float m_eff,
+                                          bool all_visible, int lim_c, uint32_t tS, float& xh) {
+  const uint64_t nm2 = f2_pack(-m_eff, -m_eff);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int c = 2 * H; c < 2 * H + 2; ++c) {
+    uint32_t pk[16];
+    if (all_visible)
+      exp_pack32<BF16, true, true>(s[c], sc2, nm2, 32 * c, lim_c, pk, acc, mx);
+    else
+      exp_pack32<BF16, false, true>(s[c], sc2, nm2, 32 * c, lim_c, pk, acc, mx);
+    tmem_st_32x32b_x16(tS + 16 * c, pk);
+  }
+  xh = fmaxf(mx[0], mx[1]);
+  float a0, a1;
+  f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+  return a0 + a1;
+}
+
+// round16(p) - p for the largest p = 2^xh of a half tile (0 when xh = -inf).
+template <bool BF16>
+__device__ __forceinline__ float round_error(float xh) {
+  if (xh == -INFINITY) return 0.f;
+  const float pmax = ex2(xh);
+  float r0, r1;
+  unpack2<BF16>(pack2<BF16>(pmax, 0.f), r0, r1);
+  return r0 - pmax;
 }
 
 // NEG: the scale is negative, so the row maximum of scale * s comes from the minimum of s.
-template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN>
+// QK8: E4M3 queries and keys; with per-tile scales (p.q_tscale, p.k_tscale) each score
+// tile's factor is scale * (its Q tile's scale) * (its K tile's scale).
+template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN, bool QK8>
 __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t tmem, void* o,
                                  float* lse, int t, int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -427,8 +467,6 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
   const uint32_t tS = lane_base + t * 128;
   const uint32_t tO = lane_base + 256 + t * D;
-  const float scale_log2 = p.scale_log2;
-  const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
   uint32_t s_seen = 0, o_seen = 0;
   // Warp-uniform result: tcgen05.ld/st below are warp-collective, so a warp never splits
   // on a wait that finished on some lanes and ran out on others.
@@ -437,8 +475,9 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     return __all_sync(0xffffffffu, ok);
   };
 
-  for (int rnd = 0, u = unit_of_round(0); u < p.n_units; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of<VARLEN>(p, u, status, false);
+  const int n_units = unit_count<VARLEN>(p);
+  for (int rnd = 0, u = unit_of_round(0); u < n_units; u = unit_of_round(++rnd)) {
+    const Unit x = unit_of<VARLEN>(p, u);
     const int qtile = 2 * x.pair + t;
     if (qtile * BM >= x.Lq) continue;
     const int n_kv = kv_tiles_for(p, x, qtile);
@@ -450,68 +489,100 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     float l = 0.f;             // running sum of the 16-bit-rounded 2^(x - m_used): divides O
     float l_exact = 0.f;       // the same sum before rounding: gives LSE
 
+    // O_t *= alpha for this thread's row (TMEM round trip; the rare lazy-rescale path).
+    auto rescale_o = [&](float alpha) {
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ob[32];
+        tmem_ld_32x32b_x32(tO + cc * 32, ob);
+        tmem_ld_wait(ob);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
+        tmem_st_32x32b_x32(tO + cc * 32, ob);
+      }
+    };
+    // Hands keys 64*h .. 64*h+63 of this tile's P (and any O rescale) to the MMA lane.
+    auto release = [&](int h) {
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarPFull + 2 * t + h));  // one per warp
+    };
+
+    // The score factor in log2 units (per tile with per-tile FP8 scales).
+    float sl2_q = p.scale_log2;
+    if constexpr (QK8) {
+      if (p.q_tscale) sl2_q *= p.q_tscale[static_cast<size_t>(x.bh) * p.n_qtiles + qtile];
+    }
     for (int j = 0; j < n_kv; ++j) {
+      float scale_log2 = sl2_q;
+      if constexpr (QK8) {  // loaded before the wait, which hides its latency
+        if (p.k_tscale) scale_log2 *= p.k_tscale[static_cast<size_t>(x.bh) * p.n_kvtiles + j];
+      }
       if (!wait(C::kBarSFull + t, s_seen & 1)) return;
       ++s_seen;
       tc_fence_after();
+      const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
       const int lim_c = limit - j * BN;  // columns c <= lim_c are visible for this row
       const bool full = __all_sync(0xffffffffu, lim_c >= BN - 1);  // warp-uniform path
-      // p = 2^(x - m_eff) for the row, stored as P over the first 64 S columns (16-bit,
-      // two per column, 16 columns per 32 scores); returns the sum of the unrounded p.
-      auto exp_pass = [&](const uint32_t (&s)[4][32], float m_eff, bool all_visible) {
-        const uint64_t nm2 = f2_pack(-m_eff, -m_eff);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (all_visible)
-            exp_pack_store32<BF16, true>(s[c], sc2, nm2, 32 * c, lim_c, tS + 16 * c, acc);
-          else
-            exp_pack_store32<BF16, false>(s[c], sc2, nm2, 32 * c, lim_c, tS + 16 * c, acc);
-        }
-        float a0, a1;
-        f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
-        return a0 + a1;
-      };
       uint32_t s[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
       tmem_ld_wait_only();
 #pragma unroll
       for (int c = 0; c < 4; ++c) reg_fence(s[c]);
-      float xm, rs_exact;  // xm: largest x - m_eff of the row's visible scores (-inf if none)
+      // O and l are divided by, and LSE taken from, sums over P: l sums the 16-bit-rounded
+      // P the P V product uses, taken as the unrounded sum plus the rounding error of each
+      // half tile's largest P (the term that decides a row whose weight sits on a few keys;
+      // the other terms' errors, relative 2^-9 for bf16 and 2^-12 for fp16 of either sign,
+      // average out); l_exact sums the unrounded P.
       bool done = false;
       if (full && __all_sync(0xffffffffu, m_used != -INFINITY)) {
         // Once a row has a finite reference max, a tile with every column visible rarely
-        // moves it: exponentiate against it straight away, taking the row max of the
-        // exponents in the same pass, so the reduction is off the path to P, and store each
-        // chunk of P as soon as it is packed.  P overwrites S columns 0-63 (score chunks 0
-        // and 1, which stay in registers); chunks 2 and 3 stay intact in TMEM.  If the max
-        // moved by more than kLazyLog2 anywhere in the warp, the tile is redone below from
-        // those; P has not been released yet.
-        const uint64_t nm2 = f2_pack(-m_used, -m_used);
-        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-        float mx[2] = {-INFINITY, -INFINITY};
+        // moves it: exponentiate against it straight away, taking each half's largest
+        // exponent in the same pass, and hand each half of P to the MMA lane as soon as it
+        // is known not to move the max of any row of the warp by more than kLazyLog2.
+        float xa;
+        const float ra = exp_half<BF16, 0>(s, sc2, m_used, true, lim_c, tS, xa);
+        if (!__any_sync(0xffffffffu, xa > kLazyLog2)) {
+          release(0);
+          l += ra + round_error<BF16>(xa);
+          l_exact += ra;
+          float xb;
+          const float rb = exp_half<BF16, 1>(s, sc2, m_used, true, lim_c, tS, xb);
+          if (!__any_sync(0xffffffffu, xb > kLazyLog2)) {
+            l += rb + round_error<BF16>(xb);
+            l_exact += rb;
+          } else {
+            // Keys 64-127 move the max of some row of the warp after keys 0-63 went out
+            // against the old reference: bring l and O (once P V over keys 0-63 is done)
+            // to the new reference, then redo keys 64-127 against it.
+            const bool move = xb > kLazyLog2;
+            const float alpha = move ? ex2(-xb) : 1.0f;
+            if (move) {
+              l *= alpha;
+              l_exact *= alpha;
+              m_used += xb;
+            }
+            if (!wait(C::kBarOHalf + t, (o_seen + j) & 1)) return;
+            tc_fence_after();
+            rescale_o(alpha);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-          exp_pack32<BF16, true, true>(s[c], sc2, nm2, 32 * c, lim_c, pk, acc, mx);
-          tmem_st_32x32b_x16(tS + 16 * c, pk);
-        }
-        xm = fmaxf(mx[0], mx[1]);
-        done = !__any_sync(0xffffffffu, xm > kLazyLog2);
-        if (done) {
-          float a0, a1;
-          f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
-          rs_exact = a0 + a1;
-        } else {
+            for (int c = 2; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
+            tmem_ld_wait_only();
 #pragma unroll
-          for (int c = 2; c < 4; ++c) tmem_ld_32x32b_x32(tS + c * 32, s[c]);
-          tmem_ld_wait_only();
-#pragma unroll
-          for (int c = 2; c < 4; ++c) reg_fence(s[c]);
+            for (int c = 2; c < 4; ++c) reg_fence(s[c]);
+            float xb2;
+            const float rb2 = exp_half<BF16, 1>(s, sc2, m_used, true, lim_c, tS, xb2);
+            l += rb2 + round_error<BF16>(xb2);
+            l_exact += rb2;
+          }
+          done = true;
         }
       }
       if (!done) {
+        // Two passes: the row max of the raw scores (masking what this row may not see),
+        // then the exponents.  Nothing of this tile has been handed out yet.
         if (!full) {
           const float sentinel = NEG ? INFINITY : -INFINITY;
 #pragma unroll
@@ -532,42 +603,22 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
           l_exact *= alpha;
           m_used = m_new;
         }
-        const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-        rs_exact = exp_pass(s, m_eff, full);
-        xm = (m_tile == -INFINITY) ? -INFINITY : fmaf(mr, scale_log2, -m_eff);
         if (j > 0 && __any_sync(0xffffffffu, move)) {
-          // O_t still holds P V of tiles < j: wait for the last of those products, then
-          // bring it to the new reference (before P is released to the next product).
+          // O_t holds P V of tiles < j (complete: S(j), ready above, was issued after it):
+          // bring it to the new reference before this tile's P goes out.
           if (!wait(C::kBarODone + t, (o_seen + j - 1) & 1)) return;
           tc_fence_after();
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t ob[32];
-            tmem_ld_32x32b_x32(tO + cc * 32, ob);
-            tmem_ld_wait(ob);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ob[i] = __float_as_uint(__uint_as_float(ob[i]) * alpha);
-            tmem_st_32x32b_x32(tO + cc * 32, ob);
-          }
+          rescale_o(alpha);
         }
+        const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+        float xa, xb;
+        const float ra = exp_half<BF16, 0>(s, sc2, m_eff, full, lim_c, tS, xa);
+        release(0);
+        const float rb = exp_half<BF16, 1>(s, sc2, m_eff, full, lim_c, tS, xb);
+        l += ra + rb + round_error<BF16>(xa) + round_error<BF16>(xb);
+        l_exact += ra + rb;
       }
-      // O is divided by the row sum of the rounded P that the P V product uses, taken as the
-      // unrounded sum plus the rounding error of each tile's largest P.  That one term
-      // dominates when a row's weight sits on a few keys; the other terms' errors (relative
-      // 2^-9 for bf16, 2^-12 for fp16, either sign) average out over many comparable keys.
-      float rs = rs_exact;
-      if (xm != -INFINITY) {
-        const float pmax = ex2(xm);
-        float r0, r1;
-        unpack2<BF16>(pack2<BF16>(pmax, 0.f), r0, r1);
-        rs += r0 - pmax;
-      }
-      l += rs;
-      l_exact += rs_exact;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarPFull + t));  // one arrival per warp
+      release(1);
     }
 
     // Epilogue: O = O_t / l and LSE = (m + log2 l) * ln 2.
@@ -643,7 +694,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_addr(bars, C::kBarSFull + t), 1);
-      mbar_init(bar_addr(bars, C::kBarPFull + t), 4);  // one arrival per softmax warp
+      mbar_init(bar_addr(bars, C::kBarPFull + 2 * t), 4);      // one arrival per softmax warp
+      mbar_init(bar_addr(bars, C::kBarPFull + 2 * t + 1), 4);
+      mbar_init(bar_addr(bars, C::kBarOHalf + t), 1);
       mbar_init(bar_addr(bars, C::kBarODone + t), 1);
     }
     mbar_init(bar_addr(bars, C::kBarDrain), 1);
@@ -682,12 +735,101 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    // (Per-tile FP8 scales are positive: they never change the score factor's sign.)
     if (p.scale_log2 < 0.f)
-      softmax_epilogue<D, BF16, OF32, true, VARLEN>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, true, VARLEN, QK8>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     else
-      softmax_epilogue<D, BF16, OF32, false, VARLEN>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, false, VARLEN, QK8>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     tc_fence_before();
     mbar_arrive(bar_addr(bars, C::kBarDone));
+  }
+}
+
+// ---------------------------------------------------------------- packed-batch plan
+// Builds the work list of a packed batch before the prefill kernel runs (one CTA): every
+// sequence's token ranges are bounds-checked once (a range outside [0, total] or longer
+// than the declared maximum is clamped and reported in the status word), and every
+// (sequence, Q-tile pair) that holds query rows becomes one item, listed heaviest first by
+// its K/V tile count (a counting sort; the order within one weight is whatever the
+// atomics give, which changes no result: a unit's rows do not depend on where it runs).
+// The persistent kernel then deals out items x heads in its snake order, with no empty
+// units and no per-unit read of the offsets.
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBuckets = 2 * kPlanThreads;  // weights above kPlanBuckets - 1 share a bucket
+
+__global__ void __launch_bounds__(kPlanThreads)
+    fa_varlen_plan(const PrefillParams p, int B, int* __restrict__ count, int4* __restrict__ seqs,
+                   int* __restrict__ items, int* __restrict__ status) {
+  __shared__ int bucket[kPlanBuckets];
+  __shared__ int warp_total[kPlanThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  bool bad = false;
+  for (int b = tid; b < B; b += kPlanThreads) {
+    int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+    if (q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
+        k1 > p.total_k || k1 - k0 > p.Nkv) {
+      bad = true;
+      q0 = min(max(q0, 0), p.total_q);
+      q1 = min(max(q1, q0), min(p.total_q, q0 + p.Nq));
+      k0 = min(max(k0, 0), p.total_k);
+      k1 = min(max(k1, k0), min(p.total_k, k0 + p.Nkv));
+    }
+    seqs[b] = make_int4(q0, q1 - q0, k0, k1 - k0);
+  }
+  if (bad) atomicOr(status, kStatusBadInput);
+  for (int i = tid; i < kPlanBuckets; i += kPlanThreads) bucket[i] = 0;
+  __syncthreads();  // also makes the seqs writes visible to the whole CTA
+  const long long n_items = static_cast<long long>(B) * p.n_pairs;
+  // Bucket of item i (heaviest first), or -1 when its Q tiles hold no query row.
+  auto bucket_of = [&](long long i) {
+    const int b = static_cast<int>(i / p.n_pairs);
+    const int pr = static_cast<int>(i - static_cast<long long>(b) * p.n_pairs);
+    const int4 sq = seqs[b];
+    Unit x;
+    x.bh = 0;
+    x.h = 0;
+    x.pair = pr;
+    x.q0 = sq.x;
+    x.Lq = sq.y;
+    x.k0 = sq.z;
+    x.Lk = sq.w;
+    if (2 * pr * BM >= x.Lq) return -1;
+    const int w = kv_tiles_for(p, x, 2 * pr) + kv_tiles_for(p, x, 2 * pr + 1);
+    return kPlanBuckets - 1 - min(w, kPlanBuckets - 1);
+  };
+  for (long long i = tid; i < n_items; i += kPlanThreads) {
+    const int bk = bucket_of(i);
+    if (bk >= 0) atomicAdd(&bucket[bk], 1);
+  }
+  __syncthreads();
+  // Exclusive prefix sum of the bucket counts: thread t owns buckets 2t and 2t+1.
+  const int c0 = bucket[2 * tid], c1 = bucket[2 * tid + 1];
+  int incl = c0 + c1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) warp_total[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int t = warp_total[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += n;
+    }
+    warp_total[lane] = t;
+  }
+  __syncthreads();
+  const int excl = incl - (c0 + c1) + (warp > 0 ? warp_total[warp - 1] : 0);
+  bucket[2 * tid] = excl;  // each thread rewrites only its own two buckets
+  bucket[2 * tid + 1] = excl + c0;
+  if (tid == kPlanThreads - 1) *count = excl + c0 + c1;
+  __syncthreads();
+  for (long long i = tid; i < n_items; i += kPlanThreads) {
+    const int bk = bucket_of(i);
+    if (bk >= 0) items[atomicAdd(&bucket[bk], 1)] = static_cast<int>(i);
   }
 }
 
@@ -718,6 +860,14 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
     if (bf16) return launch_t<128, true, false, false, true>(tq, tk, tv, o, lse, p, grid, status, stream);
     if (o_f32) return launch_t<128, false, true, false, true>(tq, tk, tv, o, lse, p, grid, status, stream);
     return launch_t<128, false, false, false, true>(tq, tk, tv, o, lse, p, grid, status, stream);
+  }
+  if (p.cu_q) {
+    // Packed batch: the plan kernel writes the work list the prefill kernel reads.
+    fa_varlen_plan<<<1, kPlanThreads, 0, stream>>>(p, p.BH / p.H, const_cast<int*>(p.vl_count),
+                                                   const_cast<int4*>(p.vl_seqs),
+                                                   const_cast<int*>(p.vl_items), status);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
 #define FA_PREFILL_CASE(D_, B_, F_)                                                               \
   if (d == D_ && bf16 == B_ && o_f32 == F_)                                                        \

@@ -1,0 +1,104 @@
+// fa_quant.cu -- E4M3 quantisation of queries and keys with one scale per 128-row tile.
+//
+// The FP8 path of "FlashAttention 1-2-3" (myaihardware), section "FlashAttention-3: FP8,
+// Async Warp Overlap, and Hopper-Specific Optimizations", feeds the tensor cores FP8
+// queries and keys quantised on the fly.  Here a tile of 128 consecutive rows of one head
+// (the prefill kernel's Q or K tile, d = 128) shares one scale: scale = max|x| / 448 over
+// the tile (1 for an all-zero tile), code = E4M3(x / scale), rounded to nearest even and
+// saturated at +-448.  A scale per tile rather than per tensor needs no pass over the
+// whole tensor before the first code is written, and it keeps small-magnitude tiles
+// accurate.  The prefill kernel multiplies each score tile by its Q tile's and K tile's
+// scales.  Memory bound: 2 bytes read and 1 written per element.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fa_device.cuh"
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+constexpr int kQuantThreads = 256;
+constexpr int kTileRows = 128;
+constexpr int kD = 128;
+// One tile is 128 rows x 256 bytes = 2048 16-byte chunks: 8 per thread, chunk i of thread t
+// at index t + 256 i (consecutive threads read consecutive 16 bytes).
+constexpr int kChunksPerThread = kTileRows * kD * 2 / 16 / kQuantThreads;
+
+// Two fp32 values to a packed E4M3 pair (round to nearest even, saturating to +-448),
+// `lo` in the low byte.
+__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kQuantThreads)
+    fa_quantize_e4m3_tiles(const uint4* __restrict__ x, int N, int n_tiles,
+                           uint2* __restrict__ codes, float* __restrict__ scales) {
+  __shared__ float warp_max[kQuantThreads / 32];
+  const long long bh = blockIdx.x / n_tiles;
+  const int tile = blockIdx.x - static_cast<int>(bh * n_tiles);
+  const int rows = min(kTileRows, N - tile * kTileRows);
+  const size_t base = (static_cast<size_t>(bh) * N + static_cast<size_t>(tile) * kTileRows) * (kD / 8);
+  uint4 raw[kChunksPerThread];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kChunksPerThread; ++i) {
+    const int c = threadIdx.x + kQuantThreads * i;
+    if (c / (kD / 8) < rows) {
+      raw[i] = x[base + c];
+      const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float a, b;
+        unpack2<BF16>(w[e], a, b);
+        amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = warp_max[0];
+#pragma unroll
+  for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, warp_max[w]);
+  const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
+  if (threadIdx.x == 0) scales[blockIdx.x] = scale;
+#pragma unroll
+  for (int i = 0; i < kChunksPerThread; ++i) {
+    const int c = threadIdx.x + kQuantThreads * i;
+    if (c / (kD / 8) < rows) {
+      const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+      uint16_t q[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float a, b;
+        unpack2<BF16>(w[e], a, b);
+        q[e] = e4m3x2(a / scale, b / scale);
+      }
+      codes[base + c] = make_uint2(q[0] | (static_cast<uint32_t>(q[1]) << 16),
+                                   q[2] | (static_cast<uint32_t>(q[3]) << 16));
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_e4m3(const void* x, bool bf16, long long BH, int N, void* codes,
+                                 float* scales, cudaStream_t stream) {
+  const int n_tiles = (N + kTileRows - 1) / kTileRows;
+  const long long blocks = BH * n_tiles;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  if (bf16)
+    fa_quantize_e4m3_tiles<true><<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(
+        static_cast<const uint4*>(x), N, n_tiles, static_cast<uint2*>(codes), scales);
+  else
+    fa_quantize_e4m3_tiles<false><<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(
+        static_cast<const uint4*>(x), N, n_tiles, static_cast<uint2*>(codes), scales);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

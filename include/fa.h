@@ -160,6 +160,36 @@ int fa_fwd_fp8(const void* q8, const void* k8, const void* v, void* o, float* ls
                float q_scale, float k_scale, int v_dtype, int o_dtype);
 
 /*
+ * fa_fwd_fp8_quant -- prefill with queries and keys quantised to FP8 on the fly
+ * ("FlashAttention 1-2-3" (myaihardware), section "FlashAttention-3: FP8, Async Warp
+ * Overlap, and Hopper-Specific Optimizations").  Same arguments, layouts and errors as
+ * fa_fwd (q, k, v in in_dtype; d must be 128; Nq > 1 or 1).  Q and K are quantised with
+ * fa_quantize_e4m3 (one scale per 128-row tile) into call-local workspace from the
+ * library's stream-ordered pool; then S = Q8 K8^T runs on tcgen05 kind::f8f6f4 and each
+ * score tile is multiplied by scale and its two tile scales; P and V stay in in_dtype.
+ * The result is softmax(scale * Qd Kd^T [+ causal]) V with Qd, Kd the dequantised tensors.
+ */
+int fa_fwd_fp8_quant(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
+                     int in_dtype, int o_dtype);
+
+/*
+ * fa_quantize_e4m3 -- E4M3 codes of a [BH, N, d] tensor with one scale per tile of 128
+ * consecutive rows of one head ("FlashAttention 1-2-3" (myaihardware), section
+ * "FlashAttention-3: FP8, Async Warp Overlap, and Hopper-Specific Optimizations": queries
+ * and keys quantised to FP8 on the fly).
+ *   x: [BH, N, d] in in_dtype (FA_F16 or FA_BF16), 16-byte aligned; d must be 128.
+ *   codes: [BH, N, d] bytes (16-byte aligned); scales: [BH, ceil(N/128)] fp32.
+ *   For the tile of rows 128t .. 128t+127 of head bh: scales[bh][t] = max|x| / 448 in fp32
+ *   (1 for an all-zero tile) and code = E4M3(x / scale) in fp32, rounded to nearest even
+ *   and saturated at +-448 (the "fn" variant: no infinities).  x ~ decode(code) * scale.
+ *   Buffers are device memory owned by the caller and must not overlap.  Enqueues one
+ *   kernel on `stream`.
+ */
+int fa_quantize_e4m3(const void* x, int in_dtype, int BH, int N, int d, void* codes,
+                     float* scales, void* stream);
+
+/*
  * fa_fwd_varlen -- prefill over a packed batch of sequences of different lengths
  * ("FlashAttention 1-2-3" (myaihardware), section "When FlashAttention Doesn't Help":
  * continuous batching, each sequence of the batch an independent problem).
@@ -220,7 +250,7 @@ int fa_fwd_decode_paged(const void* q, const void* k_cache, const void* v_cache,
  *   P is recomputed on chip tile by tile; nothing of size Nq x Nkv is stored.
  *   q, o, dout, dq [B,H,Nq,d]; k, v, dk, dv [B,H,Nkv,d]; all in_dtype (FA_F16 or FA_BF16),
  *   contiguous, 16-byte aligned.  lse [B,H,Nq] fp32 natural log as fa_fwd writes it (a
- *   row with no visible key has -inf and gets dQ = 0).  d must be 128.
+ *   row with no visible key has -inf and gets dQ = 0).  d must be 64 or 128.
  *   workspace: caller-owned device memory of at least fa_bwd_workspace_bytes bytes,
  *   16-byte aligned; overwritten (it holds the fp32 dQ accumulator and per-row D and lse).
  *   dq, dk, dv and the workspace must not overlap each other or any input.
@@ -233,7 +263,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            size_t workspace_bytes, int B, int H, int Nq, int Nkv, int d, float scale,
            int causal, void* stream, int in_dtype);
 
-/* Bytes of workspace an fa_bwd call with these sizes needs (B*H*ceil(Nq/64)*64*520). */
+/* Bytes of workspace an fa_bwd call with these sizes needs (B*H*ceil(Nq/128)*128*(8+4d)). */
 int fa_bwd_workspace_bytes(int B, int H, int Nq, int d, size_t* bytes);
 
 /* Bytes of decode workspace a fa_fwd_decode call with these arguments needs. */

@@ -27,7 +27,10 @@ Contents
                               Module 12.3" section "Prefill vs Decode", "Training").
 ``paged_decode_attention``,   attention() over a paged KV cache, over a packed batch of
 ``varlen_attention``,         sequences, and over FP8 (E4M3) queries and keys decoded
-``fp8_qk_attention``          from the format's definition (``e4m3_to_f64``).
+``fp8_qk_attention``          from the format's definition (``e4m3_to_f64``), with one
+``fp8_tile_scaled_attention`` scale per tensor or one per 128-row tile.
+``e4m3_encode``,              quantisation to E4M3 written from the format (round to
+``e4m3_quantize_tiles``       nearest even, saturating), with per-tile scales.
 ``lse_combine``               merges partial results over disjoint key sets by their
                               log-sum-exp, the reduction step of split-KV decoding
                               ("FlashAttention 1-2-3" section "Beyond FlashAttention":
@@ -236,6 +239,75 @@ def e4m3_to_f64(bits):
     mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
     out = sign * mag
     return np.where((e == 15) & ((b & 7) == 7), np.nan, out)
+
+
+def e4m3_encode(x):
+    """E4M3 ("fn") codes of float32 values: round to the nearest representable value, ties
+    to the even mantissa, magnitudes beyond the largest finite value 448 saturate to +-448
+    (no infinities).  Written from the format: for a normal magnitude 2^e * (1 + f) the
+    representable neighbours are spaced 2^(e - 3) apart; below 2^-6 (the subnormals
+    m * 2^-9) the spacing is 2^-9.  Returns a numpy uint8 array of x's shape."""
+    a = np.asarray(x, dtype=np.float32).astype(np.float64)
+    sign = np.signbit(a)
+    mag = np.abs(a)
+    _, e = np.frexp(mag)            # mag = f * 2^e with f in [0.5, 1): floor(log2 mag) = e - 1
+    e = e.astype(np.int64) - 1
+    normal = mag >= 2.0 ** -6
+    spacing = np.where(normal, np.exp2(np.maximum(e, -6) - 3.0), 2.0 ** -9)
+    q = np.round(mag / spacing)     # numpy rounds halves to even: ties to the even mantissa
+    # normal: q in [8, 16]; q == 16 carries into the next binade
+    code_n = np.where(q >= 16, ((e + 1 + 7) << 3) | 0, ((e + 7) << 3) | (q.astype(np.int64) - 8))
+    code_s = q.astype(np.int64)      # subnormal: 0..8 (8 is the smallest normal, code 0x08)
+    code = np.where(normal, code_n, code_s)
+    code = np.where(mag >= 448.0, 0x7E, code)   # saturate (this also covers rounding past 448)
+    code = np.minimum(code, 0x7E)
+    return (code | (sign.astype(np.int64) << 7)).astype(np.uint8)
+
+
+def e4m3_quantize_tiles(x, tile_rows: int = 128):
+    """Quantises x [BH, N, d] (any float type, taken exactly as float32) to E4M3 codes
+    with one scale per tile of `tile_rows` consecutive rows of one head: scale =
+    float32(max |x| over the tile) / 448 in float32 arithmetic (1 when the tile is all
+    zero), code = e4m3_encode(float32(x) / scale) with a float32 division.  Returns (codes
+    uint8 [BH, N, d], scales float32 [BH, ceil(N / tile_rows)]): x ~ codes * scale."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().to(torch.float32).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.asarray(x, dtype=np.float32)
+    BH, N, d = x.shape
+    nt = (N + tile_rows - 1) // tile_rows
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    scales = np.ones((BH, nt), dtype=np.float32)
+    for t in range(nt):
+        blk = x[:, t * tile_rows:(t + 1) * tile_rows]
+        amax = np.abs(blk).reshape(BH, -1).max(axis=1).astype(np.float32)
+        sc = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+        scales[:, t] = sc
+        codes[:, t * tile_rows:(t + 1) * tile_rows] = e4m3_encode(blk / sc[:, None, None])
+    return codes, scales
+
+
+def fp8_tile_scaled_attention(q8, q_scales, k8, k_scales, v, scale: float, causal: bool,
+                              tile_rows: int = 128, rows=None, nthreads: int = 0, lib=None):
+    """attention() of FP8 queries and keys with one scale per tile of `tile_rows` rows:
+    q8 [B,H,Nq,d], k8 [B,H,Nkv,d] E4M3 codes; q_scales [B*H, ceil(Nq/tile_rows)] and
+    k_scales [B*H, ceil(Nkv/tile_rows)]; row i of head bh stands for
+    decode(q8[.., i, :]) * q_scales[bh, i // tile_rows] (likewise for keys).  fp64."""
+    import torch
+    q8 = np.asarray(q8.cpu().numpy() if hasattr(q8, "cpu") else q8)
+    k8 = np.asarray(k8.cpu().numpy() if hasattr(k8, "cpu") else k8)
+    B, H, Nq, d = q8.shape
+    Nkv = k8.shape[2]
+    qs = np.repeat(np.asarray(q_scales, dtype=np.float64), tile_rows, axis=1)[:, :Nq]
+    ks = np.repeat(np.asarray(k_scales, dtype=np.float64), tile_rows, axis=1)[:, :Nkv]
+    qf = e4m3_to_f64(q8) * qs.reshape(B, H, Nq, 1)
+    kf = e4m3_to_f64(k8) * ks.reshape(B, H, Nkv, 1)
+    vf = torch.as_tensor(v).detach().cpu().to(torch.float64)
+    return attention(torch.from_numpy(qf), torch.from_numpy(kf), vf, scale, causal, rows=rows,
+                     nthreads=nthreads, lib=lib)
 
 
 def fp8_qk_attention(q8, k8, v, q_scale: float, k_scale: float, scale: float, causal: bool,

@@ -131,7 +131,10 @@ calls = {
     "fa_fwd_decode_paged": lambda: b.fa_fwd_decode_paged(Q, K, V, L + 64, L + 128, O, L, 1, 1,
                                                          64, 16, 4, 8, 0.1, None, 0, 2, 0),
     "fa_bwd": lambda: b.fa_bwd(Q, K, V, O, L, Q + 4096, O + 4096, O + 8192, O + 12288,
-                               O + 65536, 64 * 520, 1, 1, 4, 4, 128, 0.1, 0, None, 1),
+                               O + 65536, 128 * 520, 1, 1, 4, 4, 128, 0.1, 0, None, 1),
+    "fa_quantize_e4m3": lambda: b.fa_quantize_e4m3(Q, 1, 2, 100, 128, O, L, None),
+    "fa_fwd_fp8_quant": lambda: b.fa_fwd_fp8_quant(Q, K, V, O, L, 1, 2, 16, 16, 128, 0.1, 1,
+                                                   None, 1, 2),
     "fa_device_status": lambda: lib.fa_device_status(ctypes.byref(ctypes.c_int(0)), 0),
     "fa_selftest_wait_timeout": lambda: lib.fa_selftest_wait_timeout(None),
     "fa_release_workspace": lambda: lib.fa_release_workspace(),
@@ -255,7 +258,7 @@ def test_fp8_entry_checks():
 
 def test_backward_entry_checks():
     """fa_bwd refuses bad arguments on the host, before touching any device."""
-    ws_ok = 1 * 1 * 64 * 520
+    ws_ok = 1 * 1 * 128 * 520
     args = dict(q=Q, k=K, v=V, o=O, lse=L, do=Q + 4096, dq=O + 4096, dk=O + 8192, dv=O + 12288,
                 ws=O + 65536, wsb=ws_ok, B=1, H=1, Nq=4, Nkv=4, d=128, scale=0.1, causal=0,
                 stream=None, dt=1)
@@ -267,7 +270,7 @@ def test_backward_entry_checks():
                               a["dv"], a["ws"], a["wsb"], a["B"], a["H"], a["Nq"], a["Nkv"],
                               a["d"], a["scale"], a["causal"], a["stream"], a["dt"])
 
-    assert call(d=64) == binding.FA_ERR_UNSUPPORTED
+    assert call(d=96) == binding.FA_ERR_UNSUPPORTED
     assert call(lse=None) == binding.FA_ERR_INVALID_ARG
     assert call(ws=None) == binding.FA_ERR_INVALID_ARG
     assert call(wsb=ws_ok - 16) == binding.FA_ERR_INVALID_ARG   # workspace too small
@@ -279,8 +282,10 @@ def test_backward_entry_checks():
     assert call(dq=Q) == binding.FA_ERR_INVALID_ARG             # output overlaps an input
     assert call(dv=O + 8192) == binding.FA_ERR_INVALID_ARG      # two outputs overlap
     assert binding.fa_bwd_workspace_bytes(2, 3, 65, 128) == 2 * 3 * 128 * 520
+    assert binding.fa_bwd_workspace_bytes(1, 1, 129, 128) == 256 * 520
+    assert binding.fa_bwd_workspace_bytes(1, 1, 64, 64) == 128 * (8 + 4 * 64)
     with pytest.raises(binding.FaError):
-        binding.fa_bwd_workspace_bytes(1, 1, 64, 64)
+        binding.fa_bwd_workspace_bytes(1, 1, 64, 96)
 
 
 def _declared_param_counts():
@@ -303,3 +308,13 @@ def test_binding_signatures_match_the_header():
     for name, argtypes in binding._SIGNATURES.items():
         assert name in counts, name
         assert len(argtypes) == counts[name], (name, len(argtypes), counts[name])
+
+
+def test_quantize_entry_checks():
+    q = binding.fa_quantize_e4m3
+    assert q(Q, 1, 2, 100, 64, O, L, None) == binding.FA_ERR_UNSUPPORTED      # d must be 128
+    assert q(None, 1, 2, 100, 128, O, L, None) == binding.FA_ERR_INVALID_ARG
+    assert q(Q, 2, 2, 100, 128, O, L, None) == binding.FA_ERR_INVALID_ARG     # fp32 input
+    assert q(Q, 1, 0, 100, 128, O, L, None) == binding.FA_ERR_INVALID_ARG
+    assert q(Q + 8, 1, 2, 100, 128, O, L, None) == binding.FA_ERR_INVALID_ARG  # misaligned
+    assert q(Q, 1, 2, 100, 128, Q + 1024, L, None) == binding.FA_ERR_INVALID_ARG  # codes on x

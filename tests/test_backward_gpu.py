@@ -161,3 +161,34 @@ def test_backward_workspace_reuse_and_size():
     refs = oracle.attention_backward(q, k, v, g, 128 ** -0.5, True)
     _check([t.cpu() for t in r2], refs, torch.bfloat16, what="reuse")
     assert torch.equal(r1[1], r2[1]) and torch.equal(r1[2], r2[2])
+
+
+CASES_D64 = [
+    # B, H, Nq, Nkv, causal, dtype
+    (1, 2, 256, 256, False, torch.float16),
+    (2, 3, 200, 200, True, torch.float16),      # ragged last query and key tiles
+    (1, 2, 130, 300, True, torch.bfloat16),     # Nq < Nkv: bottom-right diagonal
+    (1, 2, 300, 130, True, torch.float16),      # Nq > Nkv: the first rows see no key
+]
+
+
+@pytest.mark.parametrize("B,H,Nq,Nkv,causal,dtype", CASES_D64)
+def test_backward_d64_matches_oracle(B, H, Nq, Nkv, causal, dtype):
+    """d = 64: K^T for the dQ product is padded to 128 rows with a zero block."""
+    q, k, v = make_qkv(B, H, Nq, Nkv, 64, dtype, 3800 + Nq + Nkv)
+    g = make_grad_out(B, H, Nq, 64, dtype, 3803 + Nq + Nkv)
+    scale = 64 ** -0.5
+    ours = _run(q, k, v, g, causal, scale)
+    refs = oracle.attention_backward(q, k, v, g, scale, causal)
+    _check(ours, refs, dtype, what=f"d64 {B}x{H}x{Nq}x{Nkv} causal={causal}")
+
+
+def test_backward_prefill_mha_every_head():
+    """The prefill MHA workload (B=2, H=8, N=2048, d=64, fp16, causal), every head."""
+    from exact_io_aware_59_b200.inputs import WORKLOADS, workload_qkv
+    w = WORKLOADS["prefill_mha"]
+    q, k, v = workload_qkv(w)
+    g = make_grad_out(w.B, w.H, w.Nq, w.d, w.dtype, 1000 * w.index + 3)
+    ours = _run(q, k, v, g, True, w.softmax_scale)
+    refs = oracle.attention_backward(q, k, v, g, w.softmax_scale, True)
+    _check(ours, refs, w.dtype, what="prefill_mha")

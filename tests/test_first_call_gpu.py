@@ -1,7 +1,8 @@
 """First calls on a device, each in a fresh process: two host threads racing the first
-launches (the per-device kernel set-up runs once, under a lock), and a decode whose first
-call is made under CUDA stream capture (its split workspace comes from the library's
-stream-ordered pool, so the capture holds the allocation and the free)."""
+launches (the per-device kernel set-up runs once, under a lock), and decode and varlen
+calls made under CUDA stream capture after the device's first call (their workspace comes
+from the library's stream-ordered pool, so the capture holds the allocation and the
+free)."""
 import os
 import subprocess
 import sys
@@ -64,13 +65,22 @@ import sys
 sys.path.insert(0, sys.argv[1])
 import torch
 from exact_io_aware_59_b200 import binding
-from exact_io_aware_59_b200.inputs import make_qkv
+from exact_io_aware_59_b200.inputs import make_qkv, randn
 
 torch.cuda.set_device(0)
 shapes = [(4, 8, 5000), (16, 32, 9000)]   # the second needs more workspace than the first
 data = [make_qkv(B, H, 1, N, 128, torch.bfloat16, 31 + B, device="cuda") for B, H, N in shapes]
 outs = [(torch.empty((B, H, 1, 128), device="cuda"), torch.empty((B, H, 1), device="cuda"))
         for B, H, _ in shapes]
+# The device's first call, outside capture (it sets the device up).
+qp, kp, vp = make_qkv(1, 2, 300, 300, 128, torch.bfloat16, 5, device="cuda")
+binding.attention(qp, kp, vp, causal=True)
+# a packed batch for a varlen call under capture
+lens = [300, 5, 700]
+cu = torch.tensor([0, 300, 305, 1005], dtype=torch.int32, device="cuda")
+vq, vk, vv = (randn((1005, 2, 64), 77 + i, torch.float16, device="cuda") for i in range(3))
+vo = torch.empty((1005, 2, 64), device="cuda")
+vl = torch.empty((1005, 2), device="cuda")
 torch.cuda.synchronize()
 s = torch.cuda.Stream()
 graph = torch.cuda.CUDAGraph()
@@ -79,9 +89,14 @@ with torch.cuda.graph(graph, stream=s):
         rc = binding.fa_fwd_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                    l.data_ptr(), B, H, N, 128, 0.088, s.cuda_stream,
                                    binding.FA_BF16, binding.FA_F32, 0)
-        assert rc == binding.FA_OK, rc
+        assert rc == binding.FA_OK, (rc, binding.fa_get_last_cuda_error())
+    rc = binding.fa_fwd_varlen(vq.data_ptr(), vk.data_ptr(), vv.data_ptr(), vo.data_ptr(),
+                               vl.data_ptr(), cu.data_ptr(), cu.data_ptr(), 3, 2, 1005, 1005,
+                               700, 700, 64, 0.125, 1, s.cuda_stream, binding.FA_F16,
+                               binding.FA_F32)
+    assert rc == binding.FA_OK, (rc, binding.fa_get_last_cuda_error())
 for _ in range(2):
-    for o, l in outs:
+    for o, l in outs + [(vo, vl)]:
         o.fill_(float("nan")); l.fill_(float("nan"))
     graph.replay()
     torch.cuda.synchronize()
@@ -89,6 +104,9 @@ for _ in range(2):
         o2, l2 = binding.attention(q, k, v, scale=0.088)
         torch.cuda.synchronize()
         assert torch.equal(o, o2) and torch.equal(l, l2)
+    o2, l2 = binding.varlen_attention(vq, vk, vv, cu, cu, 700, 700, causal=True, scale=0.125)
+    torch.cuda.synchronize()
+    assert torch.equal(vo, o2) and torch.equal(vl, l2)
 del graph
 assert binding.fa_device_status(clear=True) == 0
 binding.fa_release_workspace()
@@ -108,5 +126,5 @@ def test_two_threads_race_the_first_launches():
     _run(_THREADS)
 
 
-def test_first_decode_call_under_stream_capture():
+def test_workspace_calls_under_stream_capture():
     _run(_CAPTURE)

@@ -56,7 +56,7 @@ def test_bench_line_keeps_every_config_in_its_last_1500_characters():
 
     clk = {"sm_mhz": 1965.0, "reasons": ["sw_power_cap"]}
     names = ["mha_d64", "noncausal_8k", "peaky_8k", "causal_16k", "causal_32k", "decode",
-             "decode_paged", "fp8_8k", "bwd_8k", "varlen"]
+             "decode_paged", "fp8_8k", "fp8q_8k", "bwd_8k", "varlen"]
     configs = {n: bench.compact(1234.56789, "TFLOP/s", 0.123456789, 2000, 0.6789012,
                                 0.7890123, clk) for n in names}
     line = {"metric": bench.METRIC, "value": 1.0, "configs": configs}

@@ -96,3 +96,55 @@ def test_fp8_full_size_sampled():
                                            True, rows=rows)
     idx = torch.from_numpy(rows).cuda()
     compare(o.reshape(-1, 128)[idx], lse.reshape(-1)[idx], o_ref, l_ref)
+
+
+@pytest.mark.parametrize("N", [1, 300, 1024])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_quantize_matches_oracle_bitwise(N, dtype):
+    """fa_quantize_e4m3 against the oracle's per-tile quantisation (written from the E4M3
+    format): identical scales and identical codes, byte for byte (both take the scale and
+    the division in fp32 and round to nearest even)."""
+    x = randn((2, 3, N, 128), 1400 + N, dtype, 3.0)
+    x[0, 1, : min(N, 128)] = 0                  # an all-zero tile: scale 1, codes 0
+    if N > 200:
+        x[1, 2, 150] *= 50                      # one tile dominated by a single row
+    codes, scales = binding.quantize_e4m3(x.cuda())
+    torch.cuda.synchronize()
+    c_ref, s_ref = oracle.e4m3_quantize_tiles(x.reshape(6, N, 128))
+    assert np.array_equal(scales.cpu().numpy(), s_ref)
+    assert np.array_equal(codes.cpu().numpy().reshape(6, N, 128), c_ref)
+
+
+def _quant_reference(q, k, v, scale, causal, rows=None):
+    B, H, Nq, d = q.shape
+    Nkv = k.shape[2]
+    q8, qs = oracle.e4m3_quantize_tiles(q.reshape(B * H, Nq, d))
+    k8, ks = oracle.e4m3_quantize_tiles(k.reshape(B * H, Nkv, d))
+    return oracle.fp8_tile_scaled_attention(q8.reshape(B, H, Nq, d), qs, k8.reshape(B, H, Nkv, d),
+                                            ks, v, scale, causal, rows=rows)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_fp8_quant_matches_oracle(causal, dtype):
+    """fa_fwd_fp8_quant (Q and K quantised on the fly, one scale per 128-row tile) against
+    the oracle's quantisation and attention of the dequantised tensors; ragged tiles."""
+    B, H, Nq, Nkv = 2, 3, 300, 333
+    q = randn((B, H, Nq, 128), 1500, dtype, 2.0)
+    k = randn((B, H, Nkv, 128), 1501, dtype)
+    v = randn((B, H, Nkv, 128), 1502, dtype)
+    o, lse = binding.fp8_quant_attention(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    o_ref, l_ref = _quant_reference(q, k, v, 128 ** -0.5, causal)
+    compare(o, lse, o_ref, l_ref)
+
+
+def test_fp8_quant_full_size_every_row():
+    """The benchmark's configuration (B=1, H=32, N=8192, causal, bf16 O), every output."""
+    from exact_io_aware_59_b200.inputs import WORKLOADS, workload_qkv
+    w = WORKLOADS["long_prefill_causal"]
+    q, k, v = workload_qkv(w, device="cuda")
+    o, lse = binding.fp8_quant_attention(q, k, v, causal=True, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    o_ref, l_ref = _quant_reference(q.cpu(), k.cpu(), v.cpu(), w.softmax_scale, True)
+    compare(o, lse, o_ref, l_ref, rel_o=REL_O16[torch.bfloat16])

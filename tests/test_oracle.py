@@ -416,6 +416,90 @@ def test_fp8_attention_is_attention_of_the_dequantised_tensors(oracle_mod):
     np.testing.assert_allclose(l2, lse, rtol=0, atol=1e-12)
 
 
+def _e4m3_nearest_brute(x):
+    """Nearest finite E4M3 value by exhaustive search over the 254 finite codes, ties to
+    the code with the even mantissa; magnitudes beyond 448 saturate."""
+    import oracle
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle.e4m3_to_f64(codes)
+    fin = ~np.isnan(vals)
+    codes, vals = codes[fin], vals[fin]
+    out = np.empty(x.shape, dtype=np.uint8)
+    for i, xi in enumerate(np.asarray(x, dtype=np.float64).ravel()):
+        xi = min(max(xi, -448.0), 448.0)
+        dist = np.abs(vals - xi)
+        best = np.flatnonzero(dist == dist.min())
+        best = best[np.signbit(vals[best]) == np.signbit(xi)]   # -0.0 keeps its sign too
+        even = [b for b in best if codes[b] & 1 == 0]
+        out.ravel()[i] = codes[even[0] if even else best[0]]
+    return out
+
+
+def test_e4m3_encode_is_nearest_even_by_brute_force(oracle_mod):
+    """The encoder against an exhaustive nearest-value search: random values over the whole
+    range (subnormals and saturation included) and every midpoint between neighbours."""
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.uniform(-520, 520, 3000), rng.uniform(-0.02, 0.02, 2000),
+                        rng.normal(0, 3, 2000)]).astype(np.float32)
+    vals = np.unique(oracle_mod.e4m3_to_f64(np.arange(0, 127, dtype=np.uint8)))
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)   # exact in fp32
+    x = np.concatenate([x, mids, -mids, [0.0, -0.0, 448.0, -448.0, 464.0, 1e6]]).astype(np.float32)
+    assert np.array_equal(oracle_mod.e4m3_encode(x), _e4m3_nearest_brute(x))
+
+
+def test_e4m3_encode_matches_torch_in_range(oracle_mod):
+    """Within the finite range the encoder equals torch's float8_e4m3fn conversion (a library
+    routine, round to nearest even), and every finite code round-trips."""
+    x = randn((200000,), 905, torch.float32, 40.0).clamp(-448, 448)
+    ours = oracle_mod.e4m3_encode(x.numpy())
+    ref = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle_mod.e4m3_to_f64(codes)
+    fin = ~np.isnan(vals)
+    assert np.array_equal(oracle_mod.e4m3_encode(vals[fin].astype(np.float32)), codes[fin])
+
+
+def test_e4m3_quantize_tiles_scale_and_error(oracle_mod):
+    """Per-tile quantisation: every tile's largest magnitude maps to 448 exactly, an all-zero
+    tile keeps scale 1 and codes 0, and decode(code) * scale is within half a spacing of x."""
+    x = randn((3, 300, 16), 906, torch.bfloat16).float()
+    x[1, 128:256] = 0.0
+    codes, scales = oracle_mod.e4m3_quantize_tiles(x)
+    assert scales.shape == (3, 3) and scales.dtype == np.float32
+    dec = oracle_mod.e4m3_to_f64(codes)
+    for b in range(3):
+        for t in range(3):
+            blk = dec[b, t * 128:(t + 1) * 128]
+            if b == 1 and t == 1:
+                assert scales[b, t] == 1.0 and (codes[b, 128:256] == 0).all()
+                continue
+            assert np.abs(blk).max() == 448.0
+            xs = x[b, t * 128:(t + 1) * 128].numpy().astype(np.float64)
+            rel = np.abs(blk * scales[b, t] - xs) / np.maximum(np.abs(xs), 2.0 ** -6 * scales[b, t])
+            assert rel.max() <= 2.0 ** -4 + 1e-6   # half of the 3-bit mantissa spacing
+
+
+def test_fp8_tile_scaled_attention_is_attention_of_the_dequantised_tensors(oracle_mod):
+    B, H, N, d = 1, 2, 300, 32
+    q = randn((B, H, N, d), 907, torch.bfloat16)
+    k = randn((B, H, N, d), 908, torch.bfloat16)
+    v = randn((B, H, N, d), 909, torch.bfloat16)
+    q8, qs = oracle_mod.e4m3_quantize_tiles(q.reshape(B * H, N, d))
+    k8, ks = oracle_mod.e4m3_quantize_tiles(k.reshape(B * H, N, d))
+    q8, k8 = q8.reshape(B, H, N, d), k8.reshape(B, H, N, d)
+    o, lse = oracle_mod.fp8_tile_scaled_attention(q8, qs, k8, ks, v, 0.2, True)
+    qd = oracle_mod.e4m3_to_f64(q8) * np.repeat(qs, 128, axis=1)[:, :N].reshape(B, H, N, 1)
+    kd = oracle_mod.e4m3_to_f64(k8) * np.repeat(ks, 128, axis=1)[:, :N].reshape(B, H, N, 1)
+    o_ref, l_ref = oracle_mod.attention(torch.from_numpy(qd), torch.from_numpy(kd),
+                                        v.to(torch.float64), 0.2, True)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(lse, l_ref)
+    # and it is close to the unquantised attention (E4M3 keeps 3 mantissa bits)
+    o16, _ = oracle_mod.attention(q, k, v, 0.2, True)
+    assert np.abs(o - o16).max() < 0.1
+
+
 # ---------------------------------------------------------------- backward pass
 def _bwd_inputs(B, H, Nq, Nkv, d, seed, dtype=torch.float64):
     q, k, v = make_qkv(B, H, Nq, Nkv, d, torch.float32, seed)

@@ -140,15 +140,19 @@ def test_decode_small_full_compare():
     compare(o, lse, o_ref, l_ref)
 
 
-@pytest.mark.parametrize("growth", [12.0, 20.0, -20.0])
+@pytest.mark.parametrize("growth", [12.0, 20.0, 26.0, 40.0, -20.0])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)])
 def test_running_max_growing_along_keys(growth, causal, d, dtype):
     """Scores that rise (or fall) by `growth` log2 units per 128-key tile, plus noise.
-    Rising by 20 moves every row's reference max on every tile (rescale of O, and the
-    early exponentiation against the old max is redone); rising by 12 makes the reference
-    max lag the true one without moving it, so p reaches ~2^12 (close to the fp16 limit
-    for the lag); falling leaves the first tile's max in charge."""
+    The kernel hands each tile's P out in two halves of 64 keys, the first as soon as it is
+    known not to move the reference max.  Rising by 20 or 26 per tile, the first half
+    stays within the lazy threshold (15) of the previous tile's max and goes out, and the
+    second half moves it: O is rescaled after the first half's product and the second half
+    is redone.  Rising by 40, the first half already moves it (the whole tile is redone in
+    two passes, O rescaled before any of it goes out).  Rising by 12, the reference max
+    lags the true one without moving for a tile, so p reaches ~2^12 (close to the fp16
+    limit for the lag); falling leaves the first tile's max in charge."""
     B, H, N = 1, 2, 1000
     scale = scale_for(d)
     g = growth / (128 * scale * math.log2(math.e))
