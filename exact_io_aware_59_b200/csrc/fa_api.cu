@@ -300,14 +300,18 @@ int run_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   p.H = H;
   p.total_q = total_q;
   p.total_k = total_k;
-  // Call-local workspace for the plan: item count (16 bytes), B sequence records, items.
+  // Call-local workspace for the plan: item count (16 bytes), B sequence records, B first
+  // positions, items.
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* ws = nullptr;
-  const size_t ws_bytes = 16 + static_cast<size_t>(B) * sizeof(int4) + static_cast<size_t>(items) * 4;
+  const size_t seq_b = static_cast<size_t>(B) * sizeof(int4), first_b = static_cast<size_t>(B) * 4;
+  const size_t ws_bytes = 16 + seq_b + first_b + static_cast<size_t>(items) * 4;
   if ((rc = workspace_alloc(ds, ws_bytes, st, &ws)) != FA_OK) return rc;
-  p.vl_count = static_cast<int*>(ws);
-  p.vl_seqs = reinterpret_cast<int4*>(static_cast<char*>(ws) + 16);
-  p.vl_items = reinterpret_cast<int*>(static_cast<char*>(ws) + 16 + static_cast<size_t>(B) * sizeof(int4));
+  char* w = static_cast<char*>(ws);
+  p.vl_count = reinterpret_cast<int*>(w);
+  p.vl_seqs = reinterpret_cast<int4*>(w + 16);
+  p.vl_first = reinterpret_cast<int*>(w + 16 + seq_b);
+  p.vl_items = reinterpret_cast<int*>(w + 16 + seq_b + first_b);
   long long grid = ds->sm_count;
   if (grid > units) grid = units;
   if (grid < 1) grid = 1;

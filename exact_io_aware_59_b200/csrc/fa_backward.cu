@@ -79,8 +79,8 @@ struct BwdCfg {
   static constexpr int kQOff = kVOff + kTileBytes;          // Q stages
   static constexpr int kdOOff = kQOff + kStages * kTileBytes;  // dO (one buffer)
   static constexpr int kdSOff = kdOOff + kTileBytes;        // dS, 128 keys x 128 queries,
-                                                            // two 64-query blocks
-  static constexpr int kLseOff = kdSOff + kTileBytes;       // -LSE*log2e per stage
+  static constexpr int kdSBytes = kBK * kBQ * 2;            // two 64-query blocks (any d)
+  static constexpr int kLseOff = kdSOff + kdSBytes;         // -LSE*log2e per stage
   static constexpr int kDelOff = kLseOff + kStages * kBQ * 4;  // D per stage
   static constexpr int kBarOff = kDelOff + kStages * kBQ * 4;
   // mbarriers
@@ -252,6 +252,14 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
       mma_ts(tmem + kTdV, tmem + kTS + a16_col(kk), do_mn() + ((kk * 2048) >> 4), idesc_kv,
              (i > 0 || kk > 0) ? 1u : 0u);
     tc_commit(bar_addr(bars, C::kBarDOFree));
+    // S(i+1) over S right away (P^T(i) there has been read by dV(i), issued above), so the
+    // softmax can compute P^T(i+1) while dK(i), dQ(i) and dP(i+1) run.
+    if (i + 1 < n) {
+      if (!(ok = wait(C::kBarQFull + st1, ((i + 1) / kStages) & 1))) break;
+      tc_fence_after();
+      issue_st(kTS, k_desc(), q_kmaj(st1));
+      tc_commit(bar_addr(bars, C::kBarSFull));
+    }
     // dS^T(i) is stored over dP and dS(i) in shared memory: dK(i).
     if (!(ok = wait(C::kBarDSReady, i & 1))) break;
     tc_fence_after();
@@ -259,13 +267,6 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
     for (int kk = 0; kk < kBQ / 16; ++kk)
       mma_ts(tmem + kTdK, tmem + kTdP + a16_col(kk), q_mn(st) + ((kk * 2048) >> 4), idesc_kv,
              (i > 0 || kk > 0) ? 1u : 0u);
-    // S(i+1) over S: P^T(i) there has been read by dV(i), issued above.
-    if (i + 1 < n) {
-      if (!(ok = wait(C::kBarQFull + st1, ((i + 1) / kStages) & 1))) break;
-      tc_fence_after();
-      issue_st(kTS, k_desc(), q_kmaj(st1));
-      tc_commit(bar_addr(bars, C::kBarSFull));
-    }
     // dQ^T(i) over dP: dS^T(i) there has been read by dK(i), issued above.
 #pragma unroll
     for (int kk = 0; kk < kBK / 16; ++kk)
@@ -453,31 +454,27 @@ __device__ void dq_drain(const BwdParams& p, int bh, int i0, int n, uint32_t bar
       if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarDQEmpty));
       continue;
     }
+    // The whole row of dQ^T into registers first, so the columns are free for dP(i+1) before
+    // any reduction is issued.
+    uint32_t a[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tq + 32 * c, a[c]);
+    tmem_ld_wait_only();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) reg_fence(a[c]);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarDQEmpty));  // dP(i+1) may overwrite it
     // Accumulator row q (query q0 + q) is D contiguous floats: a warp adds 32 consecutive
     // ones per instruction.
-    float* acc = p.dq_acc + (static_cast<size_t>(bh) * p.nq_pad + static_cast<size_t>(i0 + i) * kBQ) * D + t;
+    float* row = p.dq_acc + (static_cast<size_t>(bh) * p.nq_pad + static_cast<size_t>(i0 + i) * kBQ) * D + t;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {  // queries 64h .. 64h+63
-      uint32_t a[2][32];
-      tmem_ld_32x32b_x32(tq + 64 * h, a[0]);
-      tmem_ld_32x32b_x32(tq + 64 * h + 32, a[1]);
-      tmem_ld_wait_only();
-      reg_fence(a[0]);
-      reg_fence(a[1]);
-      if (h == 1) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarDQEmpty));  // dP(i+1) may overwrite it
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        red_add_f32(row, __uint_as_float(a[c][q]));
+        row += D;
       }
-      float* row = acc + static_cast<size_t>(64 * h) * D;
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          red_add_f32(row, __uint_as_float(a[c][q]));
-          row += D;
-        }
-    }
   }
 }
 

@@ -419,36 +419,6 @@ __device__ __forceinline__ float min3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of x < 127 on the FMA pipe, to take load off the SFU.  Round-to-nearest
-// argument reduction x = j + f, |f| <= 1/2, with the 1.5 * 2^23 addition trick (the sum's
-// low mantissa bits hold j); 2^f from a degree-4 polynomial whose coefficients minimise the
-// maximum relative error on [-1/2, 1/2] (computed by linear programming over a dense grid,
-// see exp2_poly.py; max relative error 2.7e-6 in fp32, far below the 2^-9 of the bf16
-// rounding that follows); j is added to the exponent field with an integer multiply-add.
-// x is clamped at -125 so the result stays a normal number.
-constexpr float kExp2C0 = 0.9999992251396179f;
-constexpr float kExp2C1 = 0.6931217312812805f;
-constexpr float kExp2C2 = 0.24024765193462372f;
-constexpr float kExp2C3 = 0.05591819807887077f;
-constexpr float kExp2C4 = 0.009569705463945866f;
-__device__ __forceinline__ uint64_t exp2_poly_pair(float x0, float x1) {
-  const float kMagic = 12582912.0f;  // 1.5 * 2^23
-  const uint64_t xc = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
-  const uint64_t j = f2_add(t, f2_pack(-kMagic, -kMagic));
-  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), xc);
-  uint64_t p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
-  p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  const uint32_t r0 = __float_as_uint(t0) * (1u << 23) + __float_as_uint(p0);
-  const uint32_t r1 = __float_as_uint(t1) * (1u << 23) + __float_as_uint(p1);
-  return f2_pack(__uint_as_float(r0), __uint_as_float(r1));
-}
-
 // Two fp32 values rounded to nearest-even into one packed 16-bit pair, `lo` in the low
 // half.
 template <bool BF16>

@@ -27,11 +27,12 @@ struct PrefillParams {
   int total_q, total_k;
   // The packed batch's work list, built on the device by the plan kernel that runs before
   // the prefill kernel (call-local workspace): the number of (sequence, Q-tile pair) items
-  // that hold query rows, each sequence's (q0, Lq, k0, Lk) after the bounds checks, and the
-  // items heaviest first, each as b * n_pairs + pair.  Work unit u is head u % H of item
-  // u / H.
+  // that hold query rows, each sequence's (q0, Lq, k0, Lk) after the bounds checks and the
+  // position of its first item, and the items, each as b * n_pairs + pair.  Work unit u is
+  // head u % H of item u / H.
   const int* vl_count;
   const int4* vl_seqs;
+  const int* vl_first;
   const int* vl_items;
   // E4M3 queries and keys with one scale per 128-row tile (null: per-tensor scales folded
   // into scale_log2): [BH, n_qtiles] and [BH, n_kvtiles].

@@ -37,11 +37,6 @@ constexpr int kRegsLaunch = 168;   // 65536 / 384, rounded down to a multiple of
 constexpr int kRegsSide = 88;      // warpgroup 0 (load + MMA issue)
 constexpr int kRegsSoftmax = 208;  // warpgroups 1 and 2; 128*88 + 256*208 == 384*168
 static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
-// One score pair in kFmaExp2Every takes 2^x on the FMA pipe (exp2_poly_pair) instead of the
-// SFU; 0 sends every score to the SFU.  Timed back to back at the boosted clock, one pair in
-// four and none ran equally fast; timed for seconds under the 1 kW power cap, where the
-// polynomial's extra instructions cost clock, the SFU alone was 2.8% faster.
-constexpr int kFmaExp2Every = 0;
 // Lazy rescale threshold in log2 units: the reference max m_used of a row moves only when
 // a tile's max exceeds it by more than this, so p = 2^(x - m_used) <= 2^15, below the fp16
 // maximum 65504 (bf16 and the fp32 O and l have far more range).  O and l share m_used,
@@ -388,11 +383,9 @@ __device__ __forceinline__ float row_reduce(const uint32_t (&s)[4][32]) {
 }
 
 // p = 2^(s * scale_log2 - m) for 32 scores (tile columns col0 .. col0+31), rounded in
-// pairs to the 16-bit type into pk (exp_pack_store32 also stores them to 16 TMEM columns
-// at tP, two values per column); adds the unrounded p to the running sums, and with XMAX
-// folds the exponents x = s * scale_log2 - m into two running maxima.  FULL: every column
-// visible (and, with kFmaExp2Every > 0, one pair in kFmaExp2Every takes the FMA-pipe
-// exp2).  !FULL: columns past lim_c get p = 0.
+// pairs to the 16-bit type into pk; adds the unrounded p to the running sums, and with
+// XMAX folds the exponents x = s * scale_log2 - m into two running maxima.  FULL: every
+// column visible.  !FULL: columns past lim_c get p = 0.  Every 2^x goes to the SFU.
 template <bool BF16, bool FULL, bool XMAX = false>
 __device__ __forceinline__ void exp_pack32(const uint32_t (&s)[32], uint64_t sc2, uint64_t nm2,
                                            int col0, int lim_c, uint32_t (&pk)[16],
@@ -403,12 +396,8 @@ __device__ __forceinline__ void exp_pack32(const uint32_t (&s)[32], uint64_t sc2
     float x0, x1, p0, p1;
     f2_unpack(x2, x0, x1);
     if (XMAX) xmax[i & 1] = max3(xmax[i & 1], x0, x1);
-    if (FULL && kFmaExp2Every > 0 && (i % (kFmaExp2Every > 0 ? kFmaExp2Every : 1)) == 1) {
-      f2_unpack(exp2_poly_pair(x0, x1), p0, p1);
-    } else {
-      p0 = ex2(x0);
-      p1 = ex2(x1);
-    }
+    p0 = ex2(x0);
+    p1 = ex2(x1);
     if (!FULL) {
       p0 = (col0 + 2 * i <= lim_c) ? p0 : 0.f;
       p1 = (col0 + 2 * i + 1 <= lim_c) ? p1 : 0.f;
@@ -749,21 +738,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Builds the work list of a packed batch before the prefill kernel runs (one CTA): every
 // sequence's token ranges are bounds-checked once (a range outside [0, total] or longer
 // than the declared maximum is clamped and reported in the status word), and every
-// (sequence, Q-tile pair) that holds query rows becomes one item, listed heaviest first by
-// its K/V tile count (a counting sort; the order within one weight is whatever the
-// atomics give, which changes no result: a unit's rows do not depend on where it runs).
-// The persistent kernel then deals out items x heads in its snake order, with no empty
-// units and no per-unit read of the offsets.
+// (sequence, Q-tile pair) that holds query rows becomes one item.  Items are listed
+// sequence by sequence, sequences with more Q-tile pairs first (a counting sort on that
+// count; the order among sequences of one count is whatever the atomics give, which
+// changes no result: a unit's rows do not depend on where it runs), and each sequence's
+// pairs last-first (for a causal batch, its heaviest first).  The persistent kernel deals
+// items x heads out in its snake order, so the CTAs running at one time work on a few
+// Q-tile pairs of every head of one sequence and share that sequence's K and V in L2 (a
+// list sorted by item weight alone spread them over many sequences and read K and V from
+// HBM about six times over); the list is still heavy-first overall.
 constexpr int kPlanThreads = 1024;
-constexpr int kPlanBuckets = 2 * kPlanThreads;  // weights above kPlanBuckets - 1 share a bucket
+constexpr int kPlanBuckets = 2 * kPlanThreads;  // counts above kPlanBuckets - 1 share a bucket
 
 __global__ void __launch_bounds__(kPlanThreads)
     fa_varlen_plan(const PrefillParams p, int B, int* __restrict__ count, int4* __restrict__ seqs,
-                   int* __restrict__ items, int* __restrict__ status) {
+                   int* __restrict__ first, int* __restrict__ items, int* __restrict__ status) {
   __shared__ int bucket[kPlanBuckets];
   __shared__ int warp_total[kPlanThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   bool bad = false;
+  for (int i = tid; i < kPlanBuckets; i += kPlanThreads) bucket[i] = 0;
+  __syncthreads();
+  // Clamped ranges; each sequence's pair count, summed per bucket (heaviest first).
   for (int b = tid; b < B; b += kPlanThreads) {
     int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
     if (q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
@@ -775,34 +771,12 @@ __global__ void __launch_bounds__(kPlanThreads)
       k1 = min(max(k1, k0), min(p.total_k, k0 + p.Nkv));
     }
     seqs[b] = make_int4(q0, q1 - q0, k0, k1 - k0);
+    const int np = ((q1 - q0 + BM - 1) / BM + 1) / 2;  // Q-tile pairs holding query rows
+    if (np > 0) atomicAdd(&bucket[kPlanBuckets - 1 - min(np, kPlanBuckets - 1)], np);
   }
   if (bad) atomicOr(status, kStatusBadInput);
-  for (int i = tid; i < kPlanBuckets; i += kPlanThreads) bucket[i] = 0;
-  __syncthreads();  // also makes the seqs writes visible to the whole CTA
-  const long long n_items = static_cast<long long>(B) * p.n_pairs;
-  // Bucket of item i (heaviest first), or -1 when its Q tiles hold no query row.
-  auto bucket_of = [&](long long i) {
-    const int b = static_cast<int>(i / p.n_pairs);
-    const int pr = static_cast<int>(i - static_cast<long long>(b) * p.n_pairs);
-    const int4 sq = seqs[b];
-    Unit x;
-    x.bh = 0;
-    x.h = 0;
-    x.pair = pr;
-    x.q0 = sq.x;
-    x.Lq = sq.y;
-    x.k0 = sq.z;
-    x.Lk = sq.w;
-    if (2 * pr * BM >= x.Lq) return -1;
-    const int w = kv_tiles_for(p, x, 2 * pr) + kv_tiles_for(p, x, 2 * pr + 1);
-    return kPlanBuckets - 1 - min(w, kPlanBuckets - 1);
-  };
-  for (long long i = tid; i < n_items; i += kPlanThreads) {
-    const int bk = bucket_of(i);
-    if (bk >= 0) atomicAdd(&bucket[bk], 1);
-  }
   __syncthreads();
-  // Exclusive prefix sum of the bucket counts: thread t owns buckets 2t and 2t+1.
+  // Exclusive prefix sum of the per-bucket item counts: thread t owns buckets 2t and 2t+1.
   const int c0 = bucket[2 * tid], c1 = bucket[2 * tid + 1];
   int incl = c0 + c1;
 #pragma unroll
@@ -827,9 +801,18 @@ __global__ void __launch_bounds__(kPlanThreads)
   bucket[2 * tid + 1] = excl + c0;
   if (tid == kPlanThreads - 1) *count = excl + c0 + c1;
   __syncthreads();
+  // Each sequence takes a contiguous range of the list.
+  for (int b = tid; b < B; b += kPlanThreads) {
+    const int np = ((seqs[b].y + BM - 1) / BM + 1) / 2;
+    first[b] = np > 0 ? atomicAdd(&bucket[kPlanBuckets - 1 - min(np, kPlanBuckets - 1)], np) : 0;
+  }
+  __syncthreads();
+  const long long n_items = static_cast<long long>(B) * p.n_pairs;
   for (long long i = tid; i < n_items; i += kPlanThreads) {
-    const int bk = bucket_of(i);
-    if (bk >= 0) items[atomicAdd(&bucket[bk], 1)] = static_cast<int>(i);
+    const int b = static_cast<int>(i / p.n_pairs);
+    const int pr = static_cast<int>(i - static_cast<long long>(b) * p.n_pairs);
+    const int np = ((seqs[b].y + BM - 1) / BM + 1) / 2;
+    if (pr < np) items[first[b] + (np - 1 - pr)] = static_cast<int>(i);  // last pair first
   }
 }
 
@@ -865,6 +848,7 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
     // Packed batch: the plan kernel writes the work list the prefill kernel reads.
     fa_varlen_plan<<<1, kPlanThreads, 0, stream>>>(p, p.BH / p.H, const_cast<int*>(p.vl_count),
                                                    const_cast<int4*>(p.vl_seqs),
+                                                   const_cast<int*>(p.vl_first),
                                                    const_cast<int*>(p.vl_items), status);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
