@@ -194,6 +194,9 @@ def whole_job_rate(units_per_rank: float, ms_max: float, ws: int) -> float:
 
 def time_steps(fn, steps: int, warmup: int, ws: int, stream) -> float:
     """Milliseconds per step over `steps` calls, CUDA events on the launch stream."""
+    # The inputs were made on torch's default stream; the launch stream does not wait for
+    # it by itself.
+    torch.cuda.synchronize()
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()

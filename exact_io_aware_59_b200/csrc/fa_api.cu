@@ -635,6 +635,8 @@ int fa_fwd_fp8_quant(const void* q, const void* k, const void* v, void* o, float
   if ((rc = get_encoder()) != FA_OK) return rc;
   const size_t BH = static_cast<size_t>(B) * H;
   const int nqt = (Nq + 127) / 128, nkt = (Nkv + 127) / 128;
+  const long long units = static_cast<long long>(BH) * ((nqt + 1) / 2);
+  if (units > 0x7fffffffLL || static_cast<long long>(BH) * nkt > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
   auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
   // Call-local workspace: Q codes, K codes, Q tile scales, K tile scales.
   const size_t qb = up256(BH * Nq * d), kb = up256(BH * Nkv * d);
@@ -668,7 +670,6 @@ int fa_fwd_fp8_quant(const void* q, const void* k, const void* v, void* o, float
     p.n_qtiles = nqt;
     p.n_pairs = (nqt + 1) / 2;
     p.n_kvtiles = nkt;
-    const long long units = static_cast<long long>(BH) * p.n_pairs;
     p.n_units = static_cast<int>(units);
     p.scale_log2 = scale_log2(scale);
     p.H = H;
