@@ -40,6 +40,9 @@ _VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 _SIGNATURES = {
     "fa_fwd": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I],
     "fa_fwd_prefill": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I, _I],
+    "fa_fwd_prefill_split": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _I, _I, _I,
+                             _I],
+    "fa_prefill_num_splits": [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I)],
     "fa_fwd_decode": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
     "fa_fwd_decode_noalloc": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP, _I, _I, _I],
     "fa_fwd_fp8": [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP, _F, _F, _I, _I],
@@ -103,6 +106,22 @@ def fa_fwd_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_
                    o_dtype, num_ctas) -> int:
     return library().fa_fwd_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream,
                                     in_dtype, o_dtype, num_ctas)
+
+
+def fa_fwd_prefill_split(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype,
+                         o_dtype, num_ctas, num_splits) -> int:
+    return library().fa_fwd_prefill_split(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal,
+                                          stream, in_dtype, o_dtype, num_ctas, num_splits)
+
+
+def prefill_num_splits(B, H, Nq, Nkv, d, causal, sm_count=0) -> int:
+    """The K/V part count the prefill path chooses for this shape (fa_prefill_num_splits)."""
+    out = ctypes.c_int(0)
+    rc = library().fa_prefill_num_splits(B, H, Nq, Nkv, d, int(bool(causal)), sm_count,
+                                         ctypes.byref(out))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_prefill_num_splits")
+    return out.value
 
 
 def fa_fwd_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype,
@@ -255,6 +274,9 @@ def attention(q, k, v, causal: bool = False, scale: Optional[float] = None,
     """O, LSE = softmax(scale * Q K^T [+ causal]) V for contiguous CUDA tensors
     q [B,H,Nq,d], k/v [B,H,Nkv,d] (fp16 or bf16).  out_dtype: torch.float32 (default) or
     the input dtype.  path: "auto" (decode when Nq == 1), "prefill" or "decode".
+    num_ctas: the prefill's persistent grid (0: one CTA per SM).  num_splits: decode, the
+    split CTAs (0: one per SM); prefill, the K/V parts of each Q-tile pair (0: chosen by
+    the library, which splits only small problems and never under an explicit num_ctas).
     Enqueues on `stream` (default: torch's current stream) and returns (o, lse)."""
     import torch
 
@@ -283,10 +305,14 @@ def attention(q, k, v, causal: bool = False, scale: Optional[float] = None,
                 raise ValueError("the decode path takes exactly one query per head")
             rc = fa_fwd_decode(*args, B, H, Nkv, d, scale, s.cuda_stream, ic, oc, num_splits)
             where = "fa_fwd_decode"
-        elif path in ("prefill", "auto"):
+        elif path in ("prefill", "auto") and num_splits == 0:
             rc = fa_fwd_prefill(*args, B, H, Nq, Nkv, d, scale, int(bool(causal)), s.cuda_stream,
                                 ic, oc, num_ctas)
             where = "fa_fwd_prefill"
+        elif path in ("prefill", "auto"):
+            rc = fa_fwd_prefill_split(*args, B, H, Nq, Nkv, d, scale, int(bool(causal)),
+                                      s.cuda_stream, ic, oc, num_ctas, num_splits)
+            where = "fa_fwd_prefill_split"
         else:
             raise ValueError(f"unknown path {path!r}")
     if rc != FA_OK:

@@ -2,6 +2,7 @@
 // TMA descriptors and kernel launches.  Host code only.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -231,9 +232,91 @@ size_t decode_ws_bytes(const fa::DecodeParams& p, int d) {
   return recs * (d + 1) * sizeof(float);
 }
 
+// K/V parts per (head, Q-tile pair) for a prefill with fewer work units than SMs, chosen
+// with a run-time model fitted to B200 timings of 14 shapes (d 64 and 128, causal and not,
+// 1 to 32 heads, 2k to 16k tokens; predicted within about 5%):
+//   time(S) = steps of the busiest CTA, each unit adding kUnitSteps (its Q load and its
+//             pipeline's fill and drain), units dealt heaviest first in the snake order
+//             the kernel uses, times the step time (K/V tile of 128 keys for both Q tiles:
+//             about 1.8 us at d = 128, 1.62 us at d = 64)
+//           + for S > 1, the partial records and the combine launch: 8 us + 0.4 ns per
+//             partial element (S * B*H*Nq * d).
+// A split is taken only when the model predicts at least 10% less time than no split.
+constexpr int kMaxSplits = 8;
+constexpr double kUnitSteps = 3.75;
+
+// Host copy of the kernel's K/V tile count for Q tile `qtile` ([B,H,N,d] layout).
+int host_kv_tiles(const fa::PrefillParams& p, int qtile) {
+  if (qtile * 128 >= p.Nq) return 0;
+  const int ntk = p.n_kvtiles;
+  if (!p.causal) return ntk;
+  const int last_key = std::min(qtile * 128 + 127, p.Nq - 1) + p.Nkv - p.Nq;
+  return last_key < 0 ? 0 : std::min(ntk, last_key / 128 + 1);
+}
+
+// nmax[pair]: the K/V tiles of each Q-tile pair (its heavier tile's).
+double predicted_us(const fa::PrefillParams& p, const int* nmax, int S, int sm_count, int d) {
+  const long long units = static_cast<long long>(p.BH) * p.n_pairs * S;
+  const int G = static_cast<int>(std::min<long long>(sm_count, units));
+  double load[1024] = {0.0};
+  long long u = 0;
+  for (int pair = p.n_pairs - 1; pair >= 0; --pair) {
+    for (int split = 0; split < S; ++split) {
+      const int steps = (split + 1) * nmax[pair] / S - split * nmax[pair] / S;
+      const double cost = steps > 0 ? steps + kUnitSteps : 0.3;
+      for (int bh = 0; bh < p.BH; ++bh, ++u) {
+        const long long r = u / G, c = u - r * G;
+        load[(r & 1) ? G - 1 - c : c] += cost;
+      }
+    }
+  }
+  double worst = 0.0;
+  for (int c = 0; c < G; ++c) worst = std::max(worst, load[c]);
+  double t = worst * (d == 128 ? 1.8 : 1.62);
+  if (S > 1) t += 8.0 + 4e-7 * S * static_cast<double>(p.BH) * p.Nq * d;
+  return t;
+}
+
+int auto_splits_uncached(const fa::PrefillParams& p, int sm_count, int d) {
+  int nmax[1024];
+  for (int pair = 0; pair < p.n_pairs; ++pair)
+    nmax[pair] = std::max(host_kv_tiles(p, 2 * pair), host_kv_tiles(p, 2 * pair + 1));
+  const double t1 = predicted_us(p, nmax, 1, sm_count, d);
+  int best = 1;
+  double t_best = t1;
+  for (int S = 2; S <= std::min(kMaxSplits, p.n_kvtiles); ++S) {
+    const double t = predicted_us(p, nmax, S, sm_count, d);
+    if (t < t_best) {
+      t_best = t;
+      best = S;
+    }
+  }
+  return t_best < 0.9 * t1 ? best : 1;
+}
+
+// The choice for the last few shapes this thread asked about (the model's loop costs a few
+// microseconds; a program repeats its shapes).
+int auto_splits(const fa::PrefillParams& p, int sm_count, int d) {
+  const long long units = static_cast<long long>(p.BH) * p.n_pairs;
+  if (units >= sm_count || sm_count > 1024) return 1;  // then also n_pairs < 1024
+  struct Entry {
+    int BH, Nq, Nkv, causal, d, sm_count, S;
+  };
+  thread_local Entry cache[8] = {};
+  thread_local int next = 0;
+  for (const Entry& e : cache)
+    if (e.S > 0 && e.BH == p.BH && e.Nq == p.Nq && e.Nkv == p.Nkv && e.causal == p.causal &&
+        e.d == d && e.sm_count == sm_count)
+      return e.S;
+  const int S = auto_splits_uncached(p, sm_count, d);
+  cache[next] = Entry{p.BH, p.Nq, p.Nkv, p.causal, d, sm_count, S};
+  next = (next + 1) % 8;
+  return S;
+}
+
 int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                 int Nq, int Nkv, int d, float scale, int causal, void* stream, int in_dtype,
-                int o_dtype, int num_ctas) {
+                int o_dtype, int num_ctas, int num_splits) {
   DeviceState* ds = nullptr;
   int rc = device_state(&ds);
   if (rc != FA_OK) return rc;
@@ -259,12 +342,35 @@ int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse
   p.cu_q = p.cu_k = nullptr;
   p.H = H;
   p.scale_log2 = scale_log2(scale);
+  const int S = num_splits > 0 ? std::min(num_splits, p.n_kvtiles) : auto_splits(p, ds->sm_count, d);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* ws = nullptr;
+  float *part_o = nullptr, *part_lse = nullptr;
+  if (S > 1) {
+    // Split partials: fp32 O / l [S, BH*Nq, d] then the natural LSE [S, BH*Nq].
+    const long long split_units = units * S;
+    if (split_units > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+    const size_t rows = static_cast<size_t>(BH) * Nq;
+    const size_t ob = static_cast<size_t>(S) * rows * d * sizeof(float);
+    if ((rc = workspace_alloc(ds, ob + static_cast<size_t>(S) * rows * sizeof(float), st, &ws)) != FA_OK)
+      return rc;
+    p.n_splits = S;
+    part_o = static_cast<float*>(ws);
+    part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + ob);
+    p.n_units = static_cast<int>(split_units);
+  } else {
+    p.n_splits = 1;
+  }
   long long grid = num_ctas > 0 ? num_ctas : ds->sm_count;
-  if (grid > units) grid = units;
+  if (grid > p.n_units) grid = p.n_units;
   if (grid < 1) grid = 1;
   cudaError_t e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, bf16, o_dtype == FA_F32,
-                                     static_cast<int>(grid), ds->status,
-                                     static_cast<cudaStream_t>(stream));
+                                     static_cast<int>(grid), ds->status, st, false, part_o,
+                                     part_lse);
+  if (ws != nullptr) {
+    const cudaError_t ef = cudaFreeAsync(ws, st);
+    if (e == cudaSuccess) e = ef;
+  }
   return e == cudaSuccess ? FA_OK : cuda_fail(e);
 }
 
@@ -458,7 +564,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   int rc = check_args(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, in_dtype, o_dtype);
   if (rc != FA_OK) return rc;
   if (Nq == 1) return run_decode(q, k, v, o, lse, B, H, Nkv, d, scale, stream, in_dtype, o_dtype, 0);
-  return run_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype, o_dtype, 0);
+  return run_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype, o_dtype, 0,
+                     0);
 }
 
 int fa_fwd_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -467,8 +574,44 @@ int fa_fwd_prefill(const void* q, const void* k, const void* v, void* o, float* 
   int rc = check_args(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, in_dtype, o_dtype);
   if (rc != FA_OK) return rc;
   if (num_ctas < 0) return FA_ERR_INVALID_ARG;
+  // An explicit grid runs the unsplit units; the automatic one may split them.
   return run_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype, o_dtype,
-                     num_ctas);
+                     num_ctas, num_ctas > 0 ? 1 : 0);
+}
+
+int fa_prefill_num_splits(int B, int H, int Nq, int Nkv, int d, int causal, int sm_count,
+                          int* num_splits) {
+  if (!num_splits || B < 1 || H < 1 || Nq < 1 || Nkv < 1 || (d != 64 && d != 128) ||
+      (causal != 0 && causal != 1) || sm_count < 0)
+    return FA_ERR_INVALID_ARG;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (sm_count == 0) {
+    DeviceState* ds = nullptr;
+    const int rc = device_state(&ds);
+    if (rc != FA_OK) return rc;
+    sm_count = ds->sm_count;
+  }
+  fa::PrefillParams p{};
+  p.BH = static_cast<int>(BH);
+  p.Nq = Nq;
+  p.Nkv = Nkv;
+  p.causal = causal;
+  p.n_qtiles = (Nq + 127) / 128;
+  p.n_pairs = (p.n_qtiles + 1) / 2;
+  p.n_kvtiles = (Nkv + 127) / 128;
+  *num_splits = auto_splits(p, sm_count, d);
+  return FA_OK;
+}
+
+int fa_fwd_prefill_split(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
+                         int in_dtype, int o_dtype, int num_ctas, int num_splits) {
+  int rc = check_args(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, in_dtype, o_dtype);
+  if (rc != FA_OK) return rc;
+  if (num_ctas < 0 || num_splits < 0 || num_splits > 64) return FA_ERR_INVALID_ARG;
+  return run_prefill(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, stream, in_dtype, o_dtype,
+                     num_ctas, num_splits);
 }
 
 int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B,

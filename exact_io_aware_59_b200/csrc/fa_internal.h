@@ -25,6 +25,12 @@ struct PrefillParams {
   const int* cu_k;
   int H;            // heads per sequence (bh = b * H + h)
   int total_q, total_k;
+  // K/V split of problems with fewer units than SMs (> 1; else no split): each (b*h,
+  // Q-tile pair) becomes n_splits units over consecutive parts of its K/V tile range.  A
+  // unit writes its rows' partial output (divided by the part's own row sum) and natural
+  // log-sum-exp in fp32 to the kernel's o [n_splits, BH*Nq, d] and lse [n_splits, BH*Nq]
+  // arguments, which the combine kernel then merges into the caller's O and LSE.
+  int n_splits;
   // The packed batch's work list, built on the device by the plan kernel that runs before
   // the prefill kernel (call-local workspace): the number of (sequence, Q-tile pair) items
   // that hold query rows, each sequence's (q0, Lq, k0, Lk) after the bounds checks and the
@@ -88,7 +94,7 @@ struct PagedKV {
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            void* o, float* lse, const PrefillParams& p, int d, bool bf16,
                            bool o_f32, int grid, int* status, cudaStream_t stream,
-                           bool qk8 = false);
+                           bool qk8 = false, float* part_o = nullptr, float* part_lse = nullptr);
 
 cudaError_t launch_decode(const void* q, const void* k, const void* v, void* o, float* lse,
                           const DecodeParams& p, int d, bool bf16, bool o_f32, float* part_o,

@@ -72,10 +72,21 @@ struct PrefillCfg {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t bars, int i) { return bars + 8u * i; }
 
-__device__ __forceinline__ void unit_coords(const PrefillParams& p, int u, int& bh, int& pair) {
+template <bool SPLIT>
+__device__ __forceinline__ void unit_coords(const PrefillParams& p, int u, int& bh, int& pair,
+                                            int& split) {
   // Heaviest first: the last Q-tile pairs (most causal work) of every head go first.
-  pair = p.n_pairs - 1 - u / p.BH;
-  bh = u % p.BH;
+  if constexpr (!SPLIT) {
+    pair = p.n_pairs - 1 - u / p.BH;
+    bh = u % p.BH;
+    split = 0;
+  } else {
+    const int per_pair = p.BH * p.n_splits;  // every head's parts of one pair
+    pair = p.n_pairs - 1 - u / per_pair;
+    const int rem = u % per_pair;
+    split = rem / p.BH;
+    bh = rem % p.BH;
+  }
 }
 
 // The unit a CTA takes in round r of the persistent loop.  Units are numbered heaviest
@@ -91,6 +102,7 @@ __device__ __forceinline__ int unit_of_round(int r) {
 // One work unit: its (b*H + h, Q-tile pair) and the sequence it belongs to.
 struct Unit {
   int bh, pair;
+  int split;   // part of the K/V range (K/V-split launches; 0 otherwise)
   int Lq, Lk;  // queries and keys of the sequence
   int q0, k0;  // first query / key token of the sequence (packed layout)
   int h;       // head within the sequence (packed layout)
@@ -104,11 +116,12 @@ __device__ __forceinline__ int unit_count(const PrefillParams& p) {
   return p.n_units;
 }
 
-template <bool VARLEN>
+template <bool VARLEN, bool SPLIT = false>
 __device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u) {
   Unit x;
+  x.split = 0;
   if constexpr (!VARLEN) {
-    unit_coords(p, u, x.bh, x.pair);
+    unit_coords<SPLIT>(p, u, x.bh, x.pair, x.split);
     x.Lq = p.Nq;
     x.Lk = p.Nkv;
     x.q0 = x.k0 = x.h = 0;
@@ -142,6 +155,22 @@ __device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, const Unit& 
   return min(ntk, last_key / BN + 1);
 }
 
+// The K/V tiles [j0, j1) unit x visits, of the [0, nmax) its Q-tile pair needs: all of them,
+// or (K/V-split launches) its split's consecutive part.  Tile t of the pair then visits
+// [j0, min(j1, n_t)).
+template <bool SPLIT>
+__device__ __forceinline__ void kv_range(const PrefillParams& p, const Unit& x, int nmax, int& j0,
+                                         int& j1) {
+  if constexpr (!SPLIT) {
+    j0 = 0;
+    j1 = nmax;
+  } else {
+    // nmax < 2^24 (a key count over 128) and n_splits <= 64: the products fit an int.
+    j0 = x.split * nmax / p.n_splits;
+    j1 = (x.split + 1) * nmax / p.n_splits;
+  }
+}
+
 // TMA coordinates (beyond the 64-column block) of the tile whose first row is `first`
 // (a query row or a key row of the unit's sequence): (row, b*H + h) in the [B,H,N,d]
 // view, (h, token) in the packed [tokens, H, d] view.
@@ -166,9 +195,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- producer (TMA)
-// QK8: Q and K hold one-byte E4M3 codes, one 128-byte row per query / key (d = 128), so a
-// Q or K tile is a single 128 x 128 B box in the first half of its slot.
-template <int D, bool VARLEN, bool QK8>
+template <int D, bool VARLEN, bool QK8, bool SPLIT>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                          const PrefillParams& p, uint32_t sbase, uint32_t bars, int* status,
                          volatile int* abort_flag) {
@@ -178,11 +205,16 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
   bool ok = true;
   const int n_units = unit_count<VARLEN>(p);
   for (int rnd = 0, u = unit_of_round(0); u < n_units && ok; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of<VARLEN>(p, u);
+    const Unit x = unit_of<VARLEN, SPLIT>(p, u);
     const int pair = x.pair;
-    const int n0 = kv_tiles_for(p, x, 2 * pair), n1 = kv_tiles_for(p, x, 2 * pair + 1);
-    const int nmax = max(n0, n1);
-    if (nmax == 0) continue;
+    int n0 = kv_tiles_for(p, x, 2 * pair), n1 = kv_tiles_for(p, x, 2 * pair + 1);
+    int j0 = 0, j1 = max(n0, n1);
+    if constexpr (SPLIT) {
+      kv_range<SPLIT>(p, x, j1, j0, j1);
+      n0 = (min(j1, n0) > j0) ? n0 : 0;  // a tile with nothing in this part loads no Q
+      n1 = (min(j1, n1) > j0) ? n1 : 0;
+    }
+    if (j1 <= j0) continue;
     if (!mbar_wait(bar_addr(bars, C::kBarQEmpty), (q_issued & 1) ^ 1, status, abort_flag,
                    kStatusTimeoutLoad)) {
       ok = false;
@@ -205,7 +237,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
       }
     }
     ++q_issued;
-    for (int j = 0; j < nmax && ok; ++j) {
+    for (int j = j0; j < j1 && ok; ++j) {
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t slot = ld % S, ph = (ld / S) & 1;
@@ -275,7 +307,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint6
   }
 }
 
-template <int D, bool BF16, bool VARLEN, bool QK8>
+template <int D, bool BF16, bool VARLEN, bool QK8, bool SPLIT>
 __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                            int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -295,28 +327,34 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
   };
   const int n_units = unit_count<VARLEN>(p);
   for (int rnd = 0, u = unit_of_round(0); u < n_units && ok; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of<VARLEN>(p, u);
-    const int n[2] = {kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)};
-    const int nmax = max(n[0], n[1]);
-    if (nmax == 0) continue;
+    const Unit x = unit_of<VARLEN, SPLIT>(p, u);
+    // n[t]: the end of tile t's K/V range in this unit (<= j0: nothing to do).
+    int n[2] = {kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)};
+    int j0 = 0, j1 = max(n[0], n[1]);
+    if constexpr (SPLIT) {
+      kv_range<SPLIT>(p, x, j1, j0, j1);
+      n[0] = min(j1, n[0]);
+      n[1] = min(j1, n[1]);
+    }
+    if (j1 <= j0) continue;
     if (!wait(C::kBarQFull, q_used & 1)) { ok = false; break; }
     tc_fence_after();
-    // S_t(0) for both tiles from K_0.
+    // S_t(j0) for both tiles from K_j0.
     const uint32_t kslot0 = ld % S;
     if (!wait(C::kBarFull + kslot0, (ld / S) & 1)) { ok = false; break; }
     tc_fence_after();
     ++ld;
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      if (n[t] == 0) continue;
+      if (n[t] <= j0) continue;
       issue_s<D, QK8>(tmem + t * 128, q_desc(t), k_desc(kslot0), idesc_s);
       tc_commit(bar_addr(bars, C::kBarSFull + t));
     }
     tc_commit(bar_addr(bars, C::kBarEmpty + kslot0));
     // The Q tiles are free once the last S that reads them completes: release them then,
     // so the next unit's Q load overlaps this unit's last softmax and P V products.
-    if (nmax == 1) tc_commit(bar_addr(bars, C::kBarQEmpty));
-    for (int j = 0; j < nmax && ok; ++j) {
+    if (j1 - j0 == 1) tc_commit(bar_addr(bars, C::kBarQEmpty));
+    for (int j = j0; j < j1 && ok; ++j) {
       const uint32_t vslot = ld % S;
       if (!wait(C::kBarFull + vslot, (ld / S) & 1)) { ok = false; break; }
       tc_fence_after();
@@ -330,7 +368,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
         if (!mbar_wait_spin(bar_addr(bars, C::kBarPFull + 2 * t), pcount[t] & 1, status,
                             abort_flag, kStatusTimeoutMma)) { ok = false; break; }
         tc_fence_after();
-        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, j > 0, 0);
+        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, j > j0, 0);
         tc_commit(bar_addr(bars, C::kBarOHalf + t));
         if (!mbar_wait_spin(bar_addr(bars, C::kBarPFull + 2 * t + 1), pcount[t] & 1, status,
                             abort_flag, kStatusTimeoutMma)) { ok = false; break; }
@@ -352,7 +390,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
       if (!ok) break;
       tc_commit(bar_addr(bars, C::kBarEmpty + vslot));
       if (knext >= 0) tc_commit(bar_addr(bars, C::kBarEmpty + knext));
-      if (j == nmax - 2) tc_commit(bar_addr(bars, C::kBarQEmpty));  // last S was issued above
+      if (j == j1 - 2) tc_commit(bar_addr(bars, C::kBarQEmpty));  // last S was issued above
     }
     if (!ok) break;
     ++q_used;
@@ -446,7 +484,9 @@ __device__ __forceinline__ float round_error(float xh) {
 // NEG: the scale is negative, so the row maximum of scale * s comes from the minimum of s.
 // QK8: E4M3 queries and keys; with per-tile scales (p.q_tscale, p.k_tscale) each score
 // tile's factor is scale * (its Q tile's scale) * (its K tile's scale).
-template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN, bool QK8>
+// SPLIT: the unit covers part of its pair's K/V range; it writes fp32 O / l and the natural
+// LSE of that part to o / lse, here the partial arrays (the combine kernel forms the result).
+template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN, bool QK8, bool SPLIT>
 __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t tmem, void* o,
                                  float* lse, int t, int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -466,14 +506,22 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
 
   const int n_units = unit_count<VARLEN>(p);
   for (int rnd = 0, u = unit_of_round(0); u < n_units; u = unit_of_round(++rnd)) {
-    const Unit x = unit_of<VARLEN>(p, u);
+    const Unit x = unit_of<VARLEN, SPLIT>(p, u);
     const int qtile = 2 * x.pair + t;
     if (qtile * BM >= x.Lq) continue;
-    const int n_kv = kv_tiles_for(p, x, qtile);
+    // This tile visits n_kv K/V tiles from tile j0 on (j0 = 0 unless the K/V range is
+    // split); j below counts them from j0.
+    int j0 = 0, n_kv = kv_tiles_for(p, x, qtile);
+    if constexpr (SPLIT) {
+      int j1;
+      kv_range<SPLIT>(p, x, max(kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)),
+                      j0, j1);
+      n_kv = max(0, min(j1, n_kv) - j0);
+    }
     const int row = qtile * BM + r;
     // Last key this row may see (keys beyond the sequence's are padding of its last tile,
-    // or the next sequence's in a packed batch).
-    const int limit = p.causal ? min(x.Lk - 1, row + x.Lk - x.Lq) : x.Lk - 1;
+    // or the next sequence's in a packed batch), counted from key tile j0's first key.
+    const int limit = (p.causal ? min(x.Lk - 1, row + x.Lk - x.Lq) : x.Lk - 1) - j0 * BN;
     float m_used = -INFINITY;  // running max in log2 units (may lag the true max by <= 8)
     float l = 0.f;             // running sum of the 16-bit-rounded 2^(x - m_used): divides O
     float l_exact = 0.f;       // the same sum before rounding: gives LSE
@@ -506,7 +554,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     for (int j = 0; j < n_kv; ++j) {
       float scale_log2 = sl2_q;
       if constexpr (QK8) {  // loaded before the wait, which hides its latency
-        if (p.k_tscale) scale_log2 *= p.k_tscale[static_cast<size_t>(x.bh) * p.n_kvtiles + j];
+        if (p.k_tscale) scale_log2 *= p.k_tscale[static_cast<size_t>(x.bh) * p.n_kvtiles + j0 + j];
       }
       if (!wait(C::kBarSFull + t, s_seen & 1)) return;
       ++s_seen;
@@ -621,6 +669,32 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     const size_t orow_i = !VARLEN ? static_cast<size_t>(x.bh) * p.Nq + row
                                   : (static_cast<size_t>(x.q0) + row) * p.H + x.h;
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+    if constexpr (SPLIT) {
+      // This part's record: O / l in fp32 and the natural LSE (-inf: no visible key).
+      const size_t prow = static_cast<size_t>(x.split) * p.BH * p.Nq + orow_i;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ob[32];
+        if (n_kv > 0) {
+          tmem_ld_32x32b_x32(tO + cc * 32, ob);
+          tmem_ld_wait(ob);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ob[i] = 0u;
+        }
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(o) + prow * D + cc * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(ob[4 * i]) * inv_l, __uint_as_float(ob[4 * i + 1]) * inv_l,
+                                 __uint_as_float(ob[4 * i + 2]) * inv_l, __uint_as_float(ob[4 * i + 3]) * inv_l);
+        }
+      }
+      if (valid)
+        lse[prow] =
+            (l_exact > 0.f) ? (m_used + log2f(l_exact)) * 0.69314718055994531f : -INFINITY;
+      continue;
+    }
     const size_t orow = orow_i * D;
 #pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {
@@ -659,7 +733,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   }
 }
 
-template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8>
+template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_prefill_sm100(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, void* __restrict__ o,
@@ -712,9 +786,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
     if (warp == 0) {
-      if (lane == 0) producer<D, VARLEN, QK8>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
+      if (lane == 0) producer<D, VARLEN, QK8, SPLIT>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D, BF16, VARLEN, QK8>(p, sbase, bars, tmem, status, abort_flag);
+      if (lane == 0) mma_issuer<D, BF16, VARLEN, QK8, SPLIT>(p, sbase, bars, tmem, status, abort_flag);
       __syncwarp();
       // Release TMEM once both softmax warpgroups have finished reading it.
       drain_wait(bar_addr(bars, C::kBarDone), 0);
@@ -726,9 +800,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // (Per-tile FP8 scales are positive: they never change the score factor's sign.)
     if (p.scale_log2 < 0.f)
-      softmax_epilogue<D, BF16, OF32, true, VARLEN, QK8>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, true, VARLEN, QK8, SPLIT>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     else
-      softmax_epilogue<D, BF16, OF32, false, VARLEN, QK8>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, false, VARLEN, QK8, SPLIT>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     tc_fence_before();
     mbar_arrive(bar_addr(bars, C::kBarDone));
   }
@@ -816,15 +890,82 @@ __global__ void __launch_bounds__(kPlanThreads)
   }
 }
 
-template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8>
+// Merges the n_splits partial records of every output row (one warp per row, D / 32
+// consecutive columns per lane): with w_s = exp(lse_s - max_s lse_s),
+// O = sum_s w_s O_s / sum_s w_s and LSE = max_s lse_s + log(sum_s w_s).  A row no part saw
+// a key of gets O = 0 and LSE = -inf.
+constexpr int kCombineThreads = 256;
+
+template <int D, bool BF16, bool OF32>
+__global__ void __launch_bounds__(kCombineThreads)
+    fa_prefill_combine(const float* __restrict__ part_o, const float* __restrict__ part_lse,
+                       void* __restrict__ o, float* __restrict__ lse, long long rows, int n_splits) {
+  constexpr int V = D / 32;
+  const long long row = static_cast<long long>(blockIdx.x) * (kCombineThreads / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int c0 = (threadIdx.x & 31) * V;
+  float m = -INFINITY;
+  for (int sp = 0; sp < n_splits; ++sp) m = fmaxf(m, part_lse[sp * rows + row]);
+  float acc[V], wsum = 0.f;
+#pragma unroll
+  for (int i = 0; i < V; ++i) acc[i] = 0.f;
+  if (m != -INFINITY) {
+    for (int sp = 0; sp < n_splits; ++sp) {
+      const float ls = part_lse[sp * rows + row];
+      const float w = (ls == -INFINITY) ? 0.f : expf(ls - m);
+      wsum += w;
+      const float* src = part_o + (sp * rows + row) * D + c0;
+      float x[V];
+      if constexpr (V == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(src);
+        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+      } else {
+        const float2 t = *reinterpret_cast<const float2*>(src);
+        x[0] = t.x; x[1] = t.y;
+      }
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[i] = fmaf(w, x[i], acc[i]);
+    }
+  }
+  const float inv = (wsum > 0.f) ? 1.0f / wsum : 0.f;
+  if constexpr (OF32) {
+    float* dst = static_cast<float*>(o) + row * D + c0;
+    if constexpr (V == 4)
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    else
+      *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+  } else {
+    uint16_t* dst = static_cast<uint16_t*>(o) + row * D + c0;
+    if constexpr (V == 4)
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack2<BF16>(acc[0] * inv, acc[1] * inv),
+                                                  pack2<BF16>(acc[2] * inv, acc[3] * inv));
+    else
+      *reinterpret_cast<uint32_t*>(dst) = pack2<BF16>(acc[0] * inv, acc[1] * inv);
+  }
+  if (lse != nullptr && (threadIdx.x & 31) == 0)
+    lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
+}
+
+template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT = false>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                      float* lse, const PrefillParams& p, int grid, int* status,
-                     cudaStream_t stream) {
-  auto kern = fa_prefill_sm100<D, BF16, OF32, VARLEN, QK8>;
+                     cudaStream_t stream, float* part_o = nullptr, float* part_lse = nullptr) {
+  // A split launch writes fp32 partial records whatever the output type.
+  auto kern = fa_prefill_sm100<D, BF16, SPLIT ? false : OF32, VARLEN, QK8, SPLIT>;
   const cudaError_t config_err =
       configure_kernel(reinterpret_cast<const void*>(kern), PrefillCfg<D>::kAlloc, kRegsLaunch);
   if (config_err != cudaSuccess) return config_err;
-  kern<<<grid, kThreads, PrefillCfg<D>::kAlloc, stream>>>(tq, tk, tv, o, lse, p, status);
+  if constexpr (SPLIT) {
+    kern<<<grid, kThreads, PrefillCfg<D>::kAlloc, stream>>>(tq, tk, tv, part_o, part_lse, p, status);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long rows = static_cast<long long>(p.BH) * p.Nq;
+    const long long blocks = (rows + kCombineThreads / 32 - 1) / (kCombineThreads / 32);
+    fa_prefill_combine<D, BF16, OF32><<<static_cast<unsigned>(blocks), kCombineThreads, 0, stream>>>(
+        part_o, part_lse, o, lse, rows, p.n_splits);
+  } else {
+    kern<<<grid, kThreads, PrefillCfg<D>::kAlloc, stream>>>(tq, tk, tv, o, lse, p, status);
+  }
   return cudaGetLastError();
 }
 
@@ -836,7 +977,8 @@ size_t prefill_smem_bytes(int d) {
 
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            void* o, float* lse, const PrefillParams& p, int d, bool bf16,
-                           bool o_f32, int grid, int* status, cudaStream_t stream, bool qk8) {
+                           bool o_f32, int grid, int* status, cudaStream_t stream, bool qk8,
+                           float* part_o, float* part_lse) {
   if (qk8) {  // E4M3 queries and keys: d = 128, [B,H,N,d] layout
     if (d != 128 || p.cu_q) return cudaErrorInvalidValue;
     if (bf16 && o_f32) return launch_t<128, true, true, false, true>(tq, tk, tv, o, lse, p, grid, status, stream);
@@ -856,7 +998,10 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
 #define FA_PREFILL_CASE(D_, B_, F_)                                                               \
   if (d == D_ && bf16 == B_ && o_f32 == F_)                                                        \
     return p.cu_q ? launch_t<D_, B_, F_, true, false>(tq, tk, tv, o, lse, p, grid, status, stream) \
-                  : launch_t<D_, B_, F_, false, false>(tq, tk, tv, o, lse, p, grid, status, stream);
+           : p.n_splits > 1                                                                        \
+               ? launch_t<D_, B_, F_, false, false, true>(tq, tk, tv, o, lse, p, grid, status, stream, \
+                                                          part_o, part_lse)                        \
+               : launch_t<D_, B_, F_, false, false>(tq, tk, tv, o, lse, p, grid, status, stream);
   FA_PREFILL_CASE(128, true, true)
   FA_PREFILL_CASE(128, true, false)
   FA_PREFILL_CASE(128, false, true)

@@ -91,13 +91,50 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 
 /*
  * fa_fwd_prefill -- the tiled prefill path for any Nq >= 1 (the work of fa_fwd with
- * Nq > 1).  num_ctas: persistent CTAs to launch; 0 picks one per SM, larger values are
- * clamped to the number of work units (pairs of 128-row query tiles).  Same arguments,
- * layouts and errors as fa_fwd.
+ * Nq > 1).  num_ctas: persistent CTAs to launch; 0 picks one per SM (and splits the K/V
+ * range of small problems as fa_fwd_prefill_split does with num_splits = 0), larger values
+ * are clamped to the number of work units (pairs of 128-row query tiles) and run them
+ * unsplit.  Same arguments, layouts and errors as fa_fwd.
  */
 int fa_fwd_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                    int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
                    int in_dtype, int o_dtype, int num_ctas);
+
+/*
+ * fa_fwd_prefill_split -- the prefill path with the K/V range of every (head, Q-tile pair)
+ * cut into num_splits consecutive parts of whole 128-key tiles, each part a work unit of
+ * its own.  Each unit writes, per query row, the softmax-weighted mean of V over its part's
+ * keys and that part's log-sum-exp (fp32, to workspace from the library's stream-ordered
+ * pool); a combine kernel then merges the parts exactly: with w_s = exp(lse_s - max lse),
+ * O = sum w_s O_s / sum w_s and LSE = max lse + log sum w_s.  This is the decode path's
+ * split-KV merge ("FlashAttention 1-2-3" (myaihardware), the FlashDecoding split of section
+ * "Beyond FlashAttention") applied to prefills with fewer Q-tile pairs than SMs, where the
+ * longest pair would otherwise set the run time alone.
+ *   num_splits: 0 chooses (fa_prefill_num_splits: 1 once there are at least as many
+ *   units as SMs, else the count, up to 8, that a run-time model of the kernel predicts
+ *   to be fastest, if it beats no split by at least 10%); 1 runs unsplit; 2..64 forces
+ *   that many parts (clamped to the K/V tile count).
+ *   num_ctas as for fa_fwd_prefill (0: one per SM; clamped to the split unit count).
+ *   Workspace: num_splits * B*H*Nq * (d + 1) * 4 bytes, allocated and freed on `stream`.
+ *   Same arguments, layouts, results (up to the merge's rounding) and errors as fa_fwd,
+ *   plus FA_ERR_INVALID_ARG for num_ctas < 0 or num_splits outside 0..64, and FA_ERR_NOMEM
+ *   when the pool cannot supply the workspace.
+ */
+int fa_fwd_prefill_split(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int Nq, int Nkv, int d, float scale, int causal,
+                         void* stream, int in_dtype, int o_dtype, int num_ctas, int num_splits);
+
+/*
+ * fa_prefill_num_splits -- the K/V part count the prefill path chooses by itself (fa_fwd
+ * with Nq > 1, fa_fwd_prefill with num_ctas = 0, fa_fwd_prefill_split with num_splits = 0)
+ * for this shape on a GPU with sm_count SMs (0: the current device's), written to
+ * *num_splits; the split workspace of a call is then *num_splits * B*H*Nq * (d + 1) * 4
+ * bytes when *num_splits > 1.  Host arithmetic only when sm_count > 0.  FA_ERR_INVALID_ARG
+ * for a null pointer, B, H, Nq or Nkv < 1, d not 64 or 128, causal not 0 or 1, or
+ * sm_count < 0.
+ */
+int fa_prefill_num_splits(int B, int H, int Nq, int Nkv, int d, int causal, int sm_count,
+                          int* num_splits);
 
 /*
  * fa_fwd_decode -- split-KV decode for one query per head: q [B,H,1,d], k/v [B,H,Nkv,d],

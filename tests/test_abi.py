@@ -3,6 +3,7 @@ host-side argument checks return the documented codes without touching a device.
 
 Pointers below are fake integers; every case is rejected before any CUDA call, so these
 tests run on a CPU-only machine (and launch nothing on a GPU machine)."""
+import ctypes
 import math
 import subprocess
 
@@ -83,12 +84,36 @@ def test_prefill_and_decode_entry_checks():
     lib = binding
     assert lib.fa_fwd_prefill(Q, K, V, O, L, 1, 1, 4, 4, 64, 0.1, 0, None, 0, 2, -1) == \
         binding.FA_ERR_INVALID_ARG
+    for ctas, splits in ((-1, 0), (0, -1), (0, 65)):
+        assert lib.fa_fwd_prefill_split(Q, K, V, O, L, 1, 1, 4, 4, 64, 0.1, 0, None, 0, 2,
+                                        ctas, splits) == binding.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_decode(Q, K, V, O, L, 1, 1, 4, 64, 0.1, None, 0, 2, -1) == \
         binding.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_decode(None, K, V, O, L, 1, 1, 4, 64, 0.1, None, 0, 2, 0) == \
         binding.FA_ERR_INVALID_ARG
     assert lib.fa_fwd_decode(Q, K, V, O, L, 1, 1, 4, 80, 0.1, None, 0, 2, 0) == \
         binding.FA_ERR_UNSUPPORTED
+
+
+def test_prefill_split_choice_is_host_arithmetic():
+    ns = binding.prefill_num_splits
+    # at least one unit (pair of 128-row Q tiles of one head) per SM: never split
+    assert ns(1, 32, 8192, 8192, 128, True, 148) == 1
+    assert ns(3, 1, 148 * 256, 148 * 256, 64, False, 148) == 1
+    assert ns(1, 148, 256, 256, 128, False, 148) == 1
+    # one head of 16k causal tokens on 148 SMs: 64 units, the longest 128 K/V tiles
+    assert 2 <= ns(1, 1, 16384, 16384, 128, True, 148) <= 8
+    # many short units: the split's fixed cost is not worth it
+    assert ns(2, 8, 2048, 2048, 64, True, 148) == 1
+    # never more parts than K/V tiles
+    assert ns(1, 1, 300, 200, 128, False, 148) <= 2
+    for args in ((0, 1, 4, 4, 64, 0, 148), (1, 1, 4, 4, 96, 0, 148), (1, 1, 4, 4, 64, 2, 148),
+                 (1, 1, 4, 4, 64, 0, -1)):
+        out = ctypes.c_int(0)
+        assert binding.library().fa_prefill_num_splits(*args, ctypes.byref(out)) == \
+            binding.FA_ERR_INVALID_ARG
+    assert binding.library().fa_prefill_num_splits(1, 1, 4, 4, 64, 0, 148, None) == \
+        binding.FA_ERR_INVALID_ARG
 
 
 def test_decode_workspace_size_formula():
@@ -121,6 +146,10 @@ calls = {
     "fa_fwd": lambda: b.fa_fwd(Q, K, V, O, L, 1, 2, 16, 16, 64, 0.125, 0, None, 0, 2),
     "fa_fwd_prefill": lambda: b.fa_fwd_prefill(Q, K, V, O, L, 1, 2, 16, 16, 64, 0.125, 1, None,
                                                0, 2, 0),
+    "fa_fwd_prefill_split": lambda: b.fa_fwd_prefill_split(Q, K, V, O, L, 1, 2, 600, 600, 64,
+                                                           0.125, 1, None, 0, 2, 0, 3),
+    "fa_prefill_num_splits": lambda: lib.fa_prefill_num_splits(1, 1, 9000, 9000, 128, 1, 0,
+                                                               ctypes.byref(ctypes.c_int(0))),
     "fa_fwd_decode": lambda: b.fa_fwd_decode(Q, K, V, O, L, 1, 2, 16, 64, 0.125, None, 0, 2, 0),
     "fa_fwd_decode_noalloc": lambda: b.fa_fwd_decode_noalloc(Q, K, V, O, L, 1, 2, 16, 64, 0.125,
                                                              None, 0, 2, 0),

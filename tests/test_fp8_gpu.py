@@ -75,7 +75,7 @@ def test_fp8_equals_bf16_path_on_exact_values(causal):
     o8, l8 = binding.fp8_attention(q8.cuda(), k8.cuda(), v.cuda(), 1.0, 1.0, causal=causal,
                                    scale=0.02)
     o16, l16 = binding.attention(qi.to(torch.bfloat16).cuda(), ki.to(torch.bfloat16).cuda(),
-                                 v.cuda(), causal=causal, scale=0.02)
+                                 v.cuda(), causal=causal, scale=0.02, num_splits=1)
     torch.cuda.synchronize()
     assert torch.equal(o8, o16) and torch.equal(l8, l16)
 

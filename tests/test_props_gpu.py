@@ -89,20 +89,35 @@ def test_decode_split_counts_agree():
         assert (l - outs[0][1]).abs().max().item() <= 1e-4
 
 
-def test_prefill_grid_sizes_agree_bitwise():
-    """Each Q tile is computed by one CTA in a fixed order, so the grid size must not
-    change a single bit."""
+@pytest.mark.parametrize("num_splits", [1, 3])
+def test_prefill_grid_sizes_agree_bitwise(num_splits):
+    """Each Q tile (each part of its K/V range, when split) is computed by one CTA in a
+    fixed order and the parts are merged in a fixed order, so the grid size must not change
+    a single bit."""
     q, k, v = make_qkv(2, 3, 900, 900, 128, torch.bfloat16, 7, device="cuda")
-    ref = binding.attention(q, k, v, causal=True, num_ctas=0)
+    ref = binding.attention(q, k, v, causal=True, num_ctas=0, num_splits=num_splits)
     for n in (1, 5):
-        o, l = binding.attention(q, k, v, causal=True, num_ctas=n)
+        o, l = binding.attention(q, k, v, causal=True, num_ctas=n, num_splits=num_splits)
         torch.cuda.synchronize()
         assert torch.equal(o, ref[0]) and torch.equal(l, ref[1])
 
 
+def test_prefill_split_agrees_with_unsplit():
+    """Splitting the K/V range changes only the rounding of the merge."""
+    q, k, v = make_qkv(1, 4, 2048, 2048, 64, torch.float16, 8, q_std=3.0, device="cuda")
+    ref = binding.attention(q, k, v, causal=True, num_splits=1)
+    for s in (2, 4, 0):
+        o, l = binding.attention(q, k, v, causal=True, num_splits=s)
+        torch.cuda.synchronize()
+        assert (o - ref[0]).abs().max().item() <= MAX_ABS_O
+        assert (l - ref[1]).abs().max().item() <= MAX_ABS_LSE
+
+
 def test_no_score_matrix_in_memory():
     """The n x n matrix never reaches HBM: at N = 16384 one head's fp32 scores alone would
-    be 1 GiB, yet the call allocates nothing beyond O and LSE."""
+    be 1 GiB, yet a call needs nothing beyond O, LSE and (for this small problem, whose
+    K/V range is split) O(N d) partials from the library's pool, which a repeated call
+    reuses."""
     q, k, v = make_qkv(1, 2, 16384, 16384, 128, torch.bfloat16, 11, device="cuda")
     o = torch.empty(q.shape, dtype=torch.float32, device="cuda")
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")

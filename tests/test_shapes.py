@@ -3,7 +3,9 @@
 Covers: Nq and Nkv not multiples of the 128-row tile (tails), Nq != Nkv with the causal
 mask aligned bottom-right, causal rows that see no key (Nq > Nkv), one query row through
 the prefill path, head dims 64 and 128, fp16 and bf16, fp32 and 16-bit O, a persistent
-grid smaller than the work (num_ctas) and decode with several split counts.
+grid smaller than the work (num_ctas), prefill with its K/V range split into parts
+(num_splits; the small shapes above also take the split when the library chooses it) and
+decode with several split counts.
 """
 import pytest
 import torch
@@ -92,6 +94,27 @@ def test_16bit_output(d, dtype):
 @pytest.mark.parametrize("num_ctas", [1, 3, 7])
 def test_persistent_grid_smaller_than_work(num_ctas):
     _run_case(2, 3, 700, 700, 128, torch.bfloat16, True, num_ctas=num_ctas)
+
+
+@pytest.mark.parametrize("num_splits", [1, 2, 3, 4, 7, 64])
+@pytest.mark.parametrize("causal", [False, True])
+def test_prefill_kv_split_counts(num_splits, causal):
+    # 9 key tiles: 7 parts leave some pairs' parts empty, 64 is clamped to the tile count
+    _run_case(1, 2, 700, 1100, 128, torch.bfloat16, causal, num_splits=num_splits)
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 1000, 300), (2, 1, 300, 1000), (1, 1, 129, 640)])
+@pytest.mark.parametrize("num_ctas", [0, 1, 5])
+def test_prefill_kv_split_ragged_small_grid(shape, num_ctas):
+    # causal rows that see no key (Nq > Nkv), bottom-right alignment (Nq < Nkv), and a
+    # persistent grid smaller than the split work
+    _run_case(*shape, 64, torch.float16, True, num_ctas=num_ctas, num_splits=3)
+
+
+@pytest.mark.parametrize("d,dtype", [(64, torch.bfloat16), (128, torch.float16)])
+def test_prefill_kv_split_16bit_output_and_negative_scale(d, dtype):
+    _run_case(1, 3, 500, 900, d, dtype, True, out_dtype=dtype, num_splits=4)
+    _run_case(1, 2, 400, 800, d, dtype, False, scale=-0.3, num_splits=2)
 
 
 @pytest.mark.parametrize("Nkv", [1, 5, 64, 65, 1000])
