@@ -27,18 +27,21 @@
 //    has read it;
 //  * warp 1 (one lane): tcgen05.mma issue, per query tile i:
 //        dV  += P^T dO_i   (A = P^T, 16-bit, from TMEM over S; B = dO_i MN-major)
-//        dK  += dS^T Q_i   (A = dS^T, 16-bit, from TMEM over dP; B = Q_i MN-major)
 //        S^T  = K Q_{i+1}^T  (M 128 keys, N 128 queries, K = d) into S, once dV(i) is issued
 //        dQ^T = K^T dS^T   (M 128 = d, N 128 queries, K 128 keys; A = K read MN-major, B = dS
-//                           from shared memory) into dP, over dS^T once dK(i) is issued
+//                           from shared memory) into dP, whose dP(i) the softmax has read
+//        dK  += dS^T Q_i   (A = dS^T, the same shared-memory tile read K-major; B = Q_i
+//                           MN-major), issued after dQ^T(i) so that the drain of dQ^T(i)
+//                           overlaps it
 //        dP^T = V dO_{i+1}^T into dP, once the drain has read dQ^T(i) out of it
 //    tcgen05.mma operations run in issue order, so an MMA that overwrites columns an
 //    earlier MMA reads as its A operand needs no wait in between;
 //  * warpgroups 1 and 2 (warps 4-7 and 8-11) both work on every query tile, one thread per
-//    key, warpgroup w on queries 64w .. 64w+63: P^T from S^T as soon as S is ready, then
-//    dS^T = P^T (dP^T - D) once dP is; each stored back as 16-bit over the warpgroup's
-//    own S / dP columns (64w .. 64w+31), dS also to shared memory for the dQ product.  At
-//    the end warpgroup 1 writes dV and warpgroup 2 writes scale * dK;
+//    key, warpgroup w on queries 64w .. 64w+63: P^T from S^T as soon as S is ready,
+//    stored back as 16-bit over the warpgroup's own S columns (64w .. 64w+31) for dV; then
+//    dS^T = P^T (dP^T - D) once dP is, stored to shared memory (128-byte swizzle, one
+//    128-byte row per key and 64-query block) for both dQ and dK.  At the end warpgroup 1
+//    writes dV and warpgroup 2 writes scale * dK;
 //  * warpgroup 3 (warps 12-15), one thread per d-row of dQ^T: TMEM -> registers (the
 //    columns are then free for dP(i+1)) -> fp32 reductions into row-major dQ accumulator
 //    rows, each warp instruction adding 32 consecutive floats of one query row.
@@ -91,10 +94,11 @@ struct BwdCfg {
   static constexpr int kBarSFull = kBarDOFree + 1;   // S(i) complete
   static constexpr int kBarDPFull = kBarSFull + 1;   // dP(i) complete
   static constexpr int kBarPReady = kBarDPFull + 1;  // P^T(i) stored (8 softmax warps)
-  static constexpr int kBarDSReady = kBarPReady + 1; // dS^T(i) and dS(i) stored (8 warps)
+  static constexpr int kBarDSReady = kBarPReady + 1; // dS(i) stored to shared memory (8 warps)
   static constexpr int kBarDQFull = kBarDSReady + 1; // dQ^T(i) complete (and all before it)
   static constexpr int kBarDQEmpty = kBarDQFull + 1; // dQ^T(i) read out of TMEM (4 warps)
-  static constexpr int kBarDone = kBarDQEmpty + 1;   // every MMA of the CTA complete
+  static constexpr int kBarQFree = kBarDQEmpty + 1;  // dK(i) complete: Q stage i and dS free
+  static constexpr int kBarDone = kBarQFree + 1;     // every MMA of the CTA complete
   static constexpr int kBarFinished = kBarDone + 1;  // warps 4-15 done with TMEM
   static constexpr int kNumBars = kBarFinished + 1;
   static constexpr int kTmemHolderOff = kBarOff + kNumBars * 8;
@@ -110,7 +114,7 @@ struct BwdCfg {
 // TMEM columns.
 constexpr uint32_t kTdV = 0, kTdK = 128, kTS = 256, kTdP = 384;
 
-// Column of the 16-bit A operand (P^T or dS^T, 8 columns per 16 queries) for K-step kk:
+// Column of the 16-bit A operand P^T (8 columns per 16 queries) for K-step kk:
 // warpgroup w stores its queries 64w .. 64w+63 over its own columns 64w .. 64w+31.
 __device__ __forceinline__ uint32_t a16_col(int kk) { return (kk < 4) ? 8u * kk : 64u + 8u * (kk - 4); }
 
@@ -161,9 +165,10 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
   for (int i = 0; i < n; ++i) {
     const int st = i % kStages;
     const int q0 = (i0 + i) * kBQ;
-    // Q stage st held tile i - 2, whose products are all complete once its dQ is (dQ(i-1)
-    // cannot complete before Q(i) is loaded, so the barrier is at most one phase ahead).
-    if (i >= kStages && !(ok = wait(C::kBarDQFull, (i - kStages) & 1))) break;
+    // Q stage st held tile i - 2, whose products are all complete once its dK is (dK(i-1)
+    // is issued after S(i), so it cannot complete before Q(i) is loaded: the barrier is at
+    // most one phase ahead).
+    if (i >= kStages && !(ok = wait(C::kBarQFree, (i - kStages) & 1))) break;
     const uint32_t qf = bar_addr(bars, C::kBarQFull + st);
     mbar_arrive_expect_tx(qf, C::kTileBytes + 2 * kBQ * 4);
 #pragma unroll
@@ -213,6 +218,8 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
   auto kt_desc = [&]() { return at(mn0, C::kKOff); };
   // dS as the MN-major B of dQ^T: two 64-query blocks 128 keys x 128 B = 16 KB apart.
   auto ds_desc = [&]() { return at(mn0, C::kdSOff); };
+  // dS as the K-major A of dK (M = 128 keys, K = 128 queries): the same tile.
+  auto ds_kmaj = [&]() { return at(kmaj0, C::kdSOff); };
   auto q_kmaj = [&](int st) { return at(kmaj0, C::kQOff + st * C::kTileBytes); };
   auto do_kmaj = [&]() { return at(kmaj0, C::kdOOff); };
   // Q and dO as MN-major B (d contiguous): d blocks 128 x 128 B = 16 KB apart, 16 queries
@@ -260,20 +267,22 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
       issue_st(kTS, k_desc(), q_kmaj(st1));
       tc_commit(bar_addr(bars, C::kBarSFull));
     }
-    // dS^T(i) is stored over dP and dS(i) in shared memory: dK(i).
+    // dS(i) is in shared memory (the softmax has read dP(i) out of TMEM): dQ^T(i) over dP
+    // first, so that the drain starts while dK(i) runs, then dK(i) with dS^T read from the
+    // same shared-memory tile as a K-major A operand.
     if (!(ok = wait(C::kBarDSReady, i & 1))) break;
     tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < kBQ / 16; ++kk)
-      mma_ts(tmem + kTdK, tmem + kTdP + a16_col(kk), q_mn(st) + ((kk * 2048) >> 4), idesc_kv,
-             (i > 0 || kk > 0) ? 1u : 0u);
-    // dQ^T(i) over dP: dS^T(i) there has been read by dK(i), issued above.
 #pragma unroll
     for (int kk = 0; kk < kBK / 16; ++kk)
       mma_ss(tmem + kTdP, kt_desc() + ((kk * 2048) >> 4), ds_desc() + ((kk * 2048) >> 4), idesc_q,
              kk > 0 ? 1u : 0u);
-    // Tile i's products are complete: its dQ can be drained, its Q stage and dS reused.
     tc_commit(bar_addr(bars, C::kBarDQFull));
+#pragma unroll
+    for (int kk = 0; kk < kBQ / 16; ++kk)
+      mma_ss(tmem + kTdK, ds_kmaj() + kmajor_step(kk, kBK), q_mn(st) + ((kk * 2048) >> 4),
+             idesc_kv, (i > 0 || kk > 0) ? 1u : 0u);
+    // Tile i's products are complete: its Q stage and dS may be reused.
+    tc_commit(bar_addr(bars, C::kBarQFree));
     if (i + 1 < n) {
       // dP(i+1) over dP, once the drain has read dQ^T(i) and dO(i+1) has landed.
       if (!(ok = wait(C::kBarDQEmpty, i & 1))) break;
@@ -353,8 +362,8 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
     }
     tmem_st_wait();
     arrive(C::kBarPReady);
-    // dS = P (dP - D) once dP(i) is complete (dQ(i-1), issued before dP(i), is complete
-    // too, so the shared-memory dS buffer is free).
+    // dS = P (dP - D) once dP(i) is complete (dQ(i-1) and dK(i-1), issued before dP(i),
+    // are complete too, so the shared-memory dS buffer is free).
     if (!(ok = wait(C::kBarDPFull, i & 1))) break;
     tc_fence_after();
     const float4* dl = reinterpret_cast<const float4*>(sgen + C::kDelOff + st * kBQ * 4 + c0 * 4);
@@ -378,8 +387,6 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
         pk[2 * c4] = pack2<BF16>(d0, d1);
         pk[2 * c4 + 1] = pack2<BF16>(d2, d3);
       }
-      // dS^T over this warpgroup's first 32 dP columns (16-bit pairs), already read.
-      tmem_st_32x32b_x16(tdP + 16 * h, pk);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int cc = 4 * h + j;
@@ -387,7 +394,6 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
             make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
       }
     }
-    tmem_st_wait();
     fence_proxy_async_smem();
     arrive(C::kBarDSReady);
   }
@@ -511,6 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_addr(bars, C::kBarDSReady), 8);
     mbar_init(bar_addr(bars, C::kBarDQFull), 1);
     mbar_init(bar_addr(bars, C::kBarDQEmpty), 4);    // one arrival per drain warp
+    mbar_init(bar_addr(bars, C::kBarQFree), 1);
     mbar_init(bar_addr(bars, C::kBarDone), 1);
     mbar_init(bar_addr(bars, C::kBarFinished), 12);  // one per warp of warps 4-15
     *abort_flag = 0;
