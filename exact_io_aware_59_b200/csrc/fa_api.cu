@@ -406,8 +406,8 @@ int run_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   p.H = H;
   p.total_q = total_q;
   p.total_k = total_k;
-  // Call-local workspace for the plan: item count (16 bytes), B sequence records, B first
-  // positions, items.
+  // Call-local workspace for the plan: item count and work counter (16 bytes), B sequence
+  // records, B first positions, items.
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   void* ws = nullptr;
   const size_t seq_b = static_cast<size_t>(B) * sizeof(int4), first_b = static_cast<size_t>(B) * 4;
@@ -415,6 +415,7 @@ int run_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
   if ((rc = workspace_alloc(ds, ws_bytes, st, &ws)) != FA_OK) return rc;
   char* w = static_cast<char*>(ws);
   p.vl_count = reinterpret_cast<int*>(w);
+  p.vl_next = reinterpret_cast<int*>(w) + 1;
   p.vl_seqs = reinterpret_cast<int4*>(w + 16);
   p.vl_first = reinterpret_cast<int*>(w + 16 + seq_b);
   p.vl_items = reinterpret_cast<int*>(w + 16 + seq_b + first_b);

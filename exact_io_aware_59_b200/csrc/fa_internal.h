@@ -37,6 +37,9 @@ struct PrefillParams {
   // position of its first item, and the items, each as b * n_pairs + pair.  Work unit u is
   // head u % H of item u / H.
   const int* vl_count;
+  // Work counter of the packed batch: zeroed by the plan kernel; the prefill kernel's CTAs
+  // claim units from it in list order.
+  int* vl_next;
   const int4* vl_seqs;
   const int* vl_first;
   const int* vl_items;

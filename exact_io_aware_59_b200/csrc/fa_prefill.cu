@@ -43,6 +43,11 @@ static_assert(128 * kRegsSide + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "r
 // so the result is the same softmax whatever the lag.
 constexpr float kLazyLog2 = 15.0f;
 
+// Slots of the ring through which a packed batch's claimed units reach the CTA's roles.
+constexpr int kUnitSlots = 4;
+// Arrivals that free a slot: the MMA lane and the eight softmax warps.
+constexpr int kUnitReaders = 9;
+
 template <int D>
 struct PrefillCfg {
   static constexpr int kQBytes = BM * D * 2;
@@ -62,10 +67,13 @@ struct PrefillCfg {
   static constexpr int kBarODone = kBarOHalf + 2;    // + tile
   static constexpr int kBarDrain = kBarODone + 2;
   static constexpr int kBarDone = kBarDrain + 1;     // softmax warps finished with TMEM
-  static constexpr int kNumBars = kBarDone + 1;
+  static constexpr int kBarUnitFull = kBarDone + 1;  // + slot: a claimed unit published
+  static constexpr int kBarUnitEmpty = kBarUnitFull + kUnitSlots;  // + slot: read by all
+  static constexpr int kNumBars = kBarUnitEmpty + kUnitSlots;
   static constexpr int kTmemHolderOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemHolderOff + 4;
-  static constexpr int kBytes = kAbortOff + 4;
+  static constexpr int kUnitOff = kAbortOff + 4;     // the claimed-unit ring (packed batches)
+  static constexpr int kBytes = kUnitOff + 4 * kUnitSlots;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
@@ -97,6 +105,40 @@ __device__ __forceinline__ void unit_coords(const PrefillParams& p, int u, int& 
 __device__ __forceinline__ int unit_of_round(int r) {
   const int G = gridDim.x, c = blockIdx.x;
   return r * G + ((r & 1) ? (G - 1 - c) : c);
+}
+
+// Packed batches are listed sequence by sequence (so that the CTAs running together share
+// one sequence's K and V in L2), an order the static snake balances poorly on ragged
+// lengths (busiest CTA about 7% above the mean on a batch of lengths 512-8192, against
+// 0.3% for claiming in list order).  So their units are claimed from a work counter: the
+// producer lane takes the next unit with one atomicAdd (which also bounds how far it runs
+// ahead) and publishes it in a shared-memory ring slot; the MMA lane and the softmax warps
+// read the slots in the same order and free them.  A unit index >= the unit count ends
+// every role's loop.  Which CTA runs a unit changes no result: a unit's rows depend on
+// its inputs alone.
+__device__ __forceinline__ int ld_shared_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_shared_s32(uint32_t addr, int v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int claim_unit(const PrefillParams& p, uint32_t full_bar,
+                                          uint32_t empty_bar, uint32_t ring, int rnd,
+                                          int* status, volatile int* abort_flag, bool& ok) {
+  const int slot = rnd % kUnitSlots;
+  if (!mbar_wait(empty_bar + 8u * slot, ((rnd / kUnitSlots) & 1) ^ 1, status, abort_flag,
+                 kStatusTimeoutLoad)) {
+    ok = false;
+    return 0;
+  }
+  const int u = atomicAdd(p.vl_next, 1);
+  st_shared_s32(ring + 4u * slot, u);
+  mbar_arrive(full_bar + 8u * slot);  // release: waiters that see the phase see the slot
+  return u;
 }
 
 // One work unit: its (b*H + h, Q-tile pair) and the sequence it belongs to.
@@ -204,7 +246,12 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
   uint32_t ld = 0, q_issued = 0;
   bool ok = true;
   const int n_units = unit_count<VARLEN>(p);
-  for (int rnd = 0, u = unit_of_round(0); u < n_units && ok; u = unit_of_round(++rnd)) {
+  for (int rnd = 0;; ++rnd) {
+    const int u = VARLEN ? claim_unit(p, bar_addr(bars, C::kBarUnitFull),
+                                      bar_addr(bars, C::kBarUnitEmpty), sbase + C::kUnitOff,
+                                      rnd, status, abort_flag, ok)
+                         : unit_of_round(rnd);
+    if (!ok || u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
     const int pair = x.pair;
     int n0 = kv_tiles_for(p, x, 2 * pair), n1 = kv_tiles_for(p, x, 2 * pair + 1);
@@ -326,7 +373,17 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
     return mbar_wait(bar_addr(bars, b), parity, status, abort_flag, kStatusTimeoutMma);
   };
   const int n_units = unit_count<VARLEN>(p);
-  for (int rnd = 0, u = unit_of_round(0); u < n_units && ok; u = unit_of_round(++rnd)) {
+  for (int rnd = 0;; ++rnd) {
+    int u;
+    if constexpr (VARLEN) {
+      const int slot = rnd % kUnitSlots;
+      if (!wait(C::kBarUnitFull + slot, (rnd / kUnitSlots) & 1)) { ok = false; break; }
+      u = ld_shared_s32(sbase + C::kUnitOff + 4u * slot);
+      mbar_arrive(bar_addr(bars, C::kBarUnitEmpty + slot));
+    } else {
+      u = unit_of_round(rnd);
+    }
+    if (u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
     // n[t]: the end of tile t's K/V range in this unit (<= j0: nothing to do).
     int n[2] = {kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)};
@@ -505,7 +562,18 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   };
 
   const int n_units = unit_count<VARLEN>(p);
-  for (int rnd = 0, u = unit_of_round(0); u < n_units; u = unit_of_round(++rnd)) {
+  for (int rnd = 0;; ++rnd) {
+    int u;
+    if constexpr (VARLEN) {
+      const int slot = rnd % kUnitSlots;
+      if (!wait(C::kBarUnitFull + slot, (rnd / kUnitSlots) & 1)) return;
+      u = ld_shared_s32(bars - C::kBarOff + C::kUnitOff + 4u * slot);
+      __syncwarp();  // every lane has read the slot before it is freed
+      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarUnitEmpty + slot));
+    } else {
+      u = unit_of_round(rnd);
+    }
+    if (u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
     const int qtile = 2 * x.pair + t;
     if (qtile * BM >= x.Lq) continue;
@@ -764,6 +832,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar_addr(bars, C::kBarDrain), 1);
     mbar_init(bar_addr(bars, C::kBarDone), 256);
+    for (int s = 0; s < kUnitSlots; ++s) {
+      mbar_init(bar_addr(bars, C::kBarUnitFull + s), 1);
+      mbar_init(bar_addr(bars, C::kBarUnitEmpty + s), kUnitReaders);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -874,6 +946,7 @@ __global__ void __launch_bounds__(kPlanThreads)
   bucket[2 * tid] = excl;  // each thread rewrites only its own two buckets
   bucket[2 * tid + 1] = excl + c0;
   if (tid == kPlanThreads - 1) *count = excl + c0 + c1;
+  if (tid == 0) *p.vl_next = 0;  // the prefill kernel's CTAs claim units from it
   __syncthreads();
   // Each sequence takes a contiguous range of the list.
   for (int b = tid; b < B; b += kPlanThreads) {
