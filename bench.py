@@ -232,24 +232,63 @@ def make_call(w: Workload, q, k, v, o, lse, stream):
 
 
 def run_e2e(w: Workload, tensors, steps, warmup, ws, stream):
-    """The same call with pinned HOST inputs: per step, copy Q/K/V host->device, run,
-    copy O and LSE device->host; all inside the timed region."""
+    """The same call with pinned HOST inputs and results, pipelined as a serving loop runs
+    it: step i uploads its Q/K/V on one copy stream, runs fa_fwd on the launch stream once
+    they have landed, and downloads O and LSE on a second copy stream.  Two device buffer
+    sets let step i+1's upload and step i-1's download overlap step i's kernel (the upload
+    into a set waits for the kernel that last read it, the kernel for the download that
+    last read its outputs).  Every step's copies are inside the timed region: the clock
+    starts before step 0's upload and stops after the last step's download."""
     q, k, v, o, lse = tensors
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    call = make_call(w, q, k, v, o, lse, stream)
+    sets = [(q, k, v, o, lse), tuple(torch.empty_like(t) for t in (q, k, v, o, lse))]
+    calls = [make_call(w, *sets[j], stream) for j in (0, 1)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in (0, 1)]    # set j's inputs have landed
+    ev_done = [torch.cuda.Event() for _ in (0, 1)]  # the kernel on set j has finished
+    ev_out = [torch.cuda.Event() for _ in (0, 1)]   # set j's results are on the host
+    state = {"i": 0}
 
     def step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        call()
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
+        i = state["i"]
+        j = i % 2
+        sq, sk, sv, so, sl = sets[j]
+        if i >= 2:
+            up.wait_event(ev_done[j])
+        with torch.cuda.stream(up):
+            sq.copy_(hq, non_blocking=True)
+            sk.copy_(hk, non_blocking=True)
+            sv.copy_(hv, non_blocking=True)
+        ev_in[j].record(up)
+        stream.wait_event(ev_in[j])
+        if i >= 2:
+            stream.wait_event(ev_out[j])
+        calls[j]()
+        ev_done[j].record(stream)
+        down.wait_event(ev_done[j])
+        with torch.cuda.stream(down):
+            ho.copy_(so, non_blocking=True)
+            hl.copy_(sl, non_blocking=True)
+        ev_out[j].record(down)
+        state["i"] = i + 1
 
-    with torch.cuda.stream(stream):
-        ms = time_steps(step, steps, warmup, ws, stream)
+    torch.cuda.synchronize()
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(up)
+    for _ in range(steps):
+        step()
+    end.record(down)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = max_over_ranks(start.elapsed_time(end) / steps, ws)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
     return ms, h2d, d2h
@@ -559,7 +598,7 @@ def arm_ours(args, ws, rank, local):
         ms_e, h2d, d2h = run_e2e(wp, tensors, args.steps, args.warmup, ws, stream)
         e2e = {"value": r4(whole_job_rate(flops, ms_e, ws) / 1e12), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": r4(ms_e),
-               "steps": args.steps}
+               "steps": args.steps, "copies": "pipelined: 2 buffer sets, upload and download streams"}
     del tensors
 
     cpu = None
@@ -599,10 +638,10 @@ BWD_REV = "backward-v6"
 BWD_TRAFFIC = {("backward-v6", "long_prefill_causal"): 629.2e6}
 
 # Bumped whenever the prefill kernel changes, so stale ncu traffic is not reported.
-KERNEL_REV = "prefill-v22"
+KERNEL_REV = "prefill-v23"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the
 # kernel at this revision (profiles/fa_prefill_sm100_<workload>.md).
-DRAM_TRAFFIC = {("prefill-v22", "long_prefill_causal"): 587.2e6}
+DRAM_TRAFFIC = {("prefill-v23", "long_prefill_causal"): 600.4e6}
 # The decode kernel's traffic per launch, taken on decode_4k (B16 H32 Nkv4096: 1.0816 GB)
 # and scaled by the keys streamed (x8 for Nkv 32768): the kernel reads each key once.
 DECODE_REV = "decode-v1"
