@@ -141,3 +141,27 @@ def test_varlen_claimed_units_repeat_bitwise():
                            for b, n in enumerate(lq)])
     o_ref, l_ref = oracle.varlen_attention(q, k, v, cq.tolist(), ck.tolist(), 0.088, True)
     compare(outs[0][0][rows], outs[0][1][rows], o_ref[rows], l_ref[rows])
+
+
+def test_varlen_benchmark_batch_sampled():
+    """The benchmark's packed batch in the benchmark's launch configuration: 16 sequences
+    of seeded log-uniform lengths in [512, 8192], H = 32, d = 128, bf16 in and out,
+    causal, the inputs bench.py times.  Checked against the oracle on the first and last
+    query token of every sequence, the tokens on both sides of its first Q-tile boundary
+    and 16 random tokens."""
+    from exact_io_aware_59_b200.inputs import varlen_inputs, varlen_lengths
+
+    lens = varlen_lengths(16, 512, 8192, 4242)
+    H, d, scale = 32, 128, 128 ** -0.5
+    q, k, v, cu = varlen_inputs(lens, H, d, torch.bfloat16, 8000, device="cuda")
+    o, lse = _run(q, k, v, cu, cu, lens, lens, True, scale, out_dtype=torch.bfloat16)
+    rng = np.random.default_rng(4242)
+    for b, n in enumerate(lens):
+        c0 = int(cu[b])
+        picks = sorted({0, n - 1, 127, 128} | set(rng.integers(0, n, size=16).tolist()))
+        for t in picks:
+            L = t + 1  # causal: token t sees keys 0..t of its sequence
+            o_ref, l_ref = oracle.varlen_attention(
+                q[c0 + t: c0 + t + 1].cpu(), k[c0: c0 + L].cpu(), v[c0: c0 + L].cpu(), [0, 1],
+                [0, L], scale, False)
+            compare(o[c0 + t], lse[c0 + t], o_ref[0], l_ref[0], rel_o=REL_O16[torch.bfloat16])
