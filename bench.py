@@ -644,7 +644,7 @@ KERNEL_REV = "prefill-v23"
 DRAM_TRAFFIC = {("prefill-v23", "long_prefill_causal"): 600.4e6}
 # The decode kernel's traffic per launch, taken on decode_4k (B16 H32 Nkv4096: 1.0816 GB)
 # and scaled by the keys streamed (x8 for Nkv 32768): the kernel reads each key once.
-DECODE_REV = "decode-v1"
+DECODE_REV = "decode-v2"
 DECODE_TRAFFIC = {("decode-v1", "decode"): 8 * 1.0816e9}
 
 

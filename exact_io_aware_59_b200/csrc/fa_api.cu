@@ -228,7 +228,7 @@ fa::DecodeParams decode_params(int B, int H, int Nkv, float scale, int num_split
 }
 
 size_t decode_ws_bytes(const fa::DecodeParams& p, int d) {
-  const size_t recs = static_cast<size_t>(p.grid) * p.max_seg * 8;  // 8 consumer warps
+  const size_t recs = static_cast<size_t>(p.grid) * p.max_seg * fa::kDecodeRecords;
   return recs * (d + 1) * sizeof(float);
 }
 
@@ -472,7 +472,7 @@ int run_decode(const void* q, const void* k, const void* v, void* o, float* lse,
   void* ws = nullptr;
   if ((rc = workspace_alloc(ds, decode_ws_bytes(p, d), st, &ws)) != FA_OK) return rc;
   float* part_o = static_cast<float*>(ws);
-  float* part_lse = part_o + static_cast<size_t>(p.grid) * p.max_seg * 8 * d;
+  float* part_lse = part_o + static_cast<size_t>(p.grid) * p.max_seg * fa::kDecodeRecords * d;
   cudaError_t e = fa::launch_decode(q, k, v, o, lse, p, d, in_dtype == FA_BF16, o_dtype == FA_F32,
                                     part_o, part_lse, ds->status, st, paged);
   const cudaError_t ef = cudaFreeAsync(ws, st);

@@ -32,10 +32,17 @@
 namespace fa {
 namespace {
 
-constexpr int kWarps = 8;                     // consumer warps
+// Consumer warps: two groups of eight.  Stage i of the ring (the i-th chunk with keys) goes
+// to group i % 2, whose warps take 8 keys each.  A warp's work on a chunk is a chain of
+// dependent steps (shared-memory loads, a shuffle butterfly, the softmax update, P V), so
+// two groups working on consecutive chunks at once keep the ring draining at the rate the
+// copies arrive; with one group of eight the ring stayed full and the copies waited.
+constexpr int kGroupWarps = 8;
+constexpr int kWarps = 2 * kGroupWarps;       // consumer warps
 constexpr int kThreads = (kWarps + 1) * 32;   // + one producer warp
-constexpr int kKeysPerWarp = kDecodeChunk / kWarps;
+constexpr int kKeysPerWarp = kDecodeChunk / kGroupWarps;
 static_assert(kKeysPerWarp == 8, "the butterfly below reduces 8 keys per warp");
+static_assert(kWarps == kDecodeRecords, "one partial record per consumer warp");
 
 template <int D>
 struct DecodeCfg {
@@ -114,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(bars + 8 * s, 1);             // full: producer's expect_tx + bytes
-      mbar_init(bars + 8 * (S + s), kWarps);  // empty: one arrival per consumer warp
+      mbar_init(bars + 8 * (S + s), kGroupWarps);  // empty: one arrival per warp of its group
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -234,12 +241,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ consumers
     const long long first_head = c_begin / p.n_chunks;
+    const int group = warp / kGroupWarps;  // takes the stages i with i % 2 == group
+    const int slice = warp % kGroupWarps;  // keys 8 * slice .. 8 * slice + 7 of a chunk
     // Key (0..7 within this warp's 8) whose full dot product this lane ends up holding.
     const int my_key = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
 
     float qv[E], acc[E];
     float m = -INFINITY, l_lane = 0.f;
     int cur_h = -1;
+    int len = p.Nkv;  // keys of the current head's sequence
     uint32_t ld = 0;
     bool ok = true;
 
@@ -259,11 +269,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     for (long long c = c_begin; c < c_end; ++c) {
-      int h, key0, nk;
-      chunk_info<PAGED>(p, pk, c, h, key0, nk, status, false);
+      const int h = static_cast<int>(c / p.n_chunks);
+      const int key0 = static_cast<int>(c % p.n_chunks) * kDecodeChunk;
       if (h != cur_h) {
         if (cur_h >= 0) finish_segment(cur_h);
         cur_h = h;
+        if constexpr (PAGED) {
+          // The sequence's length, clamped as the producer clamps it (the producer reports
+          // a bad length); read once per head rather than once per chunk.
+          const int cap = pk.max_pages << pk.page_shift;
+          len = pk.seq_lens[h / pk.H];
+          len = len < 0 ? 0 : (len > cap ? cap : len);
+        }
         float qf[E];
         load_slice<D, BF16>(reinterpret_cast<const uint8_t*>(q + static_cast<size_t>(h) * D), lane, qf);
 #pragma unroll
@@ -274,17 +291,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = -INFINITY;
         l_lane = 0.f;
       }
+      const int nk = min(kDecodeChunk, len - key0);
       // An empty slot still opens its head (so every segment gets its records), but has
       // no stage to read.
       if (nk <= 0) continue;
       const uint32_t slot = ld % S;
-      const bool got = mbar_wait(bars + 8 * slot, (ld / S) & 1, status, abort_flag,
+      const uint32_t phase = (ld / S) & 1;
+      const bool mine = (ld & 1) == static_cast<uint32_t>(group);
+      ++ld;
+      if (!mine) continue;  // the other group's stage
+      const bool got = mbar_wait(bars + 8 * slot, phase, status, abort_flag,
                                  kStatusTimeoutDecode);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
-      const uint8_t* ks = smem + slot * C::kStageBytes + warp * kKeysPerWarp * D * 2;
+      const uint8_t* ks = smem + slot * C::kStageBytes + slice * kKeysPerWarp * D * 2;
       const uint8_t* vs = ks + C::kChunkBytes;
 
       // Partial dot products of this lane's d-slice with the warp's 8 keys.
@@ -321,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       part[0] += __shfl_xor_sync(0xffffffffu, part[0], 2);
       part[0] += __shfl_xor_sync(0xffffffffu, part[0], 1);
-      const int nvalid = nk - warp * kKeysPerWarp;  // keys of this warp inside the chunk
+      const int nvalid = nk - slice * kKeysPerWarp;  // keys of this warp inside the chunk
       const float x = (my_key < nvalid) ? part[0] : -INFINITY;
 
       // Online softmax over the warp's keys (eager: one exp2 for alpha per chunk).
@@ -349,7 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + 8 * (S + slot));
-      ++ld;
     }
     if (ok && cur_h >= 0) finish_segment(cur_h);
   }

@@ -81,6 +81,8 @@ struct DecodeParams {
 };
 
 constexpr int kDecodeChunk = 64;
+// Partial records the split decode writes per CTA and head segment: one per consumer warp.
+constexpr int kDecodeRecords = 16;
 
 // Paged KV cache of a decode launch (null block_table: contiguous [B,H,Nkv,d] K/V).
 struct PagedKV {

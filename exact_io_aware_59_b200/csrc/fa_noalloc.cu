@@ -69,7 +69,7 @@ extern "C" int fa_fwd_decode_noalloc(const void* q, const void* k, const void* v
   // split kernel of the same call, unless a split kernel's wait runs out, which the status
   // word reports (fa_device_status); the outputs of such a call are undefined.
   float* part_o = reinterpret_cast<float*>(base);
-  float* part_lse = part_o + static_cast<size_t>(p.grid) * p.max_seg * 8 * d;
+  float* part_lse = part_o + static_cast<size_t>(p.grid) * p.max_seg * fa::kDecodeRecords * d;
   const cudaError_t e = fa::launch_decode(q, k, v, o, lse, p, d, in_dtype == FA_BF16,
                                           o_dtype == FA_F32, part_o, part_lse, status,
                                           static_cast<cudaStream_t>(stream));

@@ -158,11 +158,11 @@ int fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* l
  *   and results as fa_fwd_decode, with the split partials kept in one fixed static device
  *   array of FA_NOALLOC_SCRATCH_BYTES bytes.  The caller still passes q, k, v, o and lse.
  *   No cudaMalloc, cudaFree or other allocating routine is called.
- *   Limit: a call whose partials need more than the array (G * max_seg * 8 * (d+1) * 4
+ *   Limit: a call whose partials need more than the array (G * max_seg * 16 * (d+1) * 4
  *   bytes, the figure fa_decode_workspace_bytes returns) is refused with
  *   FA_ERR_UNSUPPORTED before anything is enqueued.  With the default split count (one
- *   CTA per SM, 148 on B200) that holds for B*H up to about 1,700 heads at d = 128 and
- *   3,800 at d = 64, for any Nkv (B=16, H=32, d=128 needs 3.1 MB).
+ *   CTA per SM, 148 on B200) that holds for B*H up to 740 heads at d = 128 and 1,776 at
+ *   d = 64, for any Nkv (B=16, H=32, d=128 needs 6.1 MB).
  *   First call: the first call on each device (made with that device current) looks up
  *   the array's device address.  Under CUDA's default lazy module loading that lookup is
  *   what loads the array's module, so it is the moment the 8 MiB are committed on that

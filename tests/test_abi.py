@@ -117,13 +117,13 @@ def test_prefill_split_choice_is_host_arithmetic():
 
 
 def test_decode_workspace_size_formula():
-    # 8 partial records (one per consumer warp) per CTA per head segment, d+1 floats each.
+    # 16 partial records (one per consumer warp) per CTA per head segment, d+1 floats each.
     B, H, Nkv, d, G = 16, 32, 32768, 128, 148
     chunks = B * H * ((Nkv + 63) // 64)
     per_cta = -(-chunks // G)
     max_seg = -(-per_cta // ((Nkv + 63) // 64)) + 1
-    assert binding.fa_decode_workspace_bytes(B, H, Nkv, d, G) == G * max_seg * 8 * (d + 1) * 4
-    assert binding.fa_decode_workspace_bytes(1, 1, 10, 64, 5) == 1 * 2 * 8 * 65 * 4
+    assert binding.fa_decode_workspace_bytes(B, H, Nkv, d, G) == G * max_seg * 16 * (d + 1) * 4
+    assert binding.fa_decode_workspace_bytes(1, 1, 10, 64, 5) == 1 * 2 * 16 * 65 * 4
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
