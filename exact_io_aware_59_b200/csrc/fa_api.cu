@@ -794,9 +794,8 @@ int fa_fwd_fp8_quant(const void* q, const void* k, const void* v, void* o, float
   float* qs = reinterpret_cast<float*>(w + qb + kb);
   float* ks = reinterpret_cast<float*>(w + qb + kb + qsb);
   const bool bf16 = in_dtype == FA_BF16;
-  cudaError_t e = fa::launch_quantize_e4m3(q, bf16, static_cast<long long>(BH), Nq, q8, qs, st);
-  if (e == cudaSuccess)
-    e = fa::launch_quantize_e4m3(k, bf16, static_cast<long long>(BH), Nkv, k8, ks, st);
+  cudaError_t e = fa::launch_quantize_e4m3_qk(q, Nq, q8, qs, k, Nkv, k8, ks, bf16,
+                                              static_cast<long long>(BH), st);
   CUtensorMap tq, tk, tv;
   if (e == cudaSuccess) {
     if ((rc = make_map_u8(&tq, q8, Nq, static_cast<long long>(BH), d)) != FA_OK ||

@@ -118,6 +118,10 @@ size_t backward_smem_bytes(int d);
 // (fa_quant.cu): codes [BH, N, 128] bytes, scales [BH, ceil(N / 128)] fp32.
 cudaError_t launch_quantize_e4m3(const void* x, bool bf16, long long BH, int N, void* codes,
                                  float* scales, cudaStream_t stream);
+// Q and K of one call in a single launch (each [BH, N, 128], one scale per 128-row tile).
+cudaError_t launch_quantize_e4m3_qk(const void* q, int Nq, void* q8, float* qs, const void* k,
+                                    int Nkv, void* k8, float* ks, bool bf16, long long BH,
+                                    cudaStream_t stream);
 
 // Diagnostic kernel whose only wait can never finish (see fa_selftest_wait_timeout).
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t stream);

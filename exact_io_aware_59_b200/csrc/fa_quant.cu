@@ -33,13 +33,30 @@ __device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
   return r;
 }
 
+// One tensor to quantise: [BH, N, 128] 16-bit values in, codes and one scale per tile out.
+struct QuantJob {
+  const uint4* x;
+  uint2* codes;
+  float* scales;
+  int N, n_tiles;
+  long long blocks;  // BH * n_tiles: one CTA per tile
+};
+
+// Blocks [0, a.blocks) quantise tensor a, the rest tensor b (b.blocks = 0: none), so that
+// Q and K of one call take a single launch.
 template <bool BF16>
 __global__ void __launch_bounds__(kQuantThreads)
-    fa_quantize_e4m3_tiles(const uint4* __restrict__ x, int N, int n_tiles,
-                           uint2* __restrict__ codes, float* __restrict__ scales) {
+    fa_quantize_e4m3_tiles(const QuantJob a, const QuantJob b) {
   __shared__ float warp_max[kQuantThreads / 32];
-  const long long bh = blockIdx.x / n_tiles;
-  const int tile = blockIdx.x - static_cast<int>(bh * n_tiles);
+  const bool second = blockIdx.x >= a.blocks;
+  const long long blk = second ? blockIdx.x - a.blocks : blockIdx.x;
+  const uint4* __restrict__ x = second ? b.x : a.x;
+  uint2* __restrict__ codes = second ? b.codes : a.codes;
+  float* __restrict__ scales = second ? b.scales : a.scales;
+  const int N = second ? b.N : a.N;
+  const int n_tiles = second ? b.n_tiles : a.n_tiles;
+  const long long bh = blk / n_tiles;
+  const int tile = static_cast<int>(blk - bh * n_tiles);
   const int rows = min(kTileRows, N - tile * kTileRows);
   const size_t base = (static_cast<size_t>(bh) * N + static_cast<size_t>(tile) * kTileRows) * (kD / 8);
   uint4 raw[kChunksPerThread];
@@ -66,7 +83,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 #pragma unroll
   for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, warp_max[w]);
   const float scale = amax > 0.f ? amax / 448.0f : 1.0f;
-  if (threadIdx.x == 0) scales[blockIdx.x] = scale;
+  if (threadIdx.x == 0) scales[blk] = scale;
 #pragma unroll
   for (int i = 0; i < kChunksPerThread; ++i) {
     const int c = threadIdx.x + kQuantThreads * i;
@@ -85,20 +102,39 @@ __global__ void __launch_bounds__(kQuantThreads)
   }
 }
 
+QuantJob make_job(const void* x, long long BH, int N, void* codes, float* scales) {
+  QuantJob j;
+  j.x = static_cast<const uint4*>(x);
+  j.codes = static_cast<uint2*>(codes);
+  j.scales = scales;
+  j.N = N;
+  j.n_tiles = (N + kTileRows - 1) / kTileRows;
+  j.blocks = BH * j.n_tiles;
+  return j;
+}
+
+cudaError_t launch_jobs(const QuantJob& a, const QuantJob& b, bool bf16, cudaStream_t stream) {
+  const long long blocks = a.blocks + b.blocks;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  if (bf16)
+    fa_quantize_e4m3_tiles<true><<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(a, b);
+  else
+    fa_quantize_e4m3_tiles<false><<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(a, b);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_quantize_e4m3(const void* x, bool bf16, long long BH, int N, void* codes,
                                  float* scales, cudaStream_t stream) {
-  const int n_tiles = (N + kTileRows - 1) / kTileRows;
-  const long long blocks = BH * n_tiles;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  if (bf16)
-    fa_quantize_e4m3_tiles<true><<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), N, n_tiles, static_cast<uint2*>(codes), scales);
-  else
-    fa_quantize_e4m3_tiles<false><<<static_cast<int>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4*>(x), N, n_tiles, static_cast<uint2*>(codes), scales);
-  return cudaGetLastError();
+  QuantJob none = make_job(x, 0, N, codes, scales);
+  return launch_jobs(make_job(x, BH, N, codes, scales), none, bf16, stream);
+}
+
+cudaError_t launch_quantize_e4m3_qk(const void* q, int Nq, void* q8, float* qs, const void* k,
+                                    int Nkv, void* k8, float* ks, bool bf16, long long BH,
+                                    cudaStream_t stream) {
+  return launch_jobs(make_job(q, BH, Nq, q8, qs), make_job(k, BH, Nkv, k8, ks), bf16, stream);
 }
 
 }  // namespace fa
