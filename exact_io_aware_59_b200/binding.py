@@ -55,6 +55,9 @@ _SIGNATURES = {
     "fa_bwd": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _I, _I, _I, _I,
                _I, _F, _I, _VP, _I],
     "fa_bwd_workspace_bytes": [_I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
+    "fa_bwd_varlen": [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP, _VP,
+                      _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _I],
+    "fa_bwd_varlen_workspace_bytes": [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
     "fa_decode_workspace_bytes": [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_size_t)],
     "fa_device_status": [ctypes.POINTER(_I), _I],
     "fa_selftest_wait_timeout": [_VP],
@@ -215,6 +218,22 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, 
            scale, causal, stream, in_dtype) -> int:
     return library().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H,
                             Nq, Nkv, d, scale, causal, stream, in_dtype)
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, cu_seqlens_q,
+                  cu_seqlens_k, B, H, total_q, total_k, max_seqlen_q, max_seqlen_k, d, scale,
+                  causal, stream, in_dtype) -> int:
+    return library().fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                                   cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k,
+                                   max_seqlen_q, max_seqlen_k, d, scale, causal, stream, in_dtype)
+
+
+def fa_bwd_varlen_workspace_bytes(B, H, total_q, max_seqlen_k, d) -> int:
+    out = ctypes.c_size_t(0)
+    rc = library().fa_bwd_varlen_workspace_bytes(B, H, total_q, max_seqlen_k, d, ctypes.byref(out))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_varlen_workspace_bytes")
+    return int(out.value)
 
 
 def fa_bwd_workspace_bytes(B, H, Nq, d) -> int:
@@ -462,4 +481,49 @@ def attention_backward(q, k, v, o, lse, dout, causal: bool = False, scale: Optio
                     Nkv, d, scale, int(bool(causal)), s.cuda_stream, _dtype_code(q.dtype))
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def varlen_attention_backward(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k,
+                              max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,
+                              scale: Optional[float] = None, workspace=None, stream=None):
+    """dQ, dK, dV of varlen_attention() for the upstream gradient dout.  q, o, dout
+    [total_q, H, d], k, v [total_k, H, d] (d 64 or 128) contiguous CUDA tensors of one 16-bit
+    dtype, lse fp32 [total_q, H] (the forward's), cu_seqlens int32 CUDA [B+1].  workspace:
+    optional uint8 CUDA tensor of at least fa_bwd_varlen_workspace_bytes; allocated when
+    omitted.  Returns (dq, dk, dv) in the inputs' dtype; rows of tokens outside every
+    sequence are left as torch.zeros_like gives them."""
+    import torch
+
+    ts = (q, k, v, o, dout)
+    if not all(t.is_cuda and t.is_contiguous() for t in ts) or not (lse.is_cuda and lse.is_contiguous()):
+        raise ValueError("varlen_attention_backward() takes contiguous CUDA tensors")
+    if any(t.dtype != q.dtype for t in ts) or q.dtype not in (torch.float16, torch.bfloat16):
+        raise ValueError("q, k, v, o and dout must share one dtype, float16 or bfloat16")
+    if lse.dtype != torch.float32 or cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise ValueError("lse must be float32 and cu_seqlens int32")
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    B = cu_seqlens_q.numel() - 1
+    if (tuple(k.shape) != (total_k, H, d) or tuple(v.shape) != (total_k, H, d)
+            or tuple(o.shape) != (total_q, H, d) or tuple(dout.shape) != (total_q, H, d)
+            or tuple(lse.shape) != (total_q, H) or cu_seqlens_k.numel() != B + 1):
+        raise ValueError("shapes must be q/o/dout [total_q,H,d], k/v [total_k,H,d], lse [total_q,H]")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    nbytes = fa_bwd_varlen_workspace_bytes(B, H, total_q, max_seqlen_k, d)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    dq = torch.zeros_like(q)
+    dk = torch.zeros_like(k)
+    dv = torch.zeros_like(v)
+    s = torch.cuda.current_stream(q.device) if stream is None else stream
+    with torch.cuda.device(q.device):
+        rc = fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                           cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q,
+                           total_k, max_seqlen_q, max_seqlen_k, d, scale, int(bool(causal)),
+                           s.cuda_stream, _dtype_code(q.dtype))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_varlen")
     return dq, dk, dv

@@ -692,6 +692,30 @@ size_t bwd_ws_bytes(size_t BH, int Nq, int d) {
   return BH * nq_pad * (4 + 4 + static_cast<size_t>(d) * 4);
 }
 
+// Packed backward workspace: per head, rows_max rows (total_q + 128 * B rounded up to a
+// multiple of 128: every sequence's query rows padded to whole 128-row tiles fit, and every
+// head's rows, hence every tile's 512 bytes of -LSE*log2(e) and D that the main kernel
+// bulk-copies, start on a 16-byte boundary) of -LSE*log2(e), D and the fp32 dQ accumulator;
+// then the plan: item count (16 bytes), B sequence records, B + 1 padded row offsets
+// (rounded up to 16 bytes), B * n_ktiles items.
+struct VarlenBwdLayout {
+  long long rows_max;
+  size_t rows_bytes, plan_off, seqs_off, qpad_off, items_off, total;
+};
+
+VarlenBwdLayout varlen_bwd_layout(int B, int H, int total_q, int max_k, int d) {
+  VarlenBwdLayout l;
+  l.rows_max = (static_cast<long long>(total_q) + 128LL * B + 127) / 128 * 128;
+  l.rows_bytes = static_cast<size_t>(H) * l.rows_max * (4 + 4 + static_cast<size_t>(d) * 4);
+  const size_t n_ktiles = (static_cast<size_t>(max_k) + 127) / 128;
+  l.plan_off = l.rows_bytes;
+  l.seqs_off = l.plan_off + 16;
+  l.qpad_off = l.seqs_off + static_cast<size_t>(B) * 16;
+  l.items_off = l.qpad_off + (static_cast<size_t>(B + 1) * 4 + 15) / 16 * 16;
+  l.total = l.items_off + static_cast<size_t>(B) * n_ktiles * 4;
+  return l;
+}
+
 }  // namespace
 
 int fa_bwd_workspace_bytes(int B, int H, int Nq, int d, size_t* bytes) {
@@ -763,6 +787,97 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   p.dq_acc = w + 2 * BH * p.nq_pad;
   p.dk = dk;
   p.dv = dv;
+  cudaError_t e = fa::launch_backward(tq, tk, tv, tdo, o, dout, lse, dq, p, d, bf16,
+                                      ds->sm_count, ds->status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : cuda_fail(e);
+}
+
+int fa_bwd_varlen_workspace_bytes(int B, int H, int total_q, int max_seqlen_k, int d,
+                                  size_t* bytes) {
+  if (!bytes || B < 1 || H < 1 || total_q < 1 || max_seqlen_k < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  *bytes = varlen_bwd_layout(B, H, total_q, max_seqlen_k, d).total;
+  return FA_OK;
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                  size_t workspace_bytes, const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+                  int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                  float scale, int causal, void* stream, int in_dtype) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace ||
+      !cu_seqlens_q || !cu_seqlens_k)
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || total_q < 1 || total_k < 1 || max_seqlen_q < 1 || max_seqlen_k < 1)
+    return FA_ERR_INVALID_ARG;
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (in_dtype != FA_F16 && in_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const void* a16[9] = {q, k, v, o, dout, dq, dk, dv, workspace};
+  for (const void* ptr : a16)
+    if (!aligned(ptr, 16)) return FA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
+    return FA_ERR_INVALID_ARG;
+  const VarlenBwdLayout lay = varlen_bwd_layout(B, H, total_q, max_seqlen_k, d);
+  if (lay.rows_max > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < lay.total) return FA_ERR_INVALID_ARG;
+  const long long n_ktiles = (max_seqlen_k + 127) / 128;
+  if (static_cast<long long>(B) * n_ktiles * H > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  const size_t qb = static_cast<size_t>(total_q) * H * d * 2;
+  const size_t kb = static_cast<size_t>(total_k) * H * d * 2;
+  const size_t lb = static_cast<size_t>(total_q) * H * 4, cb = static_cast<size_t>(B + 1) * 4;
+  const void* outs[4] = {dq, dk, dv, workspace};
+  const size_t out_bytes[4] = {qb, kb, kb, lay.total};
+  const void* ins[8] = {q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k};
+  const size_t in_bytes[8] = {qb, kb, kb, qb, qb, lb, cb, cb};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 8; ++j)
+      if (overlaps(outs[i], out_bytes[i], ins[j], in_bytes[j])) return FA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlaps(outs[i], out_bytes[i], outs[j], out_bytes[j])) return FA_ERR_INVALID_ARG;
+  }
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != FA_OK) return rc;
+  if ((rc = get_encoder()) != FA_OK) return rc;
+  const bool bf16 = in_dtype == FA_BF16;
+  CUtensorMap tq, tk, tv, tdo;
+  if ((rc = make_map_packed(&tq, q, total_q, H, d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map_packed(&tdo, dout, total_q, H, d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map_packed(&tk, k, total_k, H, d, bf16)) != FA_OK) return rc;
+  if ((rc = make_map_packed(&tv, v, total_k, H, d, bf16)) != FA_OK) return rc;
+  fa::BwdParams p{};
+  p.BH = B * H;
+  p.Nq = max_seqlen_q;
+  p.Nkv = max_seqlen_k;
+  p.off = 0;  // per sequence in the kernels
+  p.causal = causal;
+  p.n_qtiles = (max_seqlen_q + 127) / 128;
+  p.nq_pad = p.n_qtiles * 128;
+  p.n_ktiles = static_cast<int>(n_ktiles);
+  p.scale = scale;
+  p.scale_log2 = scale_log2(scale);
+  float* w = static_cast<float*>(workspace);
+  const size_t hr = static_cast<size_t>(H) * lay.rows_max;
+  p.nlse2 = w;
+  p.delta = w + hr;
+  p.dq_acc = w + 2 * hr;
+  p.dk = dk;
+  p.dv = dv;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.B = B;
+  p.H = H;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.rows_max = lay.rows_max;
+  char* base = static_cast<char*>(workspace);
+  p.vl_count = reinterpret_cast<int*>(base + lay.plan_off);
+  p.vl_seqs = reinterpret_cast<int4*>(base + lay.seqs_off);
+  p.vl_qpad = reinterpret_cast<int*>(base + lay.qpad_off);
+  p.vl_items = reinterpret_cast<int*>(base + lay.items_off);
   cudaError_t e = fa::launch_backward(tq, tk, tv, tdo, o, dout, lse, dq, p, d, bf16,
                                       ds->sm_count, ds->status, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : cuda_fail(e);

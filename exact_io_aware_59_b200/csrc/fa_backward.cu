@@ -143,19 +143,39 @@ __device__ __forceinline__ uint64_t kmajor_step(int kk, int rows) {
   return static_cast<uint64_t>(((kk >> 2) * rows * 128 + (kk & 3) * 32) >> 4);
 }
 
+// Where one CTA's data lives.  [B,H,N,d] layout: tiles at (d column, row, b*h) of the 3-D
+// tensor maps, head bh's workspace rows from bh * nq_pad, dK/dV row (bh * Nkv + key).
+// Packed layout (VARLEN): tiles at (d column, h, token) of the (d, H, tokens) maps, the
+// sequence's first query / key token q_tok0 / k_tok0, workspace rows from wrow0 (head h's
+// rows, then the sequence's padded offset), dK/dV row (k_tok0 + key) * H + h.
+struct BwdCta {
+  int bh;            // b * H + h ([B,H,N,d]); h (packed)
+  int q_tok0, k_tok0;
+  long long wrow0;   // first workspace row of this CTA's query rows
+};
+
+template <bool VARLEN>
+__device__ __forceinline__ void tile_load(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                          int col, int row, int tok0, int bh) {
+  if constexpr (VARLEN)
+    tma_load_3d(dst, map, bar, col, bh, tok0 + row);
+  else
+    tma_load_3d(dst, map, bar, col, row, bh);
+}
+
 // ---------------------------------------------------------------- producer (TMA)
-template <int D>
+template <int D, bool VARLEN>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
-                         const CUtensorMap* tdo, const BwdParams& p, int bh, int k0, int i0,
-                         int n, uint32_t sbase, uint32_t bars, int* status,
+                         const CUtensorMap* tdo, const BwdParams& p, const BwdCta& cta, int k0,
+                         int i0, int n, uint32_t sbase, uint32_t bars, int* status,
                          volatile int* abort_flag) {
   using C = BwdCfg<D>;
   const uint32_t kv = bar_addr(bars, C::kBarKV);
   mbar_arrive_expect_tx(kv, 2 * C::kTileBytes);
 #pragma unroll
   for (int sub = 0; sub < D / 64; ++sub) {
-    tma_load_3d(sbase + C::kKOff + sub * kBK * 128, tk, kv, sub * 64, k0, bh);
-    tma_load_3d(sbase + C::kVOff + sub * kBK * 128, tv, kv, sub * 64, k0, bh);
+    tile_load<VARLEN>(sbase + C::kKOff + sub * kBK * 128, tk, kv, sub * 64, k0, cta.k_tok0, cta.bh);
+    tile_load<VARLEN>(sbase + C::kVOff + sub * kBK * 128, tv, kv, sub * 64, k0, cta.k_tok0, cta.bh);
   }
   int q_issued = 0, do_issued = 0;
   bool ok = true;
@@ -173,8 +193,9 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     mbar_arrive_expect_tx(qf, C::kTileBytes + 2 * kBQ * 4);
 #pragma unroll
     for (int sub = 0; sub < D / 64; ++sub)
-      tma_load_3d(sbase + C::kQOff + st * C::kTileBytes + sub * kBQ * 128, tq, qf, sub * 64, q0, bh);
-    const size_t row = static_cast<size_t>(bh) * p.nq_pad + q0;
+      tile_load<VARLEN>(sbase + C::kQOff + st * C::kTileBytes + sub * kBQ * 128, tq, qf, sub * 64,
+                        q0, cta.q_tok0, cta.bh);
+    const size_t row = static_cast<size_t>(cta.wrow0) + q0;
     bulk_load(sbase + C::kLseOff + st * kBQ * 4, p.nlse2 + row, kBQ * 4, qf);
     bulk_load(sbase + C::kDelOff + st * kBQ * 4, p.delta + row, kBQ * 4, qf);
     ++q_issued;
@@ -184,7 +205,8 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     mbar_arrive_expect_tx(df, C::kTileBytes);
 #pragma unroll
     for (int sub = 0; sub < D / 64; ++sub)
-      tma_load_3d(sbase + C::kdOOff + sub * kBQ * 128, tdo, df, sub * 64, q0, bh);
+      tile_load<VARLEN>(sbase + C::kdOOff + sub * kBQ * 128, tdo, df, sub * 64, q0, cta.q_tok0,
+                        cta.bh);
     ++do_issued;
   }
   if (!ok) {
@@ -297,8 +319,8 @@ __device__ void mma_issuer(int n, uint32_t sbase, uint32_t bars, uint32_t tmem, 
 
 // ---------------------------------------------------------------- P and dS (one thread per key)
 // Warpgroup `wg` (0 or 1) takes queries 64 wg .. 64 wg + 63 of every query tile.
-template <int D, bool BF16>
-__device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, int wg,
+template <int D, bool BF16, bool VARLEN>
+__device__ void softmax_grad(const BwdParams& p, const BwdCta& cta, int k0, int i0, int n, int wg,
                              uint8_t* sgen, uint32_t bars, uint32_t tmem, int* status,
                              volatile int* abort_flag) {
   using C = BwdCfg<D>;
@@ -403,7 +425,8 @@ __device__ void softmax_grad(const BwdParams& p, int bh, int k0, int i0, int n, 
   if (have) have = ok && wait(C::kBarDone, 0);
   if (n > 0 && !have) return;
   if (have) tc_fence_after();
-  const size_t orow = (static_cast<size_t>(bh) * p.Nkv + kidx) * D;
+  const size_t orow = VARLEN ? ((static_cast<size_t>(cta.k_tok0) + kidx) * p.H + cta.bh) * D
+                            : (static_cast<size_t>(cta.bh) * p.Nkv + kidx) * D;
   {
     const int which = wg;  // warpgroup 1 writes dV, warpgroup 2 writes dK
     uint16_t* dst = static_cast<uint16_t*>(which ? p.dk : p.dv) + orow;
@@ -441,7 +464,7 @@ __device__ __forceinline__ void red_add_f32(float* addr, float v) {
 }
 
 template <int D>
-__device__ void dq_drain(const BwdParams& p, int bh, int i0, int n, uint32_t bars, uint32_t tmem,
+__device__ void dq_drain(const BwdParams& p, const BwdCta& cta, int i0, int n, uint32_t bars, uint32_t tmem,
                          int* status, volatile int* abort_flag) {
   using C = BwdCfg<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -473,7 +496,7 @@ __device__ void dq_drain(const BwdParams& p, int bh, int i0, int n, uint32_t bar
     if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarDQEmpty));  // dP(i+1) may overwrite it
     // Accumulator row q (query q0 + q) is D contiguous floats: a warp adds 32 consecutive
     // ones per instruction.
-    float* row = p.dq_acc + (static_cast<size_t>(bh) * p.nq_pad + static_cast<size_t>(i0 + i) * kBQ) * D + t;
+    float* row = p.dq_acc + (static_cast<size_t>(cta.wrow0) + static_cast<size_t>(i0 + i) * kBQ) * D + t;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -484,11 +507,11 @@ __device__ void dq_drain(const BwdParams& p, int bh, int i0, int n, uint32_t bar
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_sm100(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                 const BwdParams p, int* __restrict__ status) {
+                 const BwdParams p_in, int* __restrict__ status) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -498,10 +521,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + C::kAbortOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sgen + C::kTmemHolderOff);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Head by head, so the CTAs resident together share one head's Q, dO and dQ
+  // [B,H,N,d]: head by head, so the CTAs resident together share one head's Q, dO and dQ
   // accumulator in L2; within a head the heaviest first (key tile 0 meets the most causal
-  // query tiles).
-  const int bh = blockIdx.x / p.n_ktiles, kt = blockIdx.x % p.n_ktiles;
+  // query tiles).  Packed: item it = blockIdx.x / H of the plan's list (sequence by
+  // sequence, each sequence's key tiles heaviest first), head blockIdx.x % H; the launch
+  // covers the most items there can be, so CTAs past the plan's count return at once.
+  BwdParams p = p_in;
+  BwdCta cta;
+  int kt;
+  if constexpr (!VARLEN) {
+    cta.bh = blockIdx.x / p.n_ktiles;
+    kt = blockIdx.x % p.n_ktiles;
+    cta.q_tok0 = cta.k_tok0 = 0;
+    cta.wrow0 = static_cast<long long>(cta.bh) * p.nq_pad;
+  } else {
+    const int it = blockIdx.x / p.H;
+    if (it >= *p.vl_count) return;  // the whole CTA, before any barrier or TMEM use
+    cta.bh = blockIdx.x - it * p.H;
+    const int item = p.vl_items[it];
+    const int b = item / p.n_ktiles;
+    kt = item - b * p.n_ktiles;
+    const int4 sq = p.vl_seqs[b];  // bounds-checked by the plan kernel
+    cta.q_tok0 = sq.x;
+    cta.k_tok0 = sq.z;
+    p.Nq = sq.y;
+    p.Nkv = sq.w;
+    p.off = sq.w - sq.y;  // causal alignment bottom-right per sequence
+    p.n_qtiles = (sq.y + kBQ - 1) / kBQ;
+    cta.wrow0 = static_cast<long long>(cta.bh) * p.rows_max + p.vl_qpad[b];
+  }
   const int k0 = kt * kBK;
   const int i0 = first_qtile(p, k0);
   const int n = p.n_qtiles - i0;
@@ -551,7 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
     if (warp == 0) {
-      if (lane == 0 && n > 0) producer<D>(&tq, &tk, &tv, &tdo, p, bh, k0, i0, n, sbase, bars, status, abort_flag);
+      if (lane == 0 && n > 0)
+        producer<D, VARLEN>(&tq, &tk, &tv, &tdo, p, cta, k0, i0, n, sbase, bars, status, abort_flag);
     } else if (warp == 1) {
       if (lane == 0) mma_issuer<D, BF16>(n, sbase, bars, tmem, status, abort_flag);
       __syncwarp();
@@ -564,41 +613,164 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= 12) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsDrain));
-    dq_drain<D>(p, bh, i0, n, bars, tmem, status, abort_flag);
+    dq_drain<D>(p, cta, i0, n, bars, tmem, status, abort_flag);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarFinished));
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    softmax_grad<D, BF16>(p, bh, k0, i0, n, (warp - 4) >> 2, sgen, bars, tmem, status, abort_flag);
+    softmax_grad<D, BF16, VARLEN>(p, cta, k0, i0, n, (warp - 4) >> 2, sgen, bars, tmem, status,
+                                  abort_flag);
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarFinished));
   }
 }
 
+// ---------------------------------------------------------------- packed-batch plan
+// Builds what the packed backward's kernels read (one CTA, before them on the stream):
+// every sequence's token ranges bounds-checked once (a range outside [0, total] or longer
+// than the declared maximum is clamped and reported in the status word, as in the forward
+// plan), its first workspace row (query rows padded to whole 128-row tiles, sequence after
+// sequence; a sequence that would run past the workspace gets no query rows and is
+// reported too), and the (sequence, key tile) items, sequence by sequence, key tiles in
+// order (for a causal sequence, heaviest first).
+constexpr int kPlanThreads = 1024;
+
+__global__ void __launch_bounds__(kPlanThreads) fa_bwd_varlen_plan(const BwdParams p,
+                                                                    int* __restrict__ status) {
+  __shared__ long long warp_q[kPlanThreads / 32];
+  __shared__ int warp_k[kPlanThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (p.B + kPlanThreads - 1) / kPlanThreads;  // sequences per thread
+  const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
+  bool bad = false;
+  long long q_sum = 0;
+  int k_sum = 0;
+  for (int b = b0; b < b1; ++b) {
+    int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+    if (q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Nq || k0 < 0 || k1 < k0 ||
+        k1 > p.total_k || k1 - k0 > p.Nkv) {
+      bad = true;
+      q0 = min(max(q0, 0), p.total_q);
+      q1 = min(max(q1, q0), min(p.total_q, q0 + p.Nq));
+      k0 = min(max(k0, 0), p.total_k);
+      k1 = min(max(k1, k0), min(p.total_k, k0 + p.Nkv));
+    }
+    p.vl_seqs[b] = make_int4(q0, q1 - q0, k0, k1 - k0);
+    q_sum += static_cast<long long>((q1 - q0 + kBQ - 1) / kBQ) * kBQ;
+    k_sum += (k1 - k0 + kBK - 1) / kBK;
+  }
+  // Exclusive prefix sums over the threads (sequence order) of the padded query rows and
+  // the key tiles.
+  long long q_inc = q_sum;
+  int k_inc = k_sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long qn = __shfl_up_sync(0xffffffffu, q_inc, o);
+    const int kn = __shfl_up_sync(0xffffffffu, k_inc, o);
+    if (lane >= o) {
+      q_inc += qn;
+      k_inc += kn;
+    }
+  }
+  if (lane == 31) {
+    warp_q[warp] = q_inc;
+    warp_k[warp] = k_inc;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    long long qt = warp_q[lane];
+    int kt = warp_k[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long qn = __shfl_up_sync(0xffffffffu, qt, o);
+      const int kn = __shfl_up_sync(0xffffffffu, kt, o);
+      if (lane >= o) {
+        qt += qn;
+        kt += kn;
+      }
+    }
+    warp_q[lane] = qt;
+    warp_k[lane] = kt;
+  }
+  __syncthreads();
+  long long q_off = q_inc - q_sum + (warp > 0 ? warp_q[warp - 1] : 0);
+  int k_off = k_inc - k_sum + (warp > 0 ? warp_k[warp - 1] : 0);
+  for (int b = b0; b < b1; ++b) {
+    int4 sq = p.vl_seqs[b];
+    const long long padded = static_cast<long long>((sq.y + kBQ - 1) / kBQ) * kBQ;
+    if (q_off + padded > p.rows_max) {  // overlapping ranges from bad offsets: no rows
+      bad = true;
+      sq.y = 0;
+      p.vl_seqs[b] = sq;
+    }
+    p.vl_qpad[b] = static_cast<int>(min(q_off, p.rows_max));
+    q_off += padded;
+    const int nkt = (sq.w + kBK - 1) / kBK;
+    for (int t = 0; t < nkt; ++t) p.vl_items[k_off + t] = b * p.n_ktiles + t;
+    k_off += nkt;
+  }
+  if (tid == kPlanThreads - 1) {
+    p.vl_qpad[p.B] = static_cast<int>(min(warp_q[31], p.rows_max));
+    *p.vl_count = warp_k[31];
+  }
+  if (bad) atomicOr(status, kStatusBadInput);
+}
+
+// The sequence whose padded workspace rows hold row pr (qpad[0] = 0 <= pr < qpad[B]).
+__device__ __forceinline__ int seq_of_row(const int* __restrict__ qpad, int B, long long pr) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (qpad[mid] <= pr) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// The O / dO / LSE row ([B,H,Nq]: b*h*Nq + q; packed: token * H + h) behind workspace row
+// `row`, or -1 for a padding row (then *in is false past the rows in use).
+template <bool VARLEN>
+__device__ __forceinline__ long long source_row(const BwdParams& p, long long row, bool& in) {
+  if constexpr (!VARLEN) {
+    const long long bh = row / p.nq_pad, q = row - bh * p.nq_pad;
+    return q < p.Nq ? bh * p.Nq + q : -1;
+  } else {
+    const long long h = row / p.rows_max, pr = row - h * p.rows_max;
+    if (pr >= p.vl_qpad[p.B]) {
+      in = false;
+      return -1;
+    }
+    const int b = seq_of_row(p.vl_qpad, p.B, pr);
+    const int4 sq = p.vl_seqs[b];
+    const long long q = pr - p.vl_qpad[b];
+    return q < sq.y ? (sq.x + q) * p.H + h : -1;
+  }
+}
+
 // ---------------------------------------------------------------- prep and dQ conversion
 // Per query row (D/8 threads, 16 bytes of O and dO each): D = dO . O, -LSE * log2(e), and
-// the row's D floats of the dQ accumulator zeroed.  Rows past Nq (padding of the last
-// query tile) get D = 0 and -inf, so their P is 0.
-template <int D, bool BF16>
+// the row's D floats of the dQ accumulator zeroed.  Rows past a sequence's queries
+// (padding of its last query tile) get D = 0 and -inf, so their P is 0.
+template <int D, bool BF16, bool VARLEN>
 __global__ void __launch_bounds__(256)
     fa_bwd_prep(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                 const float* __restrict__ lse, const BwdParams p) {
   constexpr int kTpr = D / 8;          // threads per row
   constexpr int kRpw = 32 / kTpr;      // rows per warp
-  const long long rows = static_cast<long long>(p.BH) * p.nq_pad;
+  const long long rows = VARLEN ? static_cast<long long>(p.H) * p.rows_max
+                                : static_cast<long long>(p.BH) * p.nq_pad;
   const int sub = threadIdx.x & (kTpr - 1);
   const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const long long nw = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
   for (long long base = kRpw * gw; base < rows; base += kRpw * nw) {
     const long long row = base + ((threadIdx.x & 31) / kTpr);
-    const bool in = row < rows;
-    const int bh = in ? static_cast<int>(row / p.nq_pad) : 0;
-    const int q = in ? static_cast<int>(row % p.nq_pad) : 0;
+    bool in = row < rows;
+    const long long src = in ? source_row<VARLEN>(p, row, in) : -1;
     float acc = 0.f;
-    if (in && q < p.Nq) {
-      const size_t e = (static_cast<size_t>(bh) * p.Nq + q) * D + sub * 8;
+    if (src >= 0) {
+      const size_t e = static_cast<size_t>(src) * D + sub * 8;
       const uint4 a = *reinterpret_cast<const uint4*>(o + e);
       const uint4 b = *reinterpret_cast<const uint4*>(dout + e);
       const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -616,7 +788,7 @@ __global__ void __launch_bounds__(256)
     if (!in) continue;
     if (sub == 0) {
       p.delta[row] = acc;
-      p.nlse2[row] = q < p.Nq ? -lse[static_cast<size_t>(bh) * p.Nq + q] * 1.4426950408889634f : -INFINITY;
+      p.nlse2[row] = src >= 0 ? -lse[src] * 1.4426950408889634f : -INFINITY;
     }
     float4* z = reinterpret_cast<float4*>(p.dq_acc + row * D) + sub * 2;
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -625,51 +797,63 @@ __global__ void __launch_bounds__(256)
 }
 
 // dQ = scale * accumulator in the 16-bit type: 8 values (one 16-byte store) per thread per
-// step, grid-stride over the B*H*Nq rows (padding rows of the accumulator are skipped).
-template <int D, bool BF16>
+// step, grid-stride over the accumulator's rows (padding rows are skipped).
+template <int D, bool BF16, bool VARLEN>
 __global__ void __launch_bounds__(256)
     fa_bwd_dq(uint16_t* __restrict__ dq, const BwdParams p) {
-  const long long total = static_cast<long long>(p.BH) * p.Nq * (D / 8);
+  const long long rows = VARLEN ? static_cast<long long>(p.H) * p.rows_max
+                                : static_cast<long long>(p.BH) * p.nq_pad;
+  const long long total = rows * (D / 8);
   for (long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; g < total;
        g += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long row = g / (D / 8);  // bh * Nq + q
+    const long long row = g / (D / 8);
     const int c8 = static_cast<int>(g - row * (D / 8));
-    const long long bh = row / p.Nq, q = row - bh * p.Nq;
-    const float4* src = reinterpret_cast<const float4*>(p.dq_acc + (bh * p.nq_pad + q) * D + 8 * c8);
+    bool in = true;
+    const long long dst = source_row<VARLEN>(p, row, in);
+    if (dst < 0) continue;
+    const float4* src = reinterpret_cast<const float4*>(p.dq_acc + row * D + 8 * c8);
     const float4 a = src[0], b = src[1];
     uint4 w;
     w.x = pack2<BF16>(a.x * p.scale, a.y * p.scale);
     w.y = pack2<BF16>(a.z * p.scale, a.w * p.scale);
     w.z = pack2<BF16>(b.x * p.scale, b.y * p.scale);
     w.w = pack2<BF16>(b.z * p.scale, b.w * p.scale);
-    reinterpret_cast<uint4*>(dq)[g] = w;
+    reinterpret_cast<uint4*>(dq + dst * D)[c8] = w;
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool VARLEN>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& tdo, const void* o, const void* dout, const float* lse,
                      void* dq, const BwdParams& p, int sm_count, int* status, cudaStream_t stream) {
-  auto kern = fa_bwd_sm100<D, BF16>;
+  auto kern = fa_bwd_sm100<D, BF16, VARLEN>;
   const cudaError_t config_err =
       configure_kernel(reinterpret_cast<const void*>(kern), BwdCfg<D>::kAlloc, kRegsLaunch);
   if (config_err != cudaSuccess) return config_err;
-  const long long rows = static_cast<long long>(p.BH) * p.nq_pad;
+  cudaError_t e;
+  if constexpr (VARLEN) {
+    fa_bwd_varlen_plan<<<1, kPlanThreads, 0, stream>>>(p, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const long long rows = VARLEN ? static_cast<long long>(p.H) * p.rows_max
+                                : static_cast<long long>(p.BH) * p.nq_pad;
   long long prep_blocks = (rows + 15) / 16;  // at least 16 rows per 256-thread block
   const long long cap = static_cast<long long>(sm_count) * 16;
   if (prep_blocks > cap) prep_blocks = cap;
   if (prep_blocks < 1) prep_blocks = 1;
-  fa_bwd_prep<D, BF16><<<static_cast<int>(prep_blocks), 256, 0, stream>>>(
+  fa_bwd_prep<D, BF16, VARLEN><<<static_cast<int>(prep_blocks), 256, 0, stream>>>(
       static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse, p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const long long grid = static_cast<long long>(p.BH) * p.n_ktiles;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // Packed: one CTA per (item, head) for the most items there can be (B * n_ktiles).
+  const long long grid = VARLEN ? static_cast<long long>(p.B) * p.n_ktiles * p.H
+                                : static_cast<long long>(p.BH) * p.n_ktiles;
   kern<<<static_cast<int>(grid), kThreads, BwdCfg<D>::kAlloc, stream>>>(tq, tk, tv, tdo, p, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const long long chunks = static_cast<long long>(p.BH) * p.Nq * (D / 8);
-  long long dq_blocks = (chunks + 255) / 256;
+  long long dq_blocks = (rows * (D / 8) + 255) / 256;
   if (dq_blocks > cap) dq_blocks = cap;
-  fa_bwd_dq<D, BF16><<<static_cast<int>(dq_blocks), 256, 0, stream>>>(static_cast<uint16_t*>(dq), p);
+  if (dq_blocks < 1) dq_blocks = 1;
+  fa_bwd_dq<D, BF16, VARLEN><<<static_cast<int>(dq_blocks), 256, 0, stream>>>(
+      static_cast<uint16_t*>(dq), p);
   return cudaGetLastError();
 }
 
@@ -681,12 +865,18 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
                             const CUtensorMap& tdo, const void* o, const void* dout,
                             const float* lse, void* dq, const BwdParams& p, int d, bool bf16,
                             int sm_count, int* status, cudaStream_t stream) {
-  if (d == 128)
-    return bf16 ? launch_t<128, true>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream)
-                : launch_t<128, false>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream);
-  if (d == 64)
-    return bf16 ? launch_t<64, true>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream)
-                : launch_t<64, false>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream);
+#define FA_BWD_CASE(D_, B_, V_)                                                              \
+  if (d == D_ && bf16 == B_ && (p.cu_q != nullptr) == V_)                                     \
+    return launch_t<D_, B_, V_>(tq, tk, tv, tdo, o, dout, lse, dq, p, sm_count, status, stream);
+  FA_BWD_CASE(128, true, false)
+  FA_BWD_CASE(128, false, false)
+  FA_BWD_CASE(64, true, false)
+  FA_BWD_CASE(64, false, false)
+  FA_BWD_CASE(128, true, true)
+  FA_BWD_CASE(128, false, true)
+  FA_BWD_CASE(64, true, true)
+  FA_BWD_CASE(64, false, true)
+#undef FA_BWD_CASE
   return cudaErrorInvalidValue;
 }
 

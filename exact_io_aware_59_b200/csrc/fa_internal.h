@@ -67,6 +67,22 @@ struct BwdParams {
   float* dq_acc;
   void* dk;         // [BH, Nkv, d], the inputs' 16-bit type
   void* dv;
+  // Packed variable-length batches (null cu_q: the [B,H,N,d] layout above).  Then q, o,
+  // dO, dQ are [total_q, H, d], k, v, dK, dV [total_k, H, d] and lse [total_q, H]; Nq and
+  // Nkv are the longest sequences (n_qtiles, n_ktiles taken from them); head h's workspace
+  // rows start at h * rows_max, each sequence's query rows padded to whole 128-row tiles.
+  const int* cu_q;
+  const int* cu_k;
+  int B, H;
+  int total_q, total_k;
+  long long rows_max;
+  // Written by the plan kernel that runs first (workspace): each sequence's (q0, Lq, k0,
+  // Lk) after the bounds checks, its first workspace row (entry B: the rows used), the
+  // (sequence, key tile) items as b * n_ktiles + kt, and their count.
+  int4* vl_seqs;
+  int* vl_qpad;
+  int* vl_items;
+  int* vl_count;
 };
 
 // Work description of one split-KV decode launch.

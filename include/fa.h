@@ -303,6 +303,38 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 /* Bytes of workspace an fa_bwd call with these sizes needs (B*H*ceil(Nq/128)*128*(8+4d)). */
 int fa_bwd_workspace_bytes(int B, int H, int Nq, int d, size_t* bytes);
 
+/*
+ * fa_bwd_varlen -- fa_bwd for a packed batch of sequences of different lengths, the
+ * gradients of fa_fwd_varlen: each sequence is an independent problem ("FlashAttention
+ * 1-2-3" (myaihardware), section "When FlashAttention Doesn't Help"), and its backward
+ * is fa_bwd's ("Flash Attention -- Module 12.3", section "Prefill vs Decode", "Training").
+ *   q, o, dout, dq [total_q, H, d]; k, v, dk, dv [total_k, H, d]; lse [total_q, H] fp32 as
+ *   fa_fwd_varlen writes it; cu_seqlens_q / cu_seqlens_k int32 device arrays [B+1] as for
+ *   fa_fwd_varlen (sequence b: query tokens cu_q[b] .. cu_q[b+1]-1, key tokens cu_k[b] ..
+ *   cu_k[b+1]-1, causal alignment bottom-right per sequence), max_seqlen_q / max_seqlen_k
+ *   bounds on the lengths.  Offsets are checked on the device like fa_fwd_varlen's (a range
+ *   outside [0, total] or longer than the maximum is clamped, sequences whose clamped query
+ *   ranges would overrun the workspace get none, and FA_DEV_BAD_INPUT is set).  Rows of dq
+ *   for tokens outside every sequence, and of dk / dv for keys outside every sequence, are
+ *   not written.
+ *   workspace: caller-owned device memory of at least fa_bwd_varlen_workspace_bytes bytes,
+ *   16-byte aligned, overwritten: per head, total_q + 128 B rows (rounded up to a multiple
+ *   of 128) of the fp32 dQ
+ *   accumulator, -LSE*log2(e) and D, then the plan of the call (sequence records, padded
+ *   row offsets, (sequence, key tile) work items).
+ *   Four kernels on `stream` (plan, prep, main, dQ conversion); no allocation, no
+ *   synchronisation.  Same dtype, alignment, overlap and error rules as fa_bwd.
+ */
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                  size_t workspace_bytes, const int* cu_seqlens_q, const int* cu_seqlens_k, int B,
+                  int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                  float scale, int causal, void* stream, int in_dtype);
+
+/* Bytes of workspace an fa_bwd_varlen call with these sizes needs. */
+int fa_bwd_varlen_workspace_bytes(int B, int H, int total_q, int max_seqlen_k, int d,
+                                  size_t* bytes);
+
 /* Bytes of decode workspace a fa_fwd_decode call with these arguments needs. */
 int fa_decode_workspace_bytes(int B, int H, int Nkv, int d, int num_splits, size_t* bytes);
 

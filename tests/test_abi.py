@@ -161,6 +161,9 @@ calls = {
                                                          64, 16, 4, 8, 0.1, None, 0, 2, 0),
     "fa_bwd": lambda: b.fa_bwd(Q, K, V, O, L, Q + 4096, O + 4096, O + 8192, O + 12288,
                                O + 65536, 128 * 520, 1, 1, 4, 4, 128, 0.1, 0, None, 1),
+    "fa_bwd_varlen": lambda: b.fa_bwd_varlen(Q, K, V, O, L, Q + 4096, O + 4096, O + 8192,
+                                             O + 12288, 6 * A, A, 7 * A, 7 * A + 64, 1, 1, 4, 4,
+                                             4, 4, 128, 0.1, 1, None, 1),
     "fa_quantize_e4m3": lambda: b.fa_quantize_e4m3(Q, 1, 2, 100, 128, O, L, None),
     "fa_fwd_fp8_quant": lambda: b.fa_fwd_fp8_quant(Q, K, V, O, L, 1, 2, 16, 16, 128, 0.1, 1,
                                                    None, 1, 2),
@@ -315,6 +318,41 @@ def test_backward_entry_checks():
     assert binding.fa_bwd_workspace_bytes(1, 1, 64, 64) == 128 * (8 + 4 * 64)
     with pytest.raises(binding.FaError):
         binding.fa_bwd_workspace_bytes(1, 1, 64, 96)
+
+
+def test_backward_varlen_entry_checks():
+    """fa_bwd_varlen refuses bad arguments on the host, before touching any device."""
+    B, H, tq, tk, d = 2, 3, 300, 400, 128
+    rows_max = (tq + 128 * B + 127) // 128 * 128
+    need = H * rows_max * (8 + 4 * d) + 16 + 16 * B + ((4 * (B + 1) + 15) // 16) * 16 + 4 * B * 2
+    assert binding.fa_bwd_varlen_workspace_bytes(B, H, tq, 200, d) == need   # 2 key tiles
+    with pytest.raises(binding.FaError):
+        binding.fa_bwd_varlen_workspace_bytes(B, H, tq, 200, 96)
+    A_ = 1 << 24
+    args = dict(q=A_, k=2 * A_, v=3 * A_, o=4 * A_, lse=5 * A_, do=6 * A_, dq=7 * A_, dk=8 * A_,
+                dv=9 * A_, ws=10 * A_, wsb=need, cq=11 * A_, ck=11 * A_ + 64, B=B, H=H, tq=tq,
+                tk=tk, mq=200, mk=200, d=d, scale=0.1, causal=1, stream=None, dt=1)
+
+    def call(**kw):
+        a = dict(args)
+        a.update(kw)
+        return binding.fa_bwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"],
+                                     a["dk"], a["dv"], a["ws"], a["wsb"], a["cq"], a["ck"], a["B"],
+                                     a["H"], a["tq"], a["tk"], a["mq"], a["mk"], a["d"],
+                                     a["scale"], a["causal"], a["stream"], a["dt"])
+
+    assert call(d=96) == binding.FA_ERR_UNSUPPORTED
+    assert call(cq=None) == binding.FA_ERR_INVALID_ARG
+    assert call(wsb=need - 4) == binding.FA_ERR_INVALID_ARG      # workspace too small
+    assert call(mq=tq + 1) == binding.FA_ERR_INVALID_ARG         # longer than the batch
+    assert call(B=0) == binding.FA_ERR_INVALID_ARG
+    assert call(causal=2) == binding.FA_ERR_INVALID_ARG
+    assert call(dt=2) == binding.FA_ERR_INVALID_ARG
+    assert call(scale=math.inf) == binding.FA_ERR_INVALID_ARG
+    assert call(dk=8 * A_ + 8) == binding.FA_ERR_INVALID_ARG      # misaligned
+    assert call(ck=11 * A_ + 2) == binding.FA_ERR_INVALID_ARG     # misaligned offsets
+    assert call(dq=A_) == binding.FA_ERR_INVALID_ARG              # output overlaps an input
+    assert call(ws=11 * A_ - 64) == binding.FA_ERR_INVALID_ARG    # workspace overlaps cu_seqlens
 
 
 def _declared_param_counts():
