@@ -17,6 +17,7 @@ timed for the line's own "steps":
   fp8q_8k       the same, Q and K quantised on the fly inside the step (fa_fwd_fp8_quant)
   bwd_8k        dQ, dK, dV of the headline shape (fa_bwd; 10*d FLOP per visible pair)
   varlen        a packed causal batch of 16 sequences, lengths log-uniform in [512, 8192]
+  bwd_varlen    the backward of that packed batch (fa_bwd_varlen), 10*d FLOP per visible pair
 Every configuration is timed for the same --steps.  Inputs are resident in HBM when the
 timed region starts; a configuration whose inputs fit in L2 (126 MB) cycles through enough
 copies of them that consecutive steps never find them there.
@@ -572,7 +573,7 @@ def arm_ours(args, ws, rank, local):
         del g, dq, dk, dv, bws
         torch.cuda.empty_cache()
 
-    if want("varlen"):
+    if want("varlen") or want("bwd_varlen"):
         # packed variable-length prefill: a ragged causal batch
         lens = varlen_lengths(16, 512, 8192, 4242)
         Hv, dv_ = 32, 128
@@ -583,12 +584,34 @@ def arm_ours(args, ws, rank, local):
                  vcu.data_ptr(), vcu.data_ptr(), len(lens), Hv, vq.shape[0], vk.shape[0],
                  max(lens), max(lens), dv_, float(dv_ ** -0.5), 1, stream.cuda_stream,
                  binding.FA_BF16, binding.FA_BF16)
-        ms_v, clk_v = timed([lambda: check(binding.fa_fwd_varlen(*vargs), "fa_fwd_varlen")],
-                            args.steps, args.warmup, ws, stream, local)
-        flops_v = sum(4 * dv_ * Hv * causal_pairs(n, n) for n in lens)
-        tf_v = flops_v / (ms_v * 1e-3) / 1e12
-        configs["varlen"] = compact(whole_job_rate(flops_v, ms_v, ws) / 1e12, "TFLOP/s", ms_v,
-                                    args.steps, tf_v / peak_t, tf_v / peak_sus, clk_v)
+        if want("varlen"):
+            ms_v, clk_v = timed([lambda: check(binding.fa_fwd_varlen(*vargs), "fa_fwd_varlen")],
+                                args.steps, args.warmup, ws, stream, local)
+            flops_v = sum(4 * dv_ * Hv * causal_pairs(n, n) for n in lens)
+            tf_v = flops_v / (ms_v * 1e-3) / 1e12
+            configs["varlen"] = compact(whole_job_rate(flops_v, ms_v, ws) / 1e12, "TFLOP/s", ms_v,
+                                        args.steps, tf_v / peak_t, tf_v / peak_sus, clk_v)
+        if want("bwd_varlen"):
+            # the backward of the same packed batch (fa_bwd_varlen), from the forward's O, LSE
+            check(binding.fa_fwd_varlen(*vargs), "fa_fwd_varlen")
+            vg = make_grad_out(1, vq.shape[0], Hv, dv_, torch.bfloat16, 8003, device="cuda")
+            vg = vg.reshape(vq.shape)
+            vdq, vdk, vdv = torch.empty_like(vq), torch.empty_like(vk), torch.empty_like(vv)
+            nvw = binding.fa_bwd_varlen_workspace_bytes(len(lens), Hv, vq.shape[0], max(lens), dv_)
+            vws = torch.empty(nvw, dtype=torch.uint8, device="cuda")
+            bvargs = (vq.data_ptr(), vk.data_ptr(), vv.data_ptr(), vo.data_ptr(), vlse.data_ptr(),
+                      vg.data_ptr(), vdq.data_ptr(), vdk.data_ptr(), vdv.data_ptr(), vws.data_ptr(),
+                      nvw, vcu.data_ptr(), vcu.data_ptr(), len(lens), Hv, vq.shape[0],
+                      vk.shape[0], max(lens), max(lens), dv_, float(dv_ ** -0.5), 1,
+                      stream.cuda_stream, binding.FA_BF16)
+            ms_bv, clk_bv = timed([lambda: check(binding.fa_bwd_varlen(*bvargs), "fa_bwd_varlen")],
+                                  args.steps, args.warmup, ws, stream, local)
+            flops_bv = sum(10 * dv_ * Hv * causal_pairs(n, n) for n in lens)
+            tf_bv = flops_bv / (ms_bv * 1e-3) / 1e12
+            configs["bwd_varlen"] = compact(whole_job_rate(flops_bv, ms_bv, ws) / 1e12, "TFLOP/s",
+                                            ms_bv, args.steps, tf_bv / peak_t, tf_bv / peak_sus,
+                                            clk_bv)
+            del vg, vdq, vdk, vdv, vws
         del vq, vk, vv, vcu, vo, vlse
         torch.cuda.empty_cache()
 
