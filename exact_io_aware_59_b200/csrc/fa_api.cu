@@ -364,6 +364,9 @@ int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse
   long long grid = num_ctas > 0 ? num_ctas : ds->sm_count;
   if (grid > p.n_units) grid = p.n_units;
   if (grid < 1) grid = 1;
+  // Every unit on its own CTA: pair each causal Q tile with its mirror image (about equal
+  // work per unit) instead of its neighbour.
+  if (causal && S == 1 && grid == p.n_units) p.causal = fa::kCausalMirror;
   cudaError_t e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, bf16, o_dtype == FA_F32,
                                      static_cast<int>(grid), ds->status, st, false, part_o,
                                      part_lse);

@@ -188,6 +188,22 @@ __device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u) {
   return x;
 }
 
+// Q tile t (0 or 1) of Q-tile pair `pair`: tiles 2*pair and 2*pair+1, or, in a causal launch
+// whose units all run at once (p.causal == kCausalMirror), tiles pair and n_qtiles-1-pair.
+// Under the causal mask the last tiles of a head see the most keys, so adjacent pairs range
+// from one K/V step to a whole row of them and the heaviest sets the launch's time; a tile
+// paired with its mirror image gives every unit about the same work.  The middle pair of
+// an odd tile count has one tile: t = 1 names tile n_qtiles, past the queries, so nothing
+// is loaded or computed for it.  A separate instantiation (MIRROR) runs such launches, so
+// the pairing costs the others nothing; packed batches and K/V-split launches never use it.
+template <bool MIRROR>
+__device__ __forceinline__ int qtile_of(const PrefillParams& p, int pair, int t) {
+  if (!MIRROR) return 2 * pair + t;
+  if (t == 0) return pair;
+  const int b = p.n_qtiles - 1 - pair;
+  return b > pair ? b : p.n_qtiles;
+}
+
 // Number of K/V tiles Q tile `qtile` of unit x must visit (0 when every row is fully
 // masked or the tile lies past the sequence's queries).
 __device__ __forceinline__ int kv_tiles_for(const PrefillParams& p, const Unit& x, int qtile) {
@@ -240,7 +256,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- producer (TMA)
-template <int D, bool VARLEN, bool QK8, bool SPLIT>
+template <int D, bool VARLEN, bool QK8, bool SPLIT, bool MIRROR>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                          const PrefillParams& p, uint32_t sbase, uint32_t bars, int* status,
                          volatile int* abort_flag) {
@@ -257,7 +273,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     if (!ok || u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
     const int pair = x.pair;
-    int n0 = kv_tiles_for(p, x, 2 * pair), n1 = kv_tiles_for(p, x, 2 * pair + 1);
+    int n0 = kv_tiles_for(p, x, qtile_of<MIRROR>(p, pair, 0)), n1 = kv_tiles_for(p, x, qtile_of<MIRROR>(p, pair, 1));
     int j0 = 0, j1 = max(n0, n1);
     if constexpr (SPLIT) {
       kv_range<SPLIT>(p, x, j1, j0, j1);
@@ -277,7 +293,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     for (int t = 0; t < 2; ++t) {
       if ((t == 0 ? n0 : n1) == 0) continue;
       int c1, c2;
-      tile_coords<VARLEN>(p, x, (2 * pair + t) * BM, true, c1, c2);
+      tile_coords<VARLEN>(p, x, qtile_of<MIRROR>(p, pair, t) * BM, true, c1, c2);
       if constexpr (QK8) {
         tma_load_3d(sbase + C::kQOff + t * C::kQBytes, tq, qf, 0, c1, c2);
       } else {
@@ -357,7 +373,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint6
   }
 }
 
-template <int D, bool BF16, bool VARLEN, bool QK8, bool SPLIT>
+template <int D, bool BF16, bool VARLEN, bool QK8, bool SPLIT, bool MIRROR>
 __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                            int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -389,7 +405,7 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
     if (u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
     // n[t]: the end of tile t's K/V range in this unit (<= j0: nothing to do).
-    int n[2] = {kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)};
+    int n[2] = {kv_tiles_for(p, x, qtile_of<MIRROR>(p, x.pair, 0)), kv_tiles_for(p, x, qtile_of<MIRROR>(p, x.pair, 1))};
     int j0 = 0, j1 = max(n[0], n[1]);
     if constexpr (SPLIT) {
       kv_range<SPLIT>(p, x, j1, j0, j1);
@@ -546,7 +562,7 @@ __device__ __forceinline__ float round_error(float xh) {
 // tile's factor is scale * (its Q tile's scale) * (its K tile's scale).
 // SPLIT: the unit covers part of its pair's K/V range; it writes fp32 O / l and the natural
 // LSE of that part to o / lse, here the partial arrays (the combine kernel forms the result).
-template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN, bool QK8, bool SPLIT>
+template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN, bool QK8, bool SPLIT, bool MIRROR>
 __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t tmem, void* o,
                                  float* lse, int t, int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -578,14 +594,14 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     }
     if (u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
-    const int qtile = 2 * x.pair + t;
+    const int qtile = qtile_of<MIRROR>(p, x.pair, t);
     if (qtile * BM >= x.Lq) continue;
     // This tile visits n_kv K/V tiles from tile j0 on (j0 = 0 unless the K/V range is
     // split); j below counts them from j0.
     int j0 = 0, n_kv = kv_tiles_for(p, x, qtile);
     if constexpr (SPLIT) {
       int j1;
-      kv_range<SPLIT>(p, x, max(kv_tiles_for(p, x, 2 * x.pair), kv_tiles_for(p, x, 2 * x.pair + 1)),
+      kv_range<SPLIT>(p, x, max(kv_tiles_for(p, x, qtile_of<MIRROR>(p, x.pair, 0)), kv_tiles_for(p, x, qtile_of<MIRROR>(p, x.pair, 1))),
                       j0, j1);
       n_kv = max(0, min(j1, n_kv) - j0);
     }
@@ -804,7 +820,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   }
 }
 
-template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT>
+template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT, bool MIRROR>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_prefill_sm100(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, void* __restrict__ o,
@@ -861,9 +877,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
     if (warp == 0) {
-      if (lane == 0) producer<D, VARLEN, QK8, SPLIT>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
+      if (lane == 0) producer<D, VARLEN, QK8, SPLIT, MIRROR>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D, BF16, VARLEN, QK8, SPLIT>(p, sbase, bars, tmem, status, abort_flag);
+      if (lane == 0) mma_issuer<D, BF16, VARLEN, QK8, SPLIT, MIRROR>(p, sbase, bars, tmem, status, abort_flag);
       __syncwarp();
       // Release TMEM once both softmax warpgroups have finished reading it.
       drain_wait(bar_addr(bars, C::kBarDone), 0);
@@ -875,9 +891,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // (Per-tile FP8 scales are positive: they never change the score factor's sign.)
     if (p.scale_log2 < 0.f)
-      softmax_epilogue<D, BF16, OF32, true, VARLEN, QK8, SPLIT>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, true, VARLEN, QK8, SPLIT, MIRROR>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     else
-      softmax_epilogue<D, BF16, OF32, false, VARLEN, QK8, SPLIT>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, false, VARLEN, QK8, SPLIT, MIRROR>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     tc_fence_before();
     mbar_arrive(bar_addr(bars, C::kBarDone));
   }
@@ -1024,12 +1040,12 @@ __global__ void __launch_bounds__(kCombineThreads)
     lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
 }
 
-template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT = false>
+template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT = false, bool MIRROR = false>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                      float* lse, const PrefillParams& p, int grid, int* status,
                      cudaStream_t stream, float* part_o = nullptr, float* part_lse = nullptr) {
   // A split launch writes fp32 partial records whatever the output type.
-  auto kern = fa_prefill_sm100<D, BF16, SPLIT ? false : OF32, VARLEN, QK8, SPLIT>;
+  auto kern = fa_prefill_sm100<D, BF16, SPLIT ? false : OF32, VARLEN, QK8, SPLIT, MIRROR>;
   const cudaError_t config_err =
       configure_kernel(reinterpret_cast<const void*>(kern), PrefillCfg<D>::kAlloc, kRegsLaunch);
   if (config_err != cudaSuccess) return config_err;
@@ -1079,6 +1095,9 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
            : p.n_splits > 1                                                                        \
                ? launch_t<D_, B_, F_, false, false, true>(tq, tk, tv, o, lse, p, grid, status, stream, \
                                                           part_o, part_lse)                        \
+           : p.causal == kCausalMirror                                                            \
+               ? launch_t<D_, B_, F_, false, false, false, true>(tq, tk, tv, o, lse, p, grid, status, \
+                                                                 stream)                            \
                : launch_t<D_, B_, F_, false, false>(tq, tk, tv, o, lse, p, grid, status, stream);
   FA_PREFILL_CASE(128, true, true)
   FA_PREFILL_CASE(128, true, false)
