@@ -115,6 +115,46 @@ def test_quantize_matches_oracle_bitwise(N, dtype):
     assert np.array_equal(codes.cpu().numpy().reshape(6, N, 128), c_ref)
 
 
+def _tiles_of_every_value_up_to(amax_bits, dtype):
+    """[T, 128, 128] tiles of the 16-bit type: for each amax bit pattern a, every
+    non-negative value with bits 0..a (alternate ones negated), 16,383 to a tile, each
+    tile also holding a itself, so that its scale is amax / 448; zeros fill the rest."""
+    tiles = []
+    for a in amax_bits:
+        vals = np.arange(a + 1, dtype=np.uint16)
+        vals[1::2] |= 0x8000
+        for g in range(0, a + 1, 16383):
+            t = np.zeros(16384, dtype=np.uint16)
+            part = vals[g:g + 16383]
+            t[:part.size] = part
+            t[16383] = a
+            tiles.append(t)
+    bits = torch.from_numpy(np.stack(tiles).view(np.int16)).reshape(-1, 128, 128)
+    return bits.view(dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_quantize_every_value_below_sampled_amax(dtype):
+    """The codes of every value at or below a tile's amax, for amax sampled over the whole
+    16-bit range (around the smallest scale, 2^-100, that takes the reciprocal-and-correction
+    quotient; subnormal and largest finite amax), equal the oracle's byte for byte: the
+    oracle divides each element by the scale in fp32."""
+    top = 0x7F7F if dtype == torch.bfloat16 else 0x7BFF
+    rng = np.random.default_rng(1600)
+    fixed = [1, 2, 3, 0x7F, 0x80, 0x0B2A, 0x0400, top]
+    if dtype == torch.bfloat16:
+        fixed += list(range(0x11D8, 0x11E9))       # scale just below and above 2^-100
+    amax_bits = sorted(set(fixed + rng.integers(1, top + 1, 150).tolist()))
+    x = _tiles_of_every_value_up_to(amax_bits, dtype)
+    codes, scales = binding.quantize_e4m3(x.reshape(1, -1, 128, 128).cuda())
+    torch.cuda.synchronize()
+    c_ref, s_ref = oracle.e4m3_quantize_tiles(x)
+    assert np.array_equal(scales.cpu().numpy().reshape(-1), s_ref.reshape(-1))
+    got = codes.cpu().numpy().reshape(c_ref.shape)
+    bad = np.argwhere(got != c_ref)
+    assert bad.size == 0, f"{len(bad)} codes differ, first at tile/row/col {bad[0].tolist()}"
+
+
 def _quant_reference(q, k, v, scale, causal, rows=None):
     B, H, Nq, d = q.shape
     Nkv = k.shape[2]
