@@ -115,6 +115,18 @@ def test_quantize_matches_oracle_bitwise(N, dtype):
     assert np.array_equal(codes.cpu().numpy().reshape(6, N, 128), c_ref)
 
 
+def test_quantize_many_tiles_per_sm_bitwise():
+    """A launch of several waves (48 heads of 4,173 rows: 33 tiles each, the last one 77 rows
+    high, about eleven tiles per SM): scales and codes equal the oracle's byte for byte."""
+    x = randn((4, 12, 4173, 128), 1700, torch.bfloat16, 2.0)
+    x[1, 3, 4096:] *= 1e-3                      # a ragged last tile at another scale
+    codes, scales = binding.quantize_e4m3(x.cuda())
+    torch.cuda.synchronize()
+    c_ref, s_ref = oracle.e4m3_quantize_tiles(x.reshape(48, 4173, 128))
+    assert np.array_equal(scales.cpu().numpy().reshape(s_ref.shape), s_ref)
+    assert np.array_equal(codes.cpu().numpy().reshape(c_ref.shape), c_ref)
+
+
 def _tiles_of_every_value_up_to(amax_bits, dtype):
     """[T, 128, 128] tiles of the 16-bit type: for each amax bit pattern a, every
     non-negative value with bits 0..a (alternate ones negated), 16,383 to a tile, each
