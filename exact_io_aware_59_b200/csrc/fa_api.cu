@@ -362,11 +362,17 @@ int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse
     p.n_splits = 1;
   }
   long long grid = num_ctas > 0 ? num_ctas : ds->sm_count;
+  if (causal && S == 1 && grid >= p.n_units && BH * p.n_qtiles <= 0x7fffffffLL) {
+    // Every Q-tile pair would get its own CTA, so a unit's serial chain of K/V steps sets
+    // the launch's time.  Make each Q tile a unit instead, its even K/V tiles on one
+    // softmax warpgroup and its odd ones on the other (merged at the end): the chain halves
+    // and both warpgroups stay busy; the CTAs take the units heaviest first.
+    p.causal = fa::kCausalKVI;
+    p.n_pairs = p.n_qtiles;
+    p.n_units = static_cast<int>(BH * p.n_qtiles);
+  }
   if (grid > p.n_units) grid = p.n_units;
   if (grid < 1) grid = 1;
-  // Every unit on its own CTA: pair each causal Q tile with its mirror image (about equal
-  // work per unit) instead of its neighbour.
-  if (causal && S == 1 && grid == p.n_units) p.causal = fa::kCausalMirror;
   cudaError_t e = fa::launch_prefill(tq, tk, tv, o, lse, p, d, bf16, o_dtype == FA_F32,
                                      static_cast<int>(grid), ds->status, st, false, part_o,
                                      part_lse);

@@ -8,18 +8,20 @@
 namespace fa {
 
 // Work description of one prefill launch (all sizes in elements / rows / tiles).
-constexpr int kCausalMirror = 2;
+constexpr int kCausalKVI = 2;
 
 struct PrefillParams {
   int BH;           // B * H
   int Nq, Nkv;
   int off;          // Nkv - Nq: causal query i sees keys j <= i + off
-  // 0: no mask; 1: causal; kCausalMirror: causal, and unit i pairs Q tiles i and
-  // n_qtiles-1-i instead of 2i and 2i+1 (launches whose units all run at once, one CTA
-  // each, no K/V split).  Kernels test it for truth except where the pairing is chosen.
+  // 0: no mask; 1: causal; kCausalKVI: causal, and a unit is one Q tile whose even K/V
+  // tiles go to one softmax warpgroup and odd ones to the other, the two partial outputs
+  // merged at the end (small launches, see run_prefill).  Kernels test it for truth except
+  // where the pairing is chosen.
   int causal;
   int n_qtiles;     // ceil(Nq / 128)
   int n_pairs;      // ceil(n_qtiles / 2): a CTA work unit is two consecutive Q tiles
+                    // (n_qtiles with kCausalKVI: a unit is one Q tile)
   int n_kvtiles;    // ceil(Nkv / 128)
   int n_units;      // BH * n_pairs
   float scale_log2; // scale * log2(e)

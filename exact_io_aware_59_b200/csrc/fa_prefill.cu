@@ -69,7 +69,11 @@ struct PrefillCfg {
   static constexpr int kBarDone = kBarDrain + 1;     // softmax warps finished with TMEM
   static constexpr int kBarUnitFull = kBarDone + 1;  // + slot: a claimed unit published
   static constexpr int kBarUnitEmpty = kBarUnitFull + kUnitSlots;  // + slot: read by all
-  static constexpr int kNumBars = kBarUnitEmpty + kUnitSlots;
+  // Interleaved-K/V units: both warpgroups' row statistics published, then both done
+  // reading the two partial outputs (one arrival per softmax warp each).
+  static constexpr int kBarStats = kBarUnitEmpty + kUnitSlots;
+  static constexpr int kBarMerged = kBarStats + 1;
+  static constexpr int kNumBars = kBarMerged + 1;
   static constexpr int kTmemHolderOff = kBarOff + kNumBars * 8;
   static constexpr int kAbortOff = kTmemHolderOff + 4;
   static constexpr int kUnitOff = kAbortOff + 4;     // the claimed-unit ring (packed batches)
@@ -124,6 +128,21 @@ __device__ __forceinline__ int ld_shared_s32(uint32_t addr) {
 
 __device__ __forceinline__ void st_shared_s32(uint32_t addr, int v) {
   asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_shared_f4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
 }
 
 __device__ __forceinline__ int claim_unit(const PrefillParams& p, uint32_t full_bar,
@@ -188,20 +207,16 @@ __device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u) {
   return x;
 }
 
-// Q tile t (0 or 1) of Q-tile pair `pair`: tiles 2*pair and 2*pair+1, or, in a causal launch
-// whose units all run at once (p.causal == kCausalMirror), tiles pair and n_qtiles-1-pair.
-// Under the causal mask the last tiles of a head see the most keys, so adjacent pairs range
-// from one K/V step to a whole row of them and the heaviest sets the launch's time; a tile
-// paired with its mirror image gives every unit about the same work.  The middle pair of
-// an odd tile count has one tile: t = 1 names tile n_qtiles, past the queries, so nothing
-// is loaded or computed for it.  A separate instantiation (MIRROR) runs such launches, so
-// the pairing costs the others nothing; packed batches and K/V-split launches never use it.
-template <bool MIRROR>
+// Q tile t (0 or 1) of Q-tile pair `pair`: tiles 2*pair and 2*pair+1.  In a small causal
+// launch (p.causal == kCausalKVI, instantiation kPairKVI) a unit is one Q tile instead
+// (`pair` names it), shared by both "tiles" t, which take its even (t = 0) and odd (t = 1)
+// K/V tiles: with a CTA per Q-tile pair the heaviest pair's serial chain of K/V steps set
+// the launch's time, and most of its steps had only one tile left.  Packed batches,
+// K/V-split and FP8 launches always pair adjacent tiles.
+constexpr int kPairAdjacent = 0, kPairKVI = 1;
+template <int PAIR>
 __device__ __forceinline__ int qtile_of(const PrefillParams& p, int pair, int t) {
-  if (!MIRROR) return 2 * pair + t;
-  if (t == 0) return pair;
-  const int b = p.n_qtiles - 1 - pair;
-  return b > pair ? b : p.n_qtiles;
+  return PAIR == kPairKVI ? pair : 2 * pair + t;
 }
 
 // Number of K/V tiles Q tile `qtile` of unit x must visit (0 when every row is fully
@@ -256,7 +271,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------- producer (TMA)
-template <int D, bool VARLEN, bool QK8, bool SPLIT, bool MIRROR>
+template <int D, bool VARLEN, bool QK8, bool SPLIT, int PAIR>
 __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUtensorMap* tv,
                          const PrefillParams& p, uint32_t sbase, uint32_t bars, int* status,
                          volatile int* abort_flag) {
@@ -273,7 +288,8 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     if (!ok || u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
     const int pair = x.pair;
-    int n0 = kv_tiles_for(p, x, qtile_of<MIRROR>(p, pair, 0)), n1 = kv_tiles_for(p, x, qtile_of<MIRROR>(p, pair, 1));
+    int n0 = kv_tiles_for(p, x, qtile_of<PAIR>(p, pair, 0)), n1 = kv_tiles_for(p, x, qtile_of<PAIR>(p, pair, 1));
+    if constexpr (PAIR == kPairKVI) n1 = 0;  // one Q tile; its K/V tiles stream in order
     int j0 = 0, j1 = max(n0, n1);
     if constexpr (SPLIT) {
       kv_range<SPLIT>(p, x, j1, j0, j1);
@@ -293,7 +309,7 @@ __device__ void producer(const CUtensorMap* tq, const CUtensorMap* tk, const CUt
     for (int t = 0; t < 2; ++t) {
       if ((t == 0 ? n0 : n1) == 0) continue;
       int c1, c2;
-      tile_coords<VARLEN>(p, x, qtile_of<MIRROR>(p, pair, t) * BM, true, c1, c2);
+      tile_coords<VARLEN>(p, x, qtile_of<PAIR>(p, pair, t) * BM, true, c1, c2);
       if constexpr (QK8) {
         tma_load_3d(sbase + C::kQOff + t * C::kQBytes, tq, qf, 0, c1, c2);
       } else {
@@ -373,7 +389,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint6
   }
 }
 
-template <int D, bool BF16, bool VARLEN, bool QK8, bool SPLIT, bool MIRROR>
+template <int D, bool BF16, bool VARLEN, bool QK8, bool SPLIT, int PAIR>
 __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars, uint32_t tmem,
                            int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -404,8 +420,59 @@ __device__ void mma_issuer(const PrefillParams& p, uint32_t sbase, uint32_t bars
     }
     if (u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
+    if constexpr (PAIR == kPairKVI) {
+      // One Q tile; K/V tile j goes to "tile" j & 1 (its S and O columns).  The ring holds
+      // K_j at index 2j and V_j at 2j + 1 from this unit's first slot on.  Per j: P V_t(j),
+      // then S_t(j + 2), so each warpgroup's next scores are ready while it finishes a tile.
+      const int n = kv_tiles_for(p, x, x.pair);
+      if (n <= 0) continue;
+      if (!wait(C::kBarQFull, q_used & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t base = ld;
+      auto slot = [&](int idx) { return (base + idx) % S; };
+      auto full = [&](int idx) { return wait(C::kBarFull + slot(idx), ((base + idx) / S) & 1); };
+      for (int t = 0; t < 2 && t < n && ok; ++t) {
+        if (!full(2 * t)) { ok = false; break; }
+        tc_fence_after();
+        issue_s<D, QK8>(tmem + t * 128, q_desc(0), k_desc(slot(2 * t)), idesc_s);
+        tc_commit(bar_addr(bars, C::kBarSFull + t));
+        tc_commit(bar_addr(bars, C::kBarEmpty + slot(2 * t)));
+      }
+      if (!ok) break;
+      if (n <= 2) tc_commit(bar_addr(bars, C::kBarQEmpty));  // every S of the unit issued
+      for (int j = 0; j < n && ok; ++j) {
+        const int t = j & 1;
+        const uint32_t vslot = slot(2 * j + 1);
+        if (!full(2 * j + 1)) { ok = false; break; }
+        tc_fence_after();
+        if (!mbar_wait_spin(bar_addr(bars, C::kBarPFull + 2 * t), pcount[t] & 1, status,
+                            abort_flag, kStatusTimeoutMma)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, j >= 2, 0);
+        tc_commit(bar_addr(bars, C::kBarOHalf + t));
+        if (!mbar_wait_spin(bar_addr(bars, C::kBarPFull + 2 * t + 1), pcount[t] & 1, status,
+                            abort_flag, kStatusTimeoutMma)) { ok = false; break; }
+        ++pcount[t];
+        tc_fence_after();
+        issue_pv<D>(tmem + 256 + t * D, tmem + t * 128, v_desc(vslot), idesc_o, true, 1);
+        tc_commit(bar_addr(bars, C::kBarODone + t));
+        if (j + 2 < n) {
+          if (!full(2 * (j + 2))) { ok = false; break; }
+          tc_fence_after();
+          issue_s<D, QK8>(tmem + t * 128, q_desc(0), k_desc(slot(2 * (j + 2))), idesc_s);
+          tc_commit(bar_addr(bars, C::kBarSFull + t));
+          tc_commit(bar_addr(bars, C::kBarEmpty + slot(2 * (j + 2))));
+          if (j + 2 == n - 1) tc_commit(bar_addr(bars, C::kBarQEmpty));  // the unit's last S
+        }
+        tc_commit(bar_addr(bars, C::kBarEmpty + vslot));
+      }
+      if (!ok) break;
+      ld = base + 2 * n;
+      ++q_used;
+      continue;
+    }
     // n[t]: the end of tile t's K/V range in this unit (<= j0: nothing to do).
-    int n[2] = {kv_tiles_for(p, x, qtile_of<MIRROR>(p, x.pair, 0)), kv_tiles_for(p, x, qtile_of<MIRROR>(p, x.pair, 1))};
+    int n[2] = {kv_tiles_for(p, x, qtile_of<PAIR>(p, x.pair, 0)), kv_tiles_for(p, x, qtile_of<PAIR>(p, x.pair, 1))};
     int j0 = 0, j1 = max(n[0], n[1]);
     if constexpr (SPLIT) {
       kv_range<SPLIT>(p, x, j1, j0, j1);
@@ -562,7 +629,7 @@ __device__ __forceinline__ float round_error(float xh) {
 // tile's factor is scale * (its Q tile's scale) * (its K tile's scale).
 // SPLIT: the unit covers part of its pair's K/V range; it writes fp32 O / l and the natural
 // LSE of that part to o / lse, here the partial arrays (the combine kernel forms the result).
-template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN, bool QK8, bool SPLIT, bool MIRROR>
+template <int D, bool BF16, bool OF32, bool NEG, bool VARLEN, bool QK8, bool SPLIT, int PAIR>
 __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t tmem, void* o,
                                  float* lse, int t, int* status, volatile int* abort_flag) {
   using C = PrefillCfg<D>;
@@ -573,6 +640,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   const uint32_t tS = lane_base + t * 128;
   const uint32_t tO = lane_base + 256 + t * D;
   uint32_t s_seen = 0, o_seen = 0;
+  uint32_t kvi_units = 0;  // interleaved-K/V units merged so far (the merge barriers' phase)
   // Warp-uniform result: tcgen05.ld/st below are warp-collective, so a warp never splits
   // on a wait that finished on some lanes and ran out on others.
   auto wait = [&](int b, uint32_t parity) {
@@ -594,14 +662,15 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     }
     if (u >= n_units) break;
     const Unit x = unit_of<VARLEN, SPLIT>(p, u);
-    const int qtile = qtile_of<MIRROR>(p, x.pair, t);
+    const int qtile = qtile_of<PAIR>(p, x.pair, t);
     if (qtile * BM >= x.Lq) continue;
     // This tile visits n_kv K/V tiles from tile j0 on (j0 = 0 unless the K/V range is
     // split); j below counts them from j0.
     int j0 = 0, n_kv = kv_tiles_for(p, x, qtile);
+    if constexpr (PAIR == kPairKVI) n_kv = (n_kv + 1 - t) / 2;  // K/V tiles t, t + 2, ...
     if constexpr (SPLIT) {
       int j1;
-      kv_range<SPLIT>(p, x, max(kv_tiles_for(p, x, qtile_of<MIRROR>(p, x.pair, 0)), kv_tiles_for(p, x, qtile_of<MIRROR>(p, x.pair, 1))),
+      kv_range<SPLIT>(p, x, max(kv_tiles_for(p, x, qtile_of<PAIR>(p, x.pair, 0)), kv_tiles_for(p, x, qtile_of<PAIR>(p, x.pair, 1))),
                       j0, j1);
       n_kv = max(0, min(j1, n_kv) - j0);
     }
@@ -647,7 +716,8 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
       ++s_seen;
       tc_fence_after();
       const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
-      const int lim_c = limit - j * BN;  // columns c <= lim_c are visible for this row
+      // columns c <= lim_c are visible for this row (K/V tile 2j + t with kPairKVI)
+      const int lim_c = limit - (PAIR == kPairKVI ? 2 * j + t : j) * BN;
       const bool full = __all_sync(0xffffffffu, lim_c >= BN - 1);  // warp-uniform path
       uint32_t s[4][32];
 #pragma unroll
@@ -755,6 +825,73 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     // Output row: (b*H + h, row) in [B,H,Nq,d]; (token, h) in the packed [tokens, H, d].
     const size_t orow_i = !VARLEN ? static_cast<size_t>(x.bh) * p.Nq + row
                                   : (static_cast<size_t>(x.q0) + row) * p.H + x.h;
+    if constexpr (PAIR == kPairKVI) {
+      // Both warpgroups hold a partial result of the same rows (O_t relative to their own
+      // reference max m_t).  Merge: m = max(m_0, m_1), a_t = 2^(m_t - m), l = sum a_t l_t,
+      // O = sum a_t O_t / l ("Online softmax", the rule that combines two partial sums).
+      // Each warpgroup publishes (m_t, l_t, l_exact_t, has O_t) in the unused second Q
+      // buffer, then forms half of the columns from both O tiles; warpgroup 0 writes LSE.
+      // The second barrier keeps either O tile from being overwritten by the next unit
+      // before the other warpgroup has read it.
+      const uint32_t stats = bars - C::kBarOff + C::kQOff + C::kQBytes;
+      st_shared_f4(stats + 16u * (t * BM + r), m_used, l, l_exact, n_kv > 0 ? 1.f : 0.f);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarStats));
+      if (!wait(C::kBarStats, kvi_units & 1)) return;
+      tc_fence_after();  // the other warpgroup saw its O tile complete before arriving
+      const float4 ot = ld_shared_f4(stats + 16u * ((1 - t) * BM + r));
+      const bool has_s = n_kv > 0, has_o = ot.w != 0.f;
+      const float ms = has_s ? m_used : -INFINITY, mo = has_o ? ot.x : -INFINITY;
+      const float m = fmaxf(ms, mo);
+      const float as = ms != -INFINITY ? ex2(ms - m) : 0.f;
+      const float ao = mo != -INFINITY ? ex2(mo - m) : 0.f;
+      const float lt = l * as + ot.y * ao, lt_exact = l_exact * as + ot.z * ao;
+      const float inv_lt = (lt > 0.f) ? 1.0f / lt : 0.f;
+      const uint32_t tOs = lane_base + 256 + t * D, tOo = lane_base + 256 + (1 - t) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 64; ++cc) {
+        const int col = t * (D / 2) + cc * 32;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+#pragma unroll 1
+        for (int side = 0; side < 2; ++side) {
+          const bool has = side == 0 ? has_s : has_o;
+          if (!has) continue;
+          uint32_t ob[32];
+          tmem_ld_32x32b_x32((side == 0 ? tOs : tOo) + col, ob);
+          tmem_ld_wait(ob);
+          const float a = side == 0 ? as : ao;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fmaf(__uint_as_float(ob[i]), a, v[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= inv_lt;
+        if (valid) {
+          if constexpr (OF32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(o) + orow_i * D + col);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(o) + orow_i * D + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack2<BF16>(v[8 * i], v[8 * i + 1]), pack2<BF16>(v[8 * i + 2], v[8 * i + 3]),
+                                  pack2<BF16>(v[8 * i + 4], v[8 * i + 5]), pack2<BF16>(v[8 * i + 6], v[8 * i + 7]));
+          }
+        }
+      }
+      if (t == 0 && valid && lse != nullptr)
+        lse[orow_i] = (lt_exact > 0.f) ? (m + log2f(lt_exact)) * 0.69314718055994531f : -INFINITY;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(bars, C::kBarMerged));
+      if (!wait(C::kBarMerged, kvi_units & 1)) return;
+      tc_fence_after();
+      ++kvi_units;
+      continue;
+    }
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
     if constexpr (SPLIT) {
       // This part's record: O / l in fp32 and the natural LSE (-inf: no visible key).
@@ -820,7 +957,7 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
   }
 }
 
-template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT, bool MIRROR>
+template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT, int PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_prefill_sm100(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                      const __grid_constant__ CUtensorMap tv, void* __restrict__ o,
@@ -855,6 +992,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_addr(bars, C::kBarUnitFull + s), 1);
       mbar_init(bar_addr(bars, C::kBarUnitEmpty + s), kUnitReaders);
     }
+    mbar_init(bar_addr(bars, C::kBarStats), 8);   // one arrival per softmax warp
+    mbar_init(bar_addr(bars, C::kBarMerged), 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -877,9 +1016,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsSide));
     if (warp == 0) {
-      if (lane == 0) producer<D, VARLEN, QK8, SPLIT, MIRROR>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
+      if (lane == 0) producer<D, VARLEN, QK8, SPLIT, PAIR>(&tq, &tk, &tv, p, sbase, bars, status, abort_flag);
     } else if (warp == 1) {
-      if (lane == 0) mma_issuer<D, BF16, VARLEN, QK8, SPLIT, MIRROR>(p, sbase, bars, tmem, status, abort_flag);
+      if (lane == 0) mma_issuer<D, BF16, VARLEN, QK8, SPLIT, PAIR>(p, sbase, bars, tmem, status, abort_flag);
       __syncwarp();
       // Release TMEM once both softmax warpgroups have finished reading it.
       drain_wait(bar_addr(bars, C::kBarDone), 0);
@@ -891,9 +1030,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // (Per-tile FP8 scales are positive: they never change the score factor's sign.)
     if (p.scale_log2 < 0.f)
-      softmax_epilogue<D, BF16, OF32, true, VARLEN, QK8, SPLIT, MIRROR>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, true, VARLEN, QK8, SPLIT, PAIR>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     else
-      softmax_epilogue<D, BF16, OF32, false, VARLEN, QK8, SPLIT, MIRROR>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
+      softmax_epilogue<D, BF16, OF32, false, VARLEN, QK8, SPLIT, PAIR>(p, bars, tmem, o, lse, (warp - 4) >> 2, status, abort_flag);
     tc_fence_before();
     mbar_arrive(bar_addr(bars, C::kBarDone));
   }
@@ -1040,12 +1179,12 @@ __global__ void __launch_bounds__(kCombineThreads)
     lse[row] = (wsum > 0.f) ? m + logf(wsum) : -INFINITY;
 }
 
-template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT = false, bool MIRROR = false>
+template <int D, bool BF16, bool OF32, bool VARLEN, bool QK8, bool SPLIT = false, int PAIR = kPairAdjacent>
 cudaError_t launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, void* o,
                      float* lse, const PrefillParams& p, int grid, int* status,
                      cudaStream_t stream, float* part_o = nullptr, float* part_lse = nullptr) {
   // A split launch writes fp32 partial records whatever the output type.
-  auto kern = fa_prefill_sm100<D, BF16, SPLIT ? false : OF32, VARLEN, QK8, SPLIT, MIRROR>;
+  auto kern = fa_prefill_sm100<D, BF16, SPLIT ? false : OF32, VARLEN, QK8, SPLIT, PAIR>;
   const cudaError_t config_err =
       configure_kernel(reinterpret_cast<const void*>(kern), PrefillCfg<D>::kAlloc, kRegsLaunch);
   if (config_err != cudaSuccess) return config_err;
@@ -1095,9 +1234,9 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
            : p.n_splits > 1                                                                        \
                ? launch_t<D_, B_, F_, false, false, true>(tq, tk, tv, o, lse, p, grid, status, stream, \
                                                           part_o, part_lse)                        \
-           : p.causal == kCausalMirror                                                            \
-               ? launch_t<D_, B_, F_, false, false, false, true>(tq, tk, tv, o, lse, p, grid, status, \
-                                                                 stream)                            \
+           : p.causal == kCausalKVI                                                               \
+               ? launch_t<D_, B_, F_, false, false, false, kPairKVI>(tq, tk, tv, o, lse, p, grid,     \
+                                                                     status, stream)                \
                : launch_t<D_, B_, F_, false, false>(tq, tk, tv, o, lse, p, grid, status, stream);
   FA_PREFILL_CASE(128, true, true)
   FA_PREFILL_CASE(128, true, false)

@@ -64,7 +64,8 @@ def test_fp8_16bit_out_peaky():
 @pytest.mark.parametrize("causal", [False, True])
 def test_fp8_equals_bf16_path_on_exact_values(causal):
     """Small integers are exact in E4M3 and bf16 and their dot products are exact in
-    fp32, so S, and with it the whole result, must equal fa_fwd's bit for bit."""
+    fp32, so S, and with it the whole result, must equal fa_fwd's bit for bit (with Q-tile
+    pairs: a one-CTA grid, since the FP8 path always pairs)."""
     B, H, N = 1, 2, 384
     g = torch.Generator().manual_seed(31)
     qi = torch.randint(-3, 4, (B, H, N, 128), generator=g).float()
@@ -75,7 +76,7 @@ def test_fp8_equals_bf16_path_on_exact_values(causal):
     o8, l8 = binding.fp8_attention(q8.cuda(), k8.cuda(), v.cuda(), 1.0, 1.0, causal=causal,
                                    scale=0.02)
     o16, l16 = binding.attention(qi.to(torch.bfloat16).cuda(), ki.to(torch.bfloat16).cuda(),
-                                 v.cuda(), causal=causal, scale=0.02, num_splits=1)
+                                 v.cuda(), causal=causal, scale=0.02, num_ctas=1, num_splits=1)
     torch.cuda.synchronize()
     assert torch.equal(o8, o16) and torch.equal(l8, l16)
 

@@ -96,29 +96,35 @@ def test_persistent_grid_smaller_than_work(num_ctas):
     _run_case(2, 3, 700, 700, 128, torch.bfloat16, True, num_ctas=num_ctas)
 
 
-# A causal launch whose units all get their own CTA pairs Q tile i with tile n-1-i (about
-# equal work per unit); a grid one CTA short of the units pairs neighbours.  The pairing
-# decides which CTA computes a row, not what the row is: both launches must match the
-# oracle and each other bit for bit.  Shapes: odd tile counts (one pair holds a single
-# tile), Nq != Nkv (bottom-right mask), a single query row, the benchmark's d=64 MHA shape.
+# A causal launch whose Q-tile pairs would all get their own CTA makes each Q tile a unit
+# instead, its even K/V tiles on one softmax warpgroup and its odd ones on the other, the two
+# partial results merged at the end.  A grid one CTA short of the pairs runs the ordinary
+# pairs.  Both must match the oracle, and each other within the same tolerance.  A grid of
+# exactly the pair count runs the per-tile units with some CTAs taking two of them.
+# Shapes: odd tile counts, Nq != Nkv (bottom-right mask; rows that see no key), a single
+# query row, a single K/V tile, the benchmark's d=64 MHA shape.
 @pytest.mark.parametrize("shape", [(1, 2, 640, 640, 64, torch.bfloat16),
                                    (2, 3, 1000, 1200, 128, torch.float16),
                                    (1, 3, 773, 773, 128, torch.bfloat16),
                                    (1, 2, 1, 300, 64, torch.bfloat16),
+                                   (1, 2, 900, 200, 64, torch.float16),
+                                   (2, 2, 100, 100, 128, torch.bfloat16),
                                    (2, 8, 2048, 2048, 64, torch.float16)])
-def test_causal_mirrored_pairs(shape):
+def test_causal_small_launch_interleaved_kv(shape):
     B, H, Nq, Nkv, d, dtype = shape
     units = B * H * (((Nq + 127) // 128 + 1) // 2)
     assert units <= torch.cuda.get_device_properties(0).multi_processor_count
     q, k, v = make_qkv(B, H, Nq, Nkv, d, dtype, 21)
     qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
-    o_m, l_m = binding.attention(qc, kc, vc, causal=True, num_ctas=0, num_splits=1)
     o_ref, l_ref = oracle.attention(q, k, v, d ** -0.5, True)
-    compare(o_m, l_m, o_ref, l_ref)
+    o_i, l_i = binding.attention(qc, kc, vc, causal=True, num_ctas=0, num_splits=1)
+    compare(o_i, l_i, o_ref, l_ref)
+    o_g, l_g = binding.attention(qc, kc, vc, causal=True, num_ctas=units, num_splits=1)
+    compare(o_g, l_g, o_ref, l_ref)
     if units > 1:
         o_a, l_a = binding.attention(qc, kc, vc, causal=True, num_ctas=units - 1, num_splits=1)
-        torch.cuda.synchronize()
-        assert torch.equal(o_a, o_m) and torch.equal(l_a, l_m)
+        compare(o_a, l_a, o_ref, l_ref)
+        compare(o_i, l_i, o_a.float().cpu().double().numpy(), l_a.cpu().double().numpy())
 
 
 @pytest.mark.parametrize("num_splits", [1, 2, 3, 4, 7, 64])

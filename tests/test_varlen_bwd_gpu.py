@@ -103,13 +103,15 @@ def test_varlen_backward_queries_and_keys_differ(causal):
 def test_varlen_backward_equal_lengths_is_the_batched_backward():
     """Equal lengths: the same tiles, products and reductions as fa_bwd on the [B,H,N,d]
     layout; dK and dV are summed in a fixed order, so they must agree bit for bit (dQ is
-    summed in arrival order, so only within rounding)."""
+    summed in arrival order, so only within rounding).  The batched forward runs with
+    Q-tile pairs (a one-CTA grid), as the packed forward does, so O and LSE agree too."""
     B, H, L, d = 3, 4, 700, 128
     q, k, v, g, cq, ck = _batch([L] * B, [L] * B, H, d, torch.bfloat16, 2500)
     ours = _run(q, k, v, g, cq, ck, [L] * B, [L] * B, True, 0.1)
     to_b = lambda t: t.reshape(B, L, H, d).permute(0, 2, 1, 3).contiguous().cuda()  # noqa: E731
     qb, kb, vb, gb = (to_b(t) for t in (q, k, v, g))
-    o, lse = binding.attention(qb, kb, vb, causal=True, scale=0.1, out_dtype=torch.bfloat16)
+    o, lse = binding.attention(qb, kb, vb, causal=True, scale=0.1, out_dtype=torch.bfloat16,
+                               num_ctas=1, num_splits=1)
     dqb, dkb, dvb = binding.attention_backward(qb, kb, vb, o, lse, gb, causal=True, scale=0.1)
     torch.cuda.synchronize()
     back = lambda t: t.permute(0, 2, 1, 3).reshape(B * L, H, d).cpu()  # noqa: E731

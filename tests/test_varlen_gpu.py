@@ -65,10 +65,11 @@ def test_varlen_queries_and_keys_differ(causal):
 @pytest.mark.parametrize("causal", [False, True])
 def test_varlen_equal_lengths_is_the_batched_kernel(causal):
     """Equal lengths: the same tiles in the same order as the unsplit prefill on the
-    [B,H,N,d] layout, so the packed call must give the batched call's result bit for bit."""
+    [B,H,N,d] layout with Q-tile pairs (a grid smaller than the pair count), so the packed
+    call must give the batched call's result bit for bit."""
     B, H, L, d = 3, 4, 700, 128
     q, k, v = make_qkv(B, H, L, L, d, torch.bfloat16, 960, device="cuda")
-    o_b, l_b = binding.attention(q, k, v, causal=causal, scale=0.1, num_splits=1)
+    o_b, l_b = binding.attention(q, k, v, causal=causal, scale=0.1, num_ctas=1, num_splits=1)
     pack = lambda x: x.permute(0, 2, 1, 3).reshape(B * L, H, d).contiguous()
     cu = torch.arange(0, (B + 1) * L, L, dtype=torch.int32, device="cuda")
     o_v, l_v = binding.varlen_attention(pack(q), pack(k), pack(v), cu, cu, L, L, causal=causal,
