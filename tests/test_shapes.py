@@ -127,6 +127,14 @@ def test_causal_small_launch_interleaved_kv(shape):
         compare(o_i, l_i, o_a.float().cpu().double().numpy(), l_a.cpu().double().numpy())
 
 
+@pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)])
+def test_interleaved_kv_16bit_output_negative_scale(d, dtype):
+    # the per-tile units' merge and store path with 16-bit output (guard bands around O and
+    # LSE), a negative scale (the row max taken from the minimum score), and a ragged tail
+    _run_case(1, 2, 700, 700, d, dtype, True, out_dtype=dtype, scale=-0.3)
+    _run_case(2, 3, 333, 333, d, dtype, True, out_dtype=dtype)
+
+
 @pytest.mark.parametrize("num_splits", [1, 2, 3, 4, 7, 64])
 @pytest.mark.parametrize("causal", [False, True])
 def test_prefill_kv_split_counts(num_splits, causal):
