@@ -828,7 +828,9 @@ __device__ void softmax_epilogue(const PrefillParams& p, uint32_t bars, uint32_t
     if constexpr (PAIR == kPairKVI) {
       // Both warpgroups hold a partial result of the same rows (O_t relative to their own
       // reference max m_t).  Merge: m = max(m_0, m_1), a_t = 2^(m_t - m), l = sum a_t l_t,
-      // O = sum a_t O_t / l ("Online softmax", the rule that combines two partial sums).
+      // O = sum a_t O_t / l: the rule that combines two partial softmax sums ("FlashAttention
+      // 1-2-3" (myaihardware), sections "The Math Behind the Online Softmax Trick" and
+      // "Beyond FlashAttention", the reduction over K/V splits).
       // Each warpgroup publishes (m_t, l_t, l_exact_t, has O_t) in the unused second Q
       // buffer, then forms half of the columns from both O tiles; warpgroup 0 writes LSE.
       // The second barrier keeps either O tile from being overwritten by the next unit
