@@ -661,10 +661,10 @@ BWD_REV = "backward-v6"
 BWD_TRAFFIC = {("backward-v6", "long_prefill_causal"): 629.2e6}
 
 # Bumped whenever the prefill kernel changes, so stale ncu traffic is not reported.
-KERNEL_REV = "prefill-v23"
+KERNEL_REV = "prefill-v24"
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the
 # kernel at this revision (profiles/fa_prefill_sm100_<workload>.md).
-DRAM_TRAFFIC = {("prefill-v23", "long_prefill_causal"): 600.4e6}
+DRAM_TRAFFIC = {("prefill-v24", "long_prefill_causal"): 583.9e6}
 # The decode kernel's traffic per launch, taken on decode_4k (B16 H32 Nkv4096: 1.0816 GB)
 # and scaled by the keys streamed (x8 for Nkv 32768): the kernel reads each key once.
 DECODE_REV = "decode-v2"
