@@ -277,6 +277,28 @@ double predicted_us(const fa::PrefillParams& p, const int* nmax, int S, int sm_c
   return t;
 }
 
+// Small causal launches left unsplit run interleaved-K/V units (run_prefill): one Q tile
+// per unit, its K/V tiles shared by two warpgroups, so a unit takes ceil(n / 2) steps of
+// two tiles, with no combine launch.  Fitted to B200 timings of 10 shapes (within 11%):
+// 3 steps of fill, drain and merge per unit, 1.34 times the paired kernel's step time.
+double predicted_kvi_us(const fa::PrefillParams& p, int sm_count, int d) {
+  const long long units = static_cast<long long>(p.BH) * p.n_qtiles;
+  const int G = static_cast<int>(std::min<long long>(sm_count, units));
+  double load[1024] = {0.0};
+  long long u = 0;
+  for (int qt = p.n_qtiles - 1; qt >= 0; --qt) {
+    const int steps = (host_kv_tiles(p, qt) + 1) / 2;
+    const double cost = steps > 0 ? steps + 3.0 : 0.3;
+    for (int bh = 0; bh < p.BH; ++bh, ++u) {
+      const long long r = u / G, c = u - r * G;
+      load[(r & 1) ? G - 1 - c : c] += cost;
+    }
+  }
+  double worst = 0.0;
+  for (int c = 0; c < G; ++c) worst = std::max(worst, load[c]);
+  return worst * (d == 128 ? 1.8 : 1.62) * 1.34;
+}
+
 int auto_splits_uncached(const fa::PrefillParams& p, int sm_count, int d) {
   int nmax[1024];
   for (int pair = 0; pair < p.n_pairs; ++pair)
@@ -291,7 +313,12 @@ int auto_splits_uncached(const fa::PrefillParams& p, int sm_count, int d) {
       best = S;
     }
   }
-  return t_best < 0.9 * t1 ? best : 1;
+  const int split = t_best < 0.9 * t1 ? best : 1;
+  // A causal launch may do better unsplit, as interleaved-K/V units (measured: when the
+  // model picks two parts, the units win by 14-21%; from three parts on, the split wins).
+  // The split's predictions run about 8% under its measured times.
+  if (p.causal && split > 1 && predicted_kvi_us(p, sm_count, d) <= 1.08 * t_best) return 1;
+  return split;
 }
 
 // The choice for the last few shapes this thread asked about (the model's loop costs a few

@@ -105,6 +105,12 @@ def test_prefill_split_choice_is_host_arithmetic():
     assert 2 <= ns(1, 1, 16384, 16384, 128, True, 148) <= 8
     # many short units: the split's fixed cost is not worth it
     assert ns(2, 8, 2048, 2048, 64, True, 148) == 1
+    # where the split would take two parts, a causal launch runs unsplit as interleaved-K/V
+    # units instead (no combine launch); from three parts on the split stays
+    assert ns(1, 8, 4096, 4096, 128, True, 148) == 1
+    assert ns(2, 4, 4096, 4096, 64, True, 148) == 1
+    assert ns(1, 2, 8192, 8192, 128, True, 148) >= 3
+    assert ns(1, 4, 4096, 4096, 128, True, 148) >= 3
     # never more parts than K/V tiles
     assert ns(1, 1, 300, 200, 128, False, 148) <= 2
     for args in ((0, 1, 4, 4, 64, 0, 148), (1, 1, 4, 4, 96, 0, 148), (1, 1, 4, 4, 64, 2, 148),
