@@ -277,7 +277,15 @@ double predicted_us(const fa::PrefillParams& p, const int* nmax, int S, int sm_c
   return t;
 }
 
-// Small causal launches left unsplit run interleaved-K/V units (run_prefill): one Q tile
+// Whether an unsplit launch of `pairs` Q-tile pairs on `grid` CTAs runs interleaved-K/V
+// units: a causal one whenever every pair would get its own CTA; a non-causal one (whose
+// pairs all take the same number of steps) only when every Q tile would, since with two
+// units on some CTAs it would gain nothing and pay a merge per unit.
+bool kvi_fits(int causal, int S, long long grid, long long pairs) {
+  return S == 1 && (causal ? grid >= pairs : grid >= 2 * pairs);
+}
+
+// Small launches left unsplit run interleaved-K/V units (run_prefill): one Q tile
 // per unit, its K/V tiles shared by two warpgroups, so a unit takes ceil(n / 2) steps of
 // two tiles, with no combine launch.  Fitted to B200 timings of 10 shapes (within 11%):
 // 3 steps of fill, drain and merge per unit, 1.34 times the paired kernel's step time.
@@ -314,10 +322,13 @@ int auto_splits_uncached(const fa::PrefillParams& p, int sm_count, int d) {
     }
   }
   const int split = t_best < 0.9 * t1 ? best : 1;
-  // A causal launch may do better unsplit, as interleaved-K/V units (measured: when the
-  // model picks two parts, the units win by 14-21%; from three parts on, the split wins).
-  // The split's predictions run about 8% under its measured times.
-  if (p.causal && split > 1 && predicted_kvi_us(p, sm_count, d) <= 1.08 * t_best) return 1;
+  // The launch may do better unsplit, as interleaved-K/V units (measured on causal
+  // launches: when the model picks two parts, the units win by 14-21%; from three parts on,
+  // the split wins).  The split's predictions run about 8% under its measured times.
+  const long long pairs = static_cast<long long>(p.BH) * p.n_pairs;
+  if (split > 1 && kvi_fits(p.causal, 1, sm_count, pairs) &&
+      predicted_kvi_us(p, sm_count, d) <= 1.08 * t_best)
+    return 1;
   return split;
 }
 
@@ -389,12 +400,13 @@ int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse
     p.n_splits = 1;
   }
   long long grid = num_ctas > 0 ? num_ctas : ds->sm_count;
-  if (causal && S == 1 && grid >= p.n_units && BH * p.n_qtiles <= 0x7fffffffLL) {
+  p.kvi = 0;
+  if (kvi_fits(causal, S, grid, p.n_units) && BH * p.n_qtiles <= 0x7fffffffLL) {
     // Every Q-tile pair would get its own CTA, so a unit's serial chain of K/V steps sets
     // the launch's time.  Make each Q tile a unit instead, its even K/V tiles on one
     // softmax warpgroup and its odd ones on the other (merged at the end): the chain halves
     // and both warpgroups stay busy; the CTAs take the units heaviest first.
-    p.causal = fa::kCausalKVI;
+    p.kvi = 1;
     p.n_pairs = p.n_qtiles;
     p.n_units = static_cast<int>(BH * p.n_qtiles);
   }

@@ -8,20 +8,19 @@
 namespace fa {
 
 // Work description of one prefill launch (all sizes in elements / rows / tiles).
-constexpr int kCausalKVI = 2;
 
 struct PrefillParams {
   int BH;           // B * H
   int Nq, Nkv;
   int off;          // Nkv - Nq: causal query i sees keys j <= i + off
-  // 0: no mask; 1: causal; kCausalKVI: causal, and a unit is one Q tile whose even K/V
-  // tiles go to one softmax warpgroup and odd ones to the other, the two partial outputs
-  // merged at the end (small launches, see run_prefill).  Kernels test it for truth except
-  // where the pairing is chosen.
-  int causal;
+  int causal;       // 0: no mask; 1: causal (bottom-right aligned when Nq != Nkv)
+  // 1: interleaved-K/V units: a unit is one Q tile whose even K/V tiles go to one softmax
+  // warpgroup and odd ones to the other, the two partial outputs merged at the end (small
+  // launches, see run_prefill); 0: units are Q-tile pairs.
+  int kvi;
   int n_qtiles;     // ceil(Nq / 128)
   int n_pairs;      // ceil(n_qtiles / 2): a CTA work unit is two consecutive Q tiles
-                    // (n_qtiles with kCausalKVI: a unit is one Q tile)
+                    // (n_qtiles with kvi: a unit is one Q tile)
   int n_kvtiles;    // ceil(Nkv / 128)
   int n_units;      // BH * n_pairs
   float scale_log2; // scale * log2(e)

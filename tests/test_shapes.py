@@ -127,6 +127,30 @@ def test_causal_small_launch_interleaved_kv(shape):
         compare(o_i, l_i, o_a.float().cpu().double().numpy(), l_a.cpu().double().numpy())
 
 
+# Without the causal mask every pair takes the same number of steps, so a non-causal launch
+# runs per-tile interleaved-K/V units only when every Q tile gets its own CTA (a grid of at
+# least twice the pair count); a grid one CTA short of that runs the pairs.
+@pytest.mark.parametrize("shape", [(1, 2, 640, 640, 64, torch.bfloat16),
+                                   (2, 3, 1000, 1200, 128, torch.float16),
+                                   (1, 1, 100, 300, 128, torch.bfloat16),
+                                   (2, 4, 2048, 2048, 64, torch.float16)])
+def test_noncausal_small_launch_interleaved_kv(shape):
+    B, H, Nq, Nkv, d, dtype = shape
+    pairs = B * H * (((Nq + 127) // 128 + 1) // 2)
+    assert 2 * pairs <= torch.cuda.get_device_properties(0).multi_processor_count
+    q, k, v = make_qkv(B, H, Nq, Nkv, d, dtype, 23)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    o_ref, l_ref = oracle.attention(q, k, v, d ** -0.5, False)
+    o_i, l_i = binding.attention(qc, kc, vc, causal=False, num_ctas=0, num_splits=1)
+    compare(o_i, l_i, o_ref, l_ref)
+    o_g, l_g = binding.attention(qc, kc, vc, causal=False, num_ctas=2 * pairs, num_splits=1)
+    torch.cuda.synchronize()
+    assert torch.equal(o_g, o_i) and torch.equal(l_g, l_i)
+    o_a, l_a = binding.attention(qc, kc, vc, causal=False, num_ctas=2 * pairs - 1, num_splits=1)
+    compare(o_a, l_a, o_ref, l_ref)
+    compare(o_i, l_i, o_a.float().cpu().double().numpy(), l_a.cpu().double().numpy())
+
+
 @pytest.mark.parametrize("d,dtype", [(64, torch.float16), (128, torch.bfloat16)])
 def test_interleaved_kv_16bit_output_negative_scale(d, dtype):
     # the per-tile units' merge and store path with 16-bit output (guard bands around O and
