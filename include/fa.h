@@ -94,10 +94,11 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
  * Nq > 1).  num_ctas: persistent CTAs to launch; 0 picks one per SM (and splits the K/V
  * range of small problems as fa_fwd_prefill_split does with num_splits = 0), larger values
  * are clamped to the number of work units and run them unsplit.  A work unit is a pair of
- * 128-row query tiles; in an unsplit causal launch with at least one CTA per pair it is a
- * single query tile whose even and odd key tiles two warpgroups of the CTA take at once
- * (the two partial results merged by their log-sum-exp).  Results do not depend on the
- * grid size within either regime.  Same arguments, layouts and errors as fa_fwd.
+ * 128-row query tiles; in an unsplit launch with at least one CTA per pair (causal) or per
+ * query tile (non-causal) it is a single query tile whose even and odd key tiles two
+ * warpgroups of the CTA take at once (the two partial results merged by their
+ * log-sum-exp).  Results do not depend on the grid size within either regime.  Same
+ * arguments, layouts and errors as fa_fwd.
  */
 int fa_fwd_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                    int H, int Nq, int Nkv, int d, float scale, int causal, void* stream,
