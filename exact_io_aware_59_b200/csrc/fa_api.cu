@@ -400,13 +400,12 @@ int run_prefill(const void* q, const void* k, const void* v, void* o, float* lse
     p.n_splits = 1;
   }
   long long grid = num_ctas > 0 ? num_ctas : ds->sm_count;
-  p.kvi = 0;
   if (kvi_fits(causal, S, grid, p.n_units) && BH * p.n_qtiles <= 0x7fffffffLL) {
     // Every Q-tile pair would get its own CTA, so a unit's serial chain of K/V steps sets
     // the launch's time.  Make each Q tile a unit instead, its even K/V tiles on one
     // softmax warpgroup and its odd ones on the other (merged at the end): the chain halves
     // and both warpgroups stay busy; the CTAs take the units heaviest first.
-    p.kvi = 1;
+    p.n_splits = 0;  // the launch's interleaved-K/V flag
     p.n_pairs = p.n_qtiles;
     p.n_units = static_cast<int>(BH * p.n_qtiles);
   }

@@ -14,13 +14,9 @@ struct PrefillParams {
   int Nq, Nkv;
   int off;          // Nkv - Nq: causal query i sees keys j <= i + off
   int causal;       // 0: no mask; 1: causal (bottom-right aligned when Nq != Nkv)
-  // 1: interleaved-K/V units: a unit is one Q tile whose even K/V tiles go to one softmax
-  // warpgroup and odd ones to the other, the two partial outputs merged at the end (small
-  // launches, see run_prefill); 0: units are Q-tile pairs.
-  int kvi;
   int n_qtiles;     // ceil(Nq / 128)
   int n_pairs;      // ceil(n_qtiles / 2): a CTA work unit is two consecutive Q tiles
-                    // (n_qtiles with kvi: a unit is one Q tile)
+                    // (n_qtiles with interleaved-K/V units: one Q tile)
   int n_kvtiles;    // ceil(Nkv / 128)
   int n_units;      // BH * n_pairs
   float scale_log2; // scale * log2(e)
@@ -31,7 +27,10 @@ struct PrefillParams {
   const int* cu_k;
   int H;            // heads per sequence (bh = b * H + h)
   int total_q, total_k;
-  // K/V split of problems with fewer units than SMs (> 1; else no split): each (b*h,
+  // K/V split of problems with fewer units than SMs (> 1; 1: no split; 0: no split, and
+  // interleaved-K/V units: a unit is one Q tile whose even K/V tiles go to one softmax
+  // warpgroup and odd ones to the other, the two partial outputs merged at the end, for
+  // small launches, see run_prefill): each (b*h,
   // Q-tile pair) becomes n_splits units over consecutive parts of its K/V tile range.  A
   // unit writes its rows' partial output (divided by the part's own row sum) and natural
   // log-sum-exp in fp32 to the kernel's o [n_splits, BH*Nq, d] and lse [n_splits, BH*Nq]

@@ -208,11 +208,11 @@ __device__ __forceinline__ Unit unit_of(const PrefillParams& p, int u) {
 }
 
 // Q tile t (0 or 1) of Q-tile pair `pair`: tiles 2*pair and 2*pair+1.  In a small launch
-// (p.kvi, instantiation kPairKVI) a unit is one Q tile instead (`pair` names it), shared
-// by both "tiles" t, which take its even (t = 0) and odd (t = 1) K/V tiles: with a CTA per
-// Q-tile pair the heaviest pair's serial chain of K/V steps set the launch's time (in a
-// causal launch most of its steps had only one tile left).  Packed batches, K/V-split and
-// FP8 launches always pair adjacent tiles.
+// (p.n_splits == 0, instantiation kPairKVI) a unit is one Q tile instead (`pair` names
+// it), shared by both "tiles" t, which take its even (t = 0) and odd (t = 1) K/V tiles:
+// with a CTA per Q-tile pair the heaviest pair's serial chain of K/V steps set the
+// launch's time (in a causal launch most of its steps had only one tile left).  Packed
+// batches, K/V-split and FP8 launches always pair adjacent tiles.
 constexpr int kPairAdjacent = 0, kPairKVI = 1;
 template <int PAIR>
 __device__ __forceinline__ int qtile_of(const PrefillParams& p, int pair, int t) {
@@ -1236,7 +1236,7 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
            : p.n_splits > 1                                                                        \
                ? launch_t<D_, B_, F_, false, false, true>(tq, tk, tv, o, lse, p, grid, status, stream, \
                                                           part_o, part_lse)                        \
-           : p.kvi                                                                                \
+           : p.n_splits == 0                                                                      \
                ? launch_t<D_, B_, F_, false, false, false, kPairKVI>(tq, tk, tv, o, lse, p, grid,     \
                                                                      status, stream)                \
                : launch_t<D_, B_, F_, false, false>(tq, tk, tv, o, lse, p, grid, status, stream);
